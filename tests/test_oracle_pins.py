@@ -1,0 +1,472 @@
+"""Pins of the oracle against facts fixed outside the oracle itself.
+
+Each test checks one oracle function against a closed form, an invariant of
+the definition, an exhaustive brute force on tiny inputs, or a textbook
+library routine (numpy matmul, torch scaled_dot_product_attention in float64)
+that the oracle does not call.  The cases are chosen so that a plausible
+slip (a dropped ReLU, a wrong sign, a transposed operand, an off-by-one in
+visibility, a wrong GQA group, a wrong tie-break) fails at least one of them.
+
+Definition being pinned (pages cited by title and section):
+  * scores: "Day-0 Adaptation for Massive LLMs ...", section 4(1) Index
+    Selection; "Day-0 Readiness for Trillion-Parameter Models ...", section
+    "Index Selection Path" -- with the adopted formula
+    S[t,b] = sum_h w[t,h] * max(0, q_idx[t,h,:] . kc[page(b),:]).
+  * selection: own block forced, then (score desc, block asc), output
+    ascending logical ids, -1 padded.
+  * attention: exact softmax attention over the selected blocks under the
+    causal valid mask ("Day-0 Adaptation for Massive LLMs ...", 4(3)).
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from oracle.harness import bf16_bits, bits_to_float64, oracle_step
+from dynamic_block_sparse_dsa_b200 import workloads as wk
+
+I64_MIN = np.iinfo(np.int64).min
+
+
+# ----------------------------------------------------------------------------- helpers
+def _single_seq_scores(q_idx, w, kc_pool, table_row, pos, bs):
+    T = q_idx.shape[0]
+    return orc.index_score(np.zeros(T, np.int32), np.asarray(pos, np.int32),
+                           np.asarray(table_row, np.int32)[None, :], bs, kc_pool, q_idx, w)
+
+
+def _rand_int8(rng, shape):
+    return rng.integers(-127, 128, size=shape).astype(np.int8)
+
+
+# ----------------------------------------------------------------------------- scores
+def test_score_hand_worked_example():
+    # 2 indexer heads, idx_dim 4, 3 blocks of 4 tokens, query at position 9
+    # (block 2 is its own block, so all 3 blocks are visible).
+    q = np.array([[[1, 2, 0, -1], [3, 0, 1, 1]]], dtype=np.int8)      # [T=1][H=2][4]
+    w = np.array([[2, 5]], dtype=np.int32)
+    kc = np.array([[1, 1, 1, 1],     # page 0
+                   [0, -2, 4, 1],    # page 1
+                   [-1, 0, 0, 2],    # page 2
+                   [9, 9, 9, 9]],    # page 3 (not referenced)
+                  dtype=np.int8)
+    table = [2, 0, 1]                 # logical block -> page
+    # block 0 -> page 2: head0 = -1+0+0-2 = -3 -> 0 ; head1 = -3+0+0+2 = -1 -> 0 ; S = 0
+    # block 1 -> page 0: head0 = 1+2+0-1 = 2 ; head1 = 3+0+1+1 = 5 ; S = 2*2 + 5*5 = 29
+    # block 2 -> page 1: head0 = 0-4+0-1 = -5 -> 0 ; head1 = 0+0+4+1 = 5 ; S = 5*5 = 25
+    s = _single_seq_scores(q, w, kc, table, [9], 4)
+    assert s[0].tolist() == [0, 29, 25]
+
+
+def test_score_visibility_boundary():
+    rng = np.random.default_rng(1)
+    bs, nb = 4, 6
+    kc = _rand_int8(rng, (nb, 8))
+    q = _rand_int8(rng, (bs * nb, 2, 8))
+    w = rng.integers(0, 17, size=(bs * nb, 2)).astype(np.int32)
+    pos = np.arange(bs * nb)
+    s = _single_seq_scores(q, w, kc, np.arange(nb), pos, bs)
+    for t, p in enumerate(pos):
+        vis = p // bs + 1
+        assert (s[t, :vis] != I64_MIN).all()
+        assert (s[t, vis:] == I64_MIN).all()
+
+
+@pytest.mark.parametrize("a,c", [(3, 5), (-7, 11), (127, 127), (-127, 127), (0, 99)])
+def test_score_closed_form_constant_vectors(a, c):
+    H, D, nb = 3, 64, 2
+    q = np.full((1, H, D), a, dtype=np.int8)
+    kc = np.full((nb, D), c, dtype=np.int8)
+    w = np.array([[4, 0, 16]], dtype=np.int32)
+    s = _single_seq_scores(q, w, kc, [1, 0], [127], 64)
+    expect = (4 + 0 + 16) * max(0, D * a * c)
+    assert s[0].tolist() == [expect, expect]
+
+
+def test_score_relu_split_identity_against_matmul():
+    # relu(x) - relu(-x) = x, so S(kc) - S(-kc) = (sum_h w_h q_h) . kc : a plain
+    # matrix product (numpy) that the oracle never computes.
+    rng = np.random.default_rng(2)
+    H, D, nb, T, bs = 16, 64, 40, 5, 64
+    q = _rand_int8(rng, (T, H, D))
+    w = rng.integers(0, 17, size=(T, H)).astype(np.int32)
+    kc = _rand_int8(rng, (nb, D))
+    perm = rng.permutation(nb)
+    pos = np.full(T, nb * bs - 1)
+    s_pos = _single_seq_scores(q, w, kc, perm, pos, bs)
+    s_neg = _single_seq_scores(q, w, (-kc.astype(np.int16)).astype(np.int8), perm, pos, bs)
+    qbar = np.einsum("th,thd->td", w.astype(np.int64), q.astype(np.int64))
+    lin = qbar @ kc.astype(np.int64)[perm].T
+    assert np.array_equal(s_pos - s_neg, lin)
+    # each term is non-negative and S >= the positive part of the linear term
+    assert (s_pos >= 0).all() and (s_neg >= 0).all()
+
+
+def test_score_one_hot_weights_match_single_head_dot():
+    rng = np.random.default_rng(3)
+    H, D, nb, bs = 4, 64, 9, 64
+    q = _rand_int8(rng, (H, H, D))   # query t uses weight one-hot on head t
+    w = np.eye(H, dtype=np.int32) * 3
+    kc = _rand_int8(rng, (nb, D))
+    s = _single_seq_scores(q, w, kc, np.arange(nb), np.full(H, nb * bs - 1), bs)
+    for t in range(H):
+        dots = kc.astype(np.int64) @ q[t, t].astype(np.int64)
+        assert np.array_equal(s[t], 3 * np.maximum(dots, 0))
+
+
+def test_score_page_permutation_invariance():
+    rng = np.random.default_rng(4)
+    H, D, nb, bs = 4, 64, 20, 64
+    q = _rand_int8(rng, (2, H, D))
+    w = rng.integers(0, 17, size=(2, H)).astype(np.int32)
+    kc_logical = _rand_int8(rng, (nb, D))
+    s0 = _single_seq_scores(q, w, kc_logical, np.arange(nb), [nb * bs - 1] * 2, bs)
+    perm = rng.permutation(nb + 7)[:nb]            # scattered pages in a larger pool
+    pool = _rand_int8(rng, (nb + 7, D))
+    pool[perm] = kc_logical
+    s1 = _single_seq_scores(q, w, pool, perm, [nb * bs - 1] * 2, bs)
+    assert np.array_equal(s0, s1)
+
+
+def test_score_bound_fits_int32_at_config_ranges():
+    # the largest possible score with 16 heads, dim 64, |int8| <= 127, w <= 16
+    H, D = 16, 64
+    q = np.full((1, H, D), 127, dtype=np.int8)
+    kc = np.full((1, D), 127, dtype=np.int8)
+    w = np.full((1, H), 16, dtype=np.int32)
+    s = _single_seq_scores(q, w, kc, [0], [0], 64)
+    assert s[0, 0] == H * 16 * D * 127 * 127 == 264257536 < 2 ** 31
+
+
+# ----------------------------------------------------------------------------- top-k
+def _brute_topk(scores, own, k):
+    """Exhaustive search: the unique (k-1)-subset of the non-own blocks in which
+    every chosen block beats every unchosen one under (score desc, index asc)."""
+    others = list(range(own))
+    if own + 1 <= k:
+        return list(range(own + 1))
+
+    def beats(a, b):
+        return scores[a] > scores[b] or (scores[a] == scores[b] and a < b)
+
+    found = []
+    for sub in itertools.combinations(others, k - 1):
+        rest = [b for b in others if b not in sub]
+        if all(beats(a, b) for a in sub for b in rest):
+            found.append(sorted(sub) + [own])
+    assert len(found) == 1
+    return found[0]
+
+
+def test_topk_brute_force_tiny():
+    rng = np.random.default_rng(5)
+    bs = 4
+    for trial in range(300):
+        nb = int(rng.integers(1, 10))
+        k = int(rng.integers(1, 9))
+        p = int(rng.integers(0, nb * bs))
+        # small value range so ties are frequent
+        sc = rng.integers(0, 4, size=nb).astype(np.int64)
+        own = p // bs
+        sc[own + 1:] = I64_MIN
+        sel, cnt = orc.topk([0], [p], bs, sc[None, :], [k], 8)
+        expect = _brute_topk(sc, own, k)
+        assert cnt[0] == len(expect)
+        assert sel[0, :cnt[0]].tolist() == expect
+        assert (sel[0, cnt[0]:] == -1).all()
+
+
+def test_topk_all_equal_scores_take_lowest_indices():
+    bs, nb, k = 64, 50, 8
+    sc = np.zeros((1, nb), np.int64)
+    sel, cnt = orc.topk([0], [nb * bs - 1], bs, sc, [k], k)
+    assert sel[0].tolist() == list(range(k - 1)) + [nb - 1]
+
+
+def test_topk_explicit_tie_break():
+    bs = 4
+    sc = np.array([[5, 7, 7, 3, 7, 0]], np.int64)        # own block = 5
+    sel, cnt = orc.topk([0], [5 * bs + 2], bs, sc, [3], 4)
+    # two slots besides the own block: the 7s at indices 1 and 2 (lowest first)
+    assert sel[0].tolist() == [1, 2, 5, -1] and cnt[0] == 3
+
+
+def test_topk_own_block_forced_even_if_lowest():
+    bs = 4
+    sc = np.array([[9, 8, 7, 6, -1]], np.int64)           # own block (4) scores lowest
+    sel, _ = orc.topk([0], [4 * bs], bs, sc, [2], 2)
+    assert sel[0].tolist() == [0, 4]
+
+
+def test_topk_k_covers_all_visible():
+    bs = 64
+    sc = np.arange(10, dtype=np.int64)[None, :]
+    sel, cnt = orc.topk([0], [5 * bs + 3], bs, sc, [16], 16)
+    assert cnt[0] == 6 and sel[0, :6].tolist() == list(range(6))
+
+
+# ----------------------------------------------------------------------------- attention
+def _tiny_spec(**kw):
+    base = dict(name="tiny", seq_lens=(37,), n_new=(1,), k_per_seq=(64,), k_max=64,
+                num_q_heads=4, num_kv_heads=2, head_dim=128, num_idx_heads=2, idx_dim=64,
+                block_size=4)
+    base.update(kw)
+    return wk.WorkloadSpec(**base)
+
+
+def _sdpa_dense(q64, k64, v64, allowed):
+    """torch float64 SDPA with a boolean mask [T][n] (True = may attend)."""
+    out = torch.nn.functional.scaled_dot_product_attention(
+        q64, k64, v64, attn_mask=allowed, scale=1.0 / math.sqrt(q64.shape[-1]))
+    return out
+
+
+def _logical_kv(wl, s, upto):
+    """K/V of sequence s for positions 0..upto-1 in logical order: [Hkv][n][D] float64."""
+    bs = wl.spec.block_size
+    table = wl.block_table[s].long()
+    pos = torch.arange(upto)
+    pages = table[pos // bs]
+    k = wl.k_pool[pages, pos % bs]     # [n][Hkv][D]
+    v = wl.v_pool[pages, pos % bs]
+    return k.double().permute(1, 0, 2), v.double().permute(1, 0, 2)
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 2), (8, 1), (6, 3)])
+def test_attention_full_coverage_equals_dense_causal_sdpa(hq, hkv):
+    spec = _tiny_spec(num_q_heads=hq, num_kv_heads=hkv, seq_lens=(37, 23), n_new=(5, 3),
+                      k_per_seq=(64, 64), q_scale=8.0)
+    wl = wk.make_workload(spec, seed=11)
+    res = oracle_step(wl, with_append=False)
+    assert (res["cnt"] == (wl.q_pos.numpy() // 4 + 1)).all()
+    cu = wl.cu_q.tolist()
+    for s in range(2):
+        L = spec.seq_lens[s]
+        k, v = _logical_kv(wl, s, L)
+        group = hq // hkv
+        k = k.repeat_interleave(group, 0)
+        v = v.repeat_interleave(group, 0)
+        ts = range(cu[s], cu[s + 1])
+        q = wl.q[list(ts)].double().permute(1, 0, 2)          # [Hq][n_q][D]
+        pos = wl.q_pos[list(ts)]
+        allowed = torch.arange(L)[None, :] <= pos[:, None].long()
+        ref = _sdpa_dense(q, k, v, allowed).permute(1, 0, 2).numpy()
+        np.testing.assert_allclose(res["out"][cu[s]:cu[s + 1]], ref, rtol=0, atol=1e-12)
+
+
+def test_attention_sparse_matches_masked_sdpa_over_selected_blocks():
+    # K smaller than the visible count: the oracle must equal SDPA with a mask
+    # that admits exactly the tokens of the blocks it selected (gather semantics).
+    spec = _tiny_spec(seq_lens=(61,), n_new=(3,), k_per_seq=(4,), k_max=4, q_scale=8.0)
+    wl = wk.make_workload(spec, seed=12)
+    res = oracle_step(wl, with_append=False)
+    L = 61
+    k, v = _logical_kv(wl, 0, L)
+    k = k.repeat_interleave(2, 0)
+    v = v.repeat_interleave(2, 0)
+    for i in range(3):
+        p = int(wl.q_pos[i])
+        blocks = res["sel"][i, :res["cnt"][i]]
+        tok = torch.arange(L)
+        allowed = torch.isin(tok // 4, torch.as_tensor(blocks)) & (tok <= p)
+        q = wl.q[i].double()[:, None, :]
+        ref = _sdpa_dense(q, k, v, allowed[None, :])[:, 0, :].numpy()
+        np.testing.assert_allclose(res["out"][i], ref, rtol=0, atol=1e-12)
+
+
+def test_attention_v_all_ones_gives_ones():
+    spec = _tiny_spec(seq_lens=(50,), n_new=(2,), k_per_seq=(5,), k_max=8, q_scale=16.0)
+    wl = wk.make_workload(spec, seed=13)
+    wl.v_pool.fill_(1.0)
+    res = oracle_step(wl, with_append=False)
+    np.testing.assert_allclose(res["out"], 1.0, rtol=0, atol=1e-14)
+
+
+def test_attention_single_token_context_returns_v0():
+    spec = _tiny_spec(seq_lens=(1,), n_new=(1,), k_per_seq=(3,), k_max=3)
+    wl = wk.make_workload(spec, seed=14)
+    res = oracle_step(wl, with_append=False)
+    page = int(wl.block_table[0, 0])
+    v0 = wl.v_pool[page, 0].double().repeat_interleave(2, 0).numpy()   # [Hq][D]
+    np.testing.assert_array_equal(res["out"][0], v0)
+    k0 = wl.k_pool[page, 0].double().repeat_interleave(2, 0)
+    logit = (wl.q[0].double() * k0).sum(-1) / math.sqrt(128)
+    np.testing.assert_allclose(res["lse"][0], logit.numpy(), rtol=0, atol=1e-14)
+
+
+def test_attention_zero_query_is_uniform_mean():
+    spec = _tiny_spec(seq_lens=(30,), n_new=(1,), k_per_seq=(3,), k_max=3)
+    wl = wk.make_workload(spec, seed=15)
+    wl.q.zero_()
+    res = oracle_step(wl, with_append=False)
+    p = int(wl.q_pos[0])
+    blocks = res["sel"][0, :res["cnt"][0]]
+    toks = [b * 4 + j for b in blocks for j in range(4) if b * 4 + j <= p]
+    table = wl.block_table[0].long()
+    vs = torch.stack([wl.v_pool[table[t // 4], t % 4] for t in toks]).double()   # [n][Hkv][D]
+    mean = vs.mean(0).repeat_interleave(2, 0).numpy()
+    np.testing.assert_allclose(res["out"][0], mean, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(res["lse"][0], math.log(len(toks)), rtol=0, atol=1e-14)
+
+
+def test_attention_two_token_hand_worked():
+    # context of two tokens, one head, D=128: logits are exactly 0 and ln(3)*... use
+    # q = e0, k0 = 0, k1 = c*e0 so logit1 = c/sqrt(128); v0 = 1, v1 = 2 in every dim.
+    spec = _tiny_spec(seq_lens=(2,), n_new=(1,), k_per_seq=(1,), k_max=1,
+                      num_q_heads=1, num_kv_heads=1)
+    wl = wk.make_workload(spec, seed=16)
+    page = int(wl.block_table[0, 0])
+    wl.q.zero_()
+    wl.q[0, 0, 0] = 1.0
+    wl.k_pool[page, 0].zero_()
+    wl.k_pool[page, 1].zero_()
+    wl.k_pool[page, 1, 0, 0] = 8.0
+    wl.v_pool[page, 0].fill_(1.0)
+    wl.v_pool[page, 1].fill_(2.0)
+    res = oracle_step(wl, with_append=False)
+    l1 = 8.0 / math.sqrt(128)
+    p1 = math.exp(l1) / (1.0 + math.exp(l1))
+    np.testing.assert_allclose(res["out"][0, 0], 1.0 + p1, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(res["lse"][0, 0], math.log(1.0 + math.exp(l1)), rtol=0, atol=1e-15)
+
+
+def test_attention_gqa_group_mapping():
+    spec = _tiny_spec(num_q_heads=6, num_kv_heads=3, seq_lens=(20,), n_new=(1,),
+                      k_per_seq=(2,), k_max=2, q_scale=8.0)
+    wl = wk.make_workload(spec, seed=17)
+    for h in range(3):
+        wl.v_pool[:, :, h, :] = float(h + 1)
+    res = oracle_step(wl, with_append=False)
+    for h in range(6):
+        np.testing.assert_allclose(res["out"][0, h], float(h // 2 + 1), rtol=0, atol=1e-14)
+
+
+def test_attention_page_permutation_bit_identical():
+    spec = _tiny_spec(seq_lens=(45, 17), n_new=(2, 1), k_per_seq=(3, 2), k_max=4, q_scale=8.0)
+    wl = wk.make_workload(spec, seed=18)
+    res0 = oracle_step(wl, with_append=True)
+    # move every page to a new physical slot and rewrite the table to match
+    perm = torch.randperm(spec.num_pages, generator=torch.Generator().manual_seed(3))
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(len(perm))
+    wl2 = wk.make_workload(spec, seed=18)
+    wl2.k_pool = wl.k_pool[inv].clone()
+    wl2.v_pool = wl.v_pool[inv].clone()
+    wl2.kc_pool = wl.kc_pool[inv].clone()
+    bt = wl.block_table.long()
+    wl2.block_table = torch.where(bt >= 0, perm[bt.clamp(min=0)], -1).to(torch.int32)
+    res1 = oracle_step(wl2, with_append=True)
+    assert np.array_equal(res0["sel"], res1["sel"])
+    assert np.array_equal(res0["out"], res1["out"])
+    assert np.array_equal(res0["lse"], res1["lse"])
+
+
+# ----------------------------------------------------------------------------- append
+def test_append_round_trip_and_coarse_key_rule():
+    spec = _tiny_spec(seq_lens=(13, 9), n_new=(6, 1), k_per_seq=(2, 2), k_max=2)
+    wl = wk.make_workload(spec, seed=19)
+    table = wl.block_table.numpy()
+    k_pool = bf16_bits(wl.k_pool).copy()
+    v_pool = bf16_bits(wl.v_pool).copy()
+    kc_pool = wl.kc_pool.numpy().copy()
+    kc_before = kc_pool.copy()
+    seq_lens, cu = wl.seq_lens.numpy(), wl.cu_q.numpy()
+    orc.kv_append(table, seq_lens, cu, bf16_bits(wl.k_new), bf16_bits(wl.v_new), k_pool, v_pool, 4)
+    orc.kc_append(table, seq_lens, cu, wl.kc_new.numpy(), kc_pool, 4)
+    kn, vn = bf16_bits(wl.k_new), bf16_bits(wl.v_new)
+    # sequence 0: 6 new tokens at positions 7..12 -> blocks 1 (pos 7), 2 (8..11), 3 (12)
+    for i, pos in enumerate(range(7, 13)):
+        page = table[0, pos // 4]
+        assert np.array_equal(k_pool[page, pos % 4], kn[i])
+        assert np.array_equal(v_pool[page, pos % 4], vn[i])
+    assert np.array_equal(kc_pool[table[0, 1]], wl.kc_new[0].numpy())   # last new token in block 1
+    assert np.array_equal(kc_pool[table[0, 2]], wl.kc_new[4].numpy())   # position 11
+    assert np.array_equal(kc_pool[table[0, 3]], wl.kc_new[5].numpy())   # position 12
+    assert np.array_equal(kc_pool[table[0, 0]], kc_before[table[0, 0]])  # untouched
+    # sequence 1: one token at position 8 -> block 2
+    assert np.array_equal(kc_pool[table[1, 2]], wl.kc_new[6].numpy())
+
+
+def test_append_batch_equals_one_token_at_a_time():
+    # prefill writes blocks in batch, decode appends token by token: both must
+    # leave the same cache ("Day-0 Readiness ...", section "KV Cache Layout").
+    spec = _tiny_spec(seq_lens=(11,), n_new=(7,), k_per_seq=(2,), k_max=2)
+    wl = wk.make_workload(spec, seed=20)
+    table = wl.block_table.numpy()
+    kn, vn, kcn = bf16_bits(wl.k_new), bf16_bits(wl.v_new), wl.kc_new.numpy()
+    a = [bf16_bits(wl.k_pool).copy(), bf16_bits(wl.v_pool).copy(), wl.kc_pool.numpy().copy()]
+    b = [x.copy() for x in a]
+    orc.kv_append(table, [11], [0, 7], kn, vn, a[0], a[1], 4)
+    orc.kc_append(table, [11], [0, 7], kcn, a[2], 4)
+    for i in range(7):
+        L = 4 + i + 1
+        orc.kv_append(table, [L], [0, 1], kn[i:i + 1], vn[i:i + 1], b[0], b[1], 4)
+        orc.kc_append(table, [L], [0, 1], kcn[i:i + 1], b[2], 4)
+    for x, y in zip(a, b):
+        assert np.array_equal(x, y)
+
+
+def test_append_rejects_bad_page():
+    spec = _tiny_spec(seq_lens=(5,), n_new=(1,), k_per_seq=(1,), k_max=1)
+    wl = wk.make_workload(spec, seed=21)
+    table = wl.block_table.numpy().copy()
+    table[0, 1] = 999
+    k_pool = bf16_bits(wl.k_pool).copy()
+    v_pool = bf16_bits(wl.v_pool).copy()
+    with pytest.raises(ValueError):
+        orc.kv_append(table, [5], [0, 1], bf16_bits(wl.k_new), bf16_bits(wl.v_new), k_pool, v_pool, 4)
+
+
+# ----------------------------------------------------------------------------- whole step
+def test_step_planted_blocks_are_found():
+    # 8 planted blocks per sequence at 3 sigma along the weighted query: most of
+    # them must reach the top-8 selection of a 512-block context.
+    spec = wk.WorkloadSpec("plant", seq_lens=(512 * 64,) * 2, n_new=(1, 1), k_per_seq=(9, 9),
+                           k_max=9, num_q_heads=8, num_kv_heads=1, plant=8)
+    wl = wk.make_workload(spec, seed=22)
+    res = oracle_step(wl, with_append=True)
+    for s in range(2):
+        chosen = set(res["sel"][s, :res["cnt"][s]].tolist())
+        planted = set(wl.planted[s].tolist())
+        assert 511 in chosen
+        assert len(chosen & planted) >= 4
+
+
+def test_bf16_decode_is_exact():
+    vals = torch.tensor([1.0, -2.5, 3.140625, 1e-30, -0.0], dtype=torch.bfloat16)
+    np.testing.assert_array_equal(bits_to_float64(bf16_bits(vals)), vals.double().numpy())
+
+
+# ----------------------------------------------------------------------------- golden fixture
+def test_hand_worked_golden_fixture():
+    import json
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "hand_worked.json")
+    g = json.load(open(path))
+    for c in g["score_cases"]:
+        q = np.array([c["q_idx"]], np.int8)
+        w = np.array([c["w"]], np.int32)
+        s = _single_seq_scores(q, w, np.array(c["kc_pool"], np.int8), c["block_table"],
+                               [c["q_pos"]], c["block_size"])
+        assert s[0].tolist() == c["scores"]
+    for c in g["topk_cases"]:
+        sel, cnt = orc.topk([0], [c["q_pos"]], c["block_size"],
+                            np.array([c["scores"]], np.int64), [c["k"]], c["k_max"])
+        assert sel[0].tolist() == c["sel"] and cnt[0] == c["cnt"]
+    (c,) = g["attention_cases"]
+    spec = _tiny_spec(seq_lens=(2,), n_new=(1,), k_per_seq=(1,), k_max=1,
+                      num_q_heads=1, num_kv_heads=1)
+    wl = wk.make_workload(spec, seed=16)
+    page = int(wl.block_table[0, 0])
+    wl.q.zero_()
+    wl.q[0, 0, 0] = 1.0
+    wl.k_pool[page, :2].zero_()
+    wl.k_pool[page, 1, 0, 0] = 8.0
+    wl.v_pool[page, 0].fill_(1.0)
+    wl.v_pool[page, 1].fill_(2.0)
+    res = oracle_step(wl, with_append=False)
+    np.testing.assert_allclose(res["out"][0, 0], c["out"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(res["lse"][0, 0], c["lse"], rtol=0, atol=1e-14)
