@@ -1,0 +1,370 @@
+#!/usr/bin/env python
+"""Benchmark of the dynamic block-sparse attention hot path on B200.
+
+One step = one pass of the whole hot path over one batch:
+  kv_append (the batch's new tokens) -> index_score -> topk_blocks -> attention.
+Default workload: 1M-context decode (8 sequences x 1,048,576 tokens, Top-K 32
+blocks of 64 tokens, 64 query / 8 KV heads, 16 indexer heads).  The step is
+captured in a CUDA graph; the L2 is flushed (512 MiB write) before every timed
+step and each step is timed with CUDA events on the launching stream.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun every rank runs its own batch (weak scaling, no collective on
+the data path); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn decode tokens/s @1M ctx; achieved HBM GB/s vs ~8 TB/s peak"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 512 << 20
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank float over all ranks (identity when world == 1)."""
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self.period = period_s
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- workload accounting
+def algorithmic_bytes(wl) -> dict:
+    """Bytes the method must move per step (decode roofline): every visible
+    block's coarse key plus the K/V page slices of the selected blocks."""
+    spec = wl.spec
+    idx = 0
+    kv = 0
+    for s in range(spec.num_seqs):
+        for i in range(spec.n_new[s]):
+            p = spec.seq_lens[s] - spec.n_new[s] + i
+            n_vis = p // spec.block_size + 1
+            idx += n_vis * spec.idx_dim
+            k = min(spec.k_per_seq[s], n_vis)
+            kv += k * spec.block_size * spec.num_kv_heads * spec.head_dim * 2 * 2
+    return {"coarse_keys": idx, "kv": kv, "total": idx + kv}
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, world, rank, device):
+    import dynamic_block_sparse_dsa_b200 as dsa
+    from dynamic_block_sparse_dsa_b200 import workloads as wk
+
+    spec = wk.NAMED[args.workload]()
+    wl = wk.make_workload(spec, seed=args.seed + rank, device=device)
+    cache = dsa.PagedKVCache(wl.k_pool, wl.v_pool, wl.kc_pool)
+    seqs = dsa.SeqBatch(wl.block_table, wl.seq_lens)
+    queries = dsa.QueryBatch(wl.cu_q, wl.q_pos)
+    decode = all(n == 1 for n in spec.n_new)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def front(b):
+        dsa.kv_append(cache, seqs, queries.cu_q, wl.k_new, wl.v_new, wl.kc_new, dev_err=err)
+        dsa.index_score(cache, seqs, queries, wl.q_idx, wl.w, 16, scores=b["scores"], dev_err=err)
+        dsa.topk_blocks(seqs, queries, b["scores"], wl.k_per_seq, spec.k_max, sel=b["sel"], cnt=b["cnt"],
+                        dev_err=err)
+
+    def attn(b):
+        if decode:
+            dsa.sparse_attn_decode(cache, seqs, queries, wl.q, b["sel"], b["cnt"], out=b["out"], lse=b["lse"],
+                                   workspace=b["workspace"], dev_err=err)
+        else:
+            dsa.sparse_attn_prefill(cache, seqs, queries, wl.q, b["sel"], b["cnt"], out=b["out"], lse=b["lse"],
+                                    dev_err=err)
+
+    with torch.cuda.stream(stream):
+        bufs = dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
+                        q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=spec.k_max, decode=decode,
+                        dev_err=err)
+    torch.cuda.synchronize(device)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(err.item())} in the first step")
+
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        ev[0].record()
+        front(bufs)
+        ev[1].record()
+        attn(bufs)
+        ev[2].record()
+    torch.cuda.synchronize(device)
+
+    def one_step():
+        with torch.cuda.stream(stream):
+            flush.fill_(1)
+            graph.replay()
+        stream.synchronize()
+        return ev[0].elapsed_time(ev[2]), ev[1].elapsed_time(ev[2])
+
+    for _ in range(args.warmup):
+        one_step()
+    barrier(world)
+    torch.cuda.synchronize(device)
+    step_ms, attn_ms = [], []
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        for _ in range(args.steps):
+            s_ms, a_ms = one_step()
+            step_ms.append(s_ms)
+            attn_ms.append(a_ms)
+    torch.cuda.synchronize(device)
+    barrier(world)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(err.item())} during timing")
+
+    total_s = sum(step_ms) / 1e3
+    total_s_max = max_over_ranks(total_s, world, device)
+    tokens_per_step = spec.total_q
+    value = tokens_per_step * args.steps * world / total_s_max
+    ab = algorithmic_bytes(wl)
+    attn_mean_s = sum(attn_ms) / len(attn_ms) / 1e3
+    step_mean_s = total_s / args.steps
+    peak, peak_kind = _peaks()
+    achieved = ab["kv"] / attn_mean_s / 1e9
+    roofline = {"bound": "hbm", "kernel": "sparse_attn_kernel (decode entry)", "achieved": round(achieved, 1),
+                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                "bytes_per_launch": ab["kv"], "traffic": None}
+    step_gbs = ab["total"] / step_mean_s / 1e9
+    step_roof = {"bytes_per_step": ab["total"], "achieved_gbs": round(step_gbs, 1),
+                 "frac_of_measured": round(step_gbs / peak, 4), "frac_of_8tbs": round(step_gbs / 8000.0, 4)}
+
+    # end to end through the public API with host buffers: inputs H2D from
+    # pinned memory, the four calls launched from Python, output D2H
+    host_in = {k: getattr(wl, k).cpu().pin_memory() for k in ("k_new", "v_new", "kc_new", "q", "q_idx", "w")}
+    dev_in = {k: getattr(wl, k) for k in host_in}
+    host_out = torch.empty(bufs["out"].shape, dtype=bufs["out"].dtype).pin_memory()
+    host_lse = torch.empty(bufs["lse"].shape, dtype=bufs["lse"].dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * host_lse.element_size()
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = []
+    n_e2e = max(3, min(args.steps, 50))
+    for i in range(n_e2e + 2):
+        with torch.cuda.stream(stream):
+            flush.fill_(1)
+            e_s.record()
+            for k, t in host_in.items():
+                dev_in[k].copy_(t, non_blocking=True)
+            dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
+                     q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=spec.k_max, decode=decode,
+                     bufs=bufs, dev_err=err)
+            host_out.copy_(bufs["out"], non_blocking=True)
+            host_lse.copy_(bufs["lse"], non_blocking=True)
+            e_e.record()
+        stream.synchronize()
+        if i >= 2:
+            e2e_ms.append(e_s.elapsed_time(e_e))
+    e2e_total = max_over_ranks(sum(e2e_ms) / 1e3, world, device)
+    e2e = {"value": round(tokens_per_step * len(e2e_ms) * world / e2e_total, 1), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_s_max / args.steps * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16+int8",
+        "data": "synthetic (seeded; N(0,1)/sqrt(128) bf16 q/k/v, uniform int8 indexer, planted blocks)",
+        "config": {"workload": spec.name, "batch_per_gpu": spec.num_seqs, "context": max(spec.seq_lens),
+                   "top_k": spec.k_max, "block_size": spec.block_size,
+                   "heads_q_kv_idx": [spec.num_q_heads, spec.num_kv_heads, spec.num_idx_heads],
+                   "global_batch": spec.num_seqs * world, "parallelism": f"dp{world} (independent sequences)",
+                   "l2": "flushed by a 512 MiB write before every timed step", "graph": "one CUDA graph per step"},
+        "roofline": roofline,
+        "step_roofline": step_roof,
+        "attn_ms_mean": round(attn_mean_s * 1e3, 5),
+        "step_ms_median": round(statistics.median(step_ms), 5),
+        "e2e": e2e,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    return res, wl
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) arm
+def cpu_baseline(wl, budget_s=10.0, max_steps=50):
+    """The oracle as it stands, single-threaded C, on whole steps of the same
+    workload until about ``budget_s`` seconds of oracle time are spent."""
+    from oracle.harness import oracle_step
+    spent, steps = 0.0, 0
+    while steps < max_steps and (spent < budget_s or steps == 0):
+        r = oracle_step(wl)
+        spent += r["seconds"]
+        steps += 1
+    tok = wl.spec.total_q * steps
+    return {"value": round(tok / spent, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{steps} full steps of {wl.spec.name} ({wl.spec.total_q} queries each); "
+                      f"{spent:.1f} s of oracle time (host-side page copies excluded)"}
+
+
+def run_reference(args, world, rank, device):
+    from dynamic_block_sparse_dsa_b200 import workloads as wk
+    from oracle.harness import oracle_step
+    spec = wk.NAMED[args.workload]()
+    wl = wk.make_workload(spec, seed=args.seed, device=device)
+    for _ in range(args.warmup):
+        oracle_step(wl)
+    secs = []
+    for _ in range(args.steps):
+        secs.append(oracle_step(wl)["seconds"])
+    total = sum(secs)
+    value = spec.total_q * args.steps / total
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64+int64",
+            "data": "synthetic (same seeded workload as our arm)",
+            "config": {"workload": spec.name, "batch_per_gpu": spec.num_seqs, "context": max(spec.seq_lens),
+                       "top_k": spec.k_max},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{args.steps} full steps of {spec.name}, single-threaded C oracle"},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode_1m")
+    ap.add_argument("--seed", type=int, default=1003)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = dist_env()
+    if world != args.gpus and world > 1:
+        print(f"warning: WORLD_SIZE={world} but --gpus={args.gpus}", file=sys.stderr)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, world, rank, device)), flush=True)
+        return 0
+
+    init_dist(world, "nccl")
+    res, wl = run_ours(args, world, rank, device)
+    if rank == 0 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        barrier(world)
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

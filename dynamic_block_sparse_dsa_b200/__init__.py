@@ -1,0 +1,236 @@
+"""dynamic_block_sparse_dsa_b200 -- query-driven dynamic block-sparse attention on B200.
+
+Thin Python face of the CUDA library ``libdsa.so`` (C ABI: include/dsa.h).
+The calls keep the C names and only marshal torch tensors (device pointers,
+the current CUDA stream); all of the method runs in the library's kernels:
+
+    kv_append            new tokens -> paged K/V pool + coarse keys
+    index_score          int8 indexer: block scores of each query
+    topk_blocks          own block + Top-(K-1) blocks, ascending logical ids
+    sparse_attn_decode   exact attention over the selected blocks (split-KV)
+    sparse_attn_prefill  same, one CTA per (query, KV head)
+
+Pages followed (cited by title and section): "Day-0 Adaptation for Massive
+LLMs: Overcoming Sparse Attention and MXFP4 Expert Weights", section 4;
+"Day-0 Readiness for Trillion-Parameter Models: Engineering Sparse Attention
+and Expert Weight Compression", sections "Index Selection Path", "KV Cache
+Layout", "Differentiated Adaptation of Prefill and Decode".
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import DsaError, load
+
+__all__ = [
+    "PagedKVCache", "SeqBatch", "QueryBatch", "DsaError", "load",
+    "kv_append", "index_score", "topk_blocks", "sparse_attn_decode", "sparse_attn_prefill",
+    "decode_workspace_size", "step",
+]
+
+BLOCK_SIZE = 64
+HEAD_DIM = 128
+IDX_DIM = 64
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("dynamic_block_sparse_dsa_b200 works on CUDA tensors only (no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _addr(t: torch.Tensor) -> int:
+    """Device address of a tensor, as a plain int (for ctypes struct fields)."""
+    return _ptr(t).value
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _expect(t: torch.Tensor, dtype, name):
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+@dataclass
+class PagedKVCache:
+    """Block-paged pools: k/v bf16 [num_pages][64][num_kv_heads][128], kc int8 [num_pages][64]."""
+    k_pool: torch.Tensor
+    v_pool: torch.Tensor
+    kc_pool: torch.Tensor
+
+    def ctype(self) -> _lib.KvCacheC:
+        _expect(self.k_pool, torch.bfloat16, "k_pool")
+        _expect(self.v_pool, torch.bfloat16, "v_pool")
+        _expect(self.kc_pool, torch.int8, "kc_pool")
+        n, bs, hkv, d = self.k_pool.shape
+        return _lib.KvCacheC(_addr(self.k_pool), _addr(self.v_pool), _addr(self.kc_pool), n, bs, hkv, d,
+                             self.kc_pool.shape[1])
+
+    @property
+    def num_kv_heads(self) -> int:
+        return self.k_pool.shape[2]
+
+
+@dataclass
+class SeqBatch:
+    """block_table int32 [num_seqs][max_blocks]; seq_lens int32 [num_seqs] (after append)."""
+    block_table: torch.Tensor
+    seq_lens: torch.Tensor
+
+    def ctype(self) -> _lib.SeqsC:
+        _expect(self.block_table, torch.int32, "block_table")
+        _expect(self.seq_lens, torch.int32, "seq_lens")
+        ns, mb = self.block_table.shape
+        return _lib.SeqsC(_addr(self.block_table), mb, _addr(self.seq_lens), ns)
+
+
+@dataclass
+class QueryBatch:
+    """cu_q int32 [num_seqs+1] ragged offsets; q_pos int32 [total_q] positions."""
+    cu_q: torch.Tensor
+    q_pos: torch.Tensor
+
+    def ctype(self) -> _lib.QueriesC:
+        _expect(self.cu_q, torch.int32, "cu_q")
+        _expect(self.q_pos, torch.int32, "q_pos")
+        return _lib.QueriesC(_addr(self.cu_q), _addr(self.q_pos), self.q_pos.numel())
+
+    @property
+    def total_q(self) -> int:
+        return self.q_pos.numel()
+
+
+def kv_append(cache: PagedKVCache, seqs: SeqBatch, cu_new: torch.Tensor, k_new: torch.Tensor,
+              v_new: torch.Tensor, kc_new: Optional[torch.Tensor] = None,
+              dev_err: Optional[torch.Tensor] = None, stream=None) -> None:
+    lib = load()
+    c, s = cache.ctype(), seqs.ctype()
+    _lib.check("dsa_kv_append", lib.dsa_kv_append(
+        ctypes.byref(c), ctypes.byref(s), _ptr(cu_new), k_new.shape[0], _ptr(k_new), _ptr(v_new),
+        _ptr(kc_new), _ptr(dev_err), _stream(stream)))
+
+
+def index_score(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, q_idx: torch.Tensor,
+                w: torch.Tensor, w_abs_max: int = 16, scores: Optional[torch.Tensor] = None,
+                dev_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """int32 scores [total_q][max_blocks]; entries past a query's own block are left as given."""
+    lib = load()
+    _expect(q_idx, torch.int8, "q_idx")
+    _expect(w, torch.int32, "w")
+    if scores is None:
+        scores = torch.empty((queries.total_q, seqs.block_table.shape[1]), dtype=torch.int32,
+                             device=q_idx.device)
+    c, s, q = cache.ctype(), seqs.ctype(), queries.ctype()
+    _lib.check("dsa_index_score", lib.dsa_index_score(
+        ctypes.byref(c), ctypes.byref(s), ctypes.byref(q), _ptr(q_idx), _ptr(w), q_idx.shape[1],
+        int(w_abs_max), _ptr(scores), _ptr(dev_err), _stream(stream)))
+    return scores
+
+
+def topk_blocks(seqs: SeqBatch, queries: QueryBatch, scores: torch.Tensor, k_per_seq: torch.Tensor,
+                k_max: int, sel: Optional[torch.Tensor] = None, cnt: Optional[torch.Tensor] = None,
+                dev_err: Optional[torch.Tensor] = None, stream=None):
+    """(sel int32 [total_q][k_max] ascending logical ids, -1 padded; cnt int32 [total_q])."""
+    lib = load()
+    dev = scores.device
+    if sel is None:
+        sel = torch.empty((queries.total_q, k_max), dtype=torch.int32, device=dev)
+    if cnt is None:
+        cnt = torch.empty((queries.total_q,), dtype=torch.int32, device=dev)
+    s, q = seqs.ctype(), queries.ctype()
+    _lib.check("dsa_topk_blocks", lib.dsa_topk_blocks(
+        ctypes.byref(s), ctypes.byref(q), _ptr(scores), _ptr(k_per_seq), int(k_max), _ptr(sel),
+        _ptr(cnt), _ptr(dev_err), _stream(stream)))
+    return sel, cnt
+
+
+def decode_workspace_size(total_q: int, num_q_heads: int, num_kv_heads: int, k_max: int) -> int:
+    return int(load().dsa_sparse_attn_decode_workspace_size(total_q, num_q_heads, num_kv_heads, k_max))
+
+
+def _attn_out(q, out, lse):
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=q.device)
+    return out, lse
+
+
+def sparse_attn_decode(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, q: torch.Tensor,
+                       sel: torch.Tensor, cnt: torch.Tensor, sm_scale: Optional[float] = None,
+                       out=None, lse=None, workspace: Optional[torch.Tensor] = None,
+                       dev_err: Optional[torch.Tensor] = None, stream=None):
+    """(out bf16 [total_q][Hq][128], lse fp32 [total_q][Hq]).  ``workspace`` is a
+    zero-initialised uint8 tensor of decode_workspace_size() bytes (allocated here if None)."""
+    lib = load()
+    _expect(q, torch.bfloat16, "q")
+    k_max = sel.shape[1]
+    out, lse = _attn_out(q, out, lse)
+    if workspace is None:
+        workspace = torch.zeros(decode_workspace_size(queries.total_q, q.shape[1], cache.num_kv_heads, k_max),
+                                dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(q.shape[2]) if sm_scale is None else float(sm_scale)
+    c, s, qq = cache.ctype(), seqs.ctype(), queries.ctype()
+    _lib.check("dsa_sparse_attn_decode", lib.dsa_sparse_attn_decode(
+        ctypes.byref(c), ctypes.byref(s), ctypes.byref(qq), _ptr(q), q.shape[1], _ptr(sel), _ptr(cnt),
+        k_max, scale, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _ptr(dev_err),
+        _stream(stream)))
+    return out, lse
+
+
+def sparse_attn_prefill(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, q: torch.Tensor,
+                        sel: torch.Tensor, cnt: torch.Tensor, sm_scale: Optional[float] = None,
+                        out=None, lse=None, dev_err: Optional[torch.Tensor] = None, stream=None):
+    lib = load()
+    _expect(q, torch.bfloat16, "q")
+    out, lse = _attn_out(q, out, lse)
+    scale = 1.0 / math.sqrt(q.shape[2]) if sm_scale is None else float(sm_scale)
+    c, s, qq = cache.ctype(), seqs.ctype(), queries.ctype()
+    _lib.check("dsa_sparse_attn_prefill", lib.dsa_sparse_attn_prefill(
+        ctypes.byref(c), ctypes.byref(s), ctypes.byref(qq), _ptr(q), q.shape[1], _ptr(sel), _ptr(cnt),
+        sel.shape[1], scale, _ptr(out), _ptr(lse), _ptr(dev_err), _stream(stream)))
+    return out, lse
+
+
+def step(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, *, k_new, v_new, kc_new, q, q_idx, w,
+         k_per_seq, k_max: int, w_abs_max: int = 16, decode: bool = True, bufs: Optional[dict] = None,
+         dev_err: Optional[torch.Tensor] = None, stream=None):
+    """One pass of the hot path: append -> index_score -> topk_blocks -> attention.
+
+    ``bufs`` (optional, reused across calls) holds the scores / sel / cnt /
+    out / lse / workspace tensors; missing ones are allocated.  Returns bufs.
+    """
+    b = {} if bufs is None else bufs
+    T, dev = queries.total_q, q.device
+    if "scores" not in b:
+        b["scores"] = torch.empty((T, seqs.block_table.shape[1]), dtype=torch.int32, device=dev)
+        b["sel"] = torch.empty((T, k_max), dtype=torch.int32, device=dev)
+        b["cnt"] = torch.empty((T,), dtype=torch.int32, device=dev)
+        b["out"] = torch.empty_like(q)
+        b["lse"] = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+        b["workspace"] = torch.zeros(decode_workspace_size(T, q.shape[1], cache.num_kv_heads, k_max),
+                                     dtype=torch.uint8, device=dev)
+    kv_append(cache, seqs, queries.cu_q, k_new, v_new, kc_new, dev_err=dev_err, stream=stream)
+    index_score(cache, seqs, queries, q_idx, w, w_abs_max, scores=b["scores"], dev_err=dev_err, stream=stream)
+    topk_blocks(seqs, queries, b["scores"], k_per_seq, k_max, sel=b["sel"], cnt=b["cnt"], dev_err=dev_err,
+                stream=stream)
+    if decode:
+        sparse_attn_decode(cache, seqs, queries, q, b["sel"], b["cnt"], out=b["out"], lse=b["lse"],
+                           workspace=b["workspace"], dev_err=dev_err, stream=stream)
+    else:
+        sparse_attn_prefill(cache, seqs, queries, q, b["sel"], b["cnt"], out=b["out"], lse=b["lse"],
+                            dev_err=dev_err, stream=stream)
+    return b

@@ -1,0 +1,246 @@
+// dsa_api.cu -- the C ABI (include/dsa.h): host-side validation, workspace
+// sizing and launches on the caller's stream.  No allocation, no host sync.
+#include <climits>
+#include <cstdint>
+
+#include "dsa_kernels.h"
+
+namespace {
+
+using namespace dsa;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cache(const dsa_kv_cache *c) {
+    if (!c || !c->k_pool || !c->v_pool || !c->kc_pool) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(c->k_pool) || !aligned16(c->v_pool) || !aligned16(c->kc_pool)) return DSA_ERR_INVALID_ARG;
+    if (c->num_pages < 1 || c->num_kv_heads < 1) return DSA_ERR_INVALID_ARG;
+    if (c->block_size != kBlockSize || c->head_dim != kHeadDim || c->idx_dim != kIdxDim)
+        return DSA_ERR_UNSUPPORTED;
+    return DSA_OK;
+}
+
+int check_seqs(const dsa_seqs *s) {
+    if (!s || !s->block_table || !s->seq_lens) return DSA_ERR_INVALID_ARG;
+    if (s->num_seqs < 1 || s->max_blocks < 1) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+}
+
+int check_queries(const dsa_queries *q) {
+    if (!q || q->total_q < 0) return DSA_ERR_INVALID_ARG;
+    if (q->total_q > 0 && (!q->cu_q || !q->q_pos)) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// decode workspace: [counters int32 T*Hkv][m,l f32 T*Hq*S*2][O f32 T*Hq*S*128], S <= k_max
+struct DecodeLayout {
+    size_t counters, ml, o, total;
+};
+DecodeLayout decode_layout(int total_q, int hq, int hkv, int splits) {
+    DecodeLayout L;
+    L.counters = 0;
+    L.ml = align_up((size_t)total_q * hkv * sizeof(int32_t), 256);
+    L.o = align_up(L.ml + (size_t)total_q * hq * splits * 2 * sizeof(float), 256);
+    L.total = align_up(L.o + (size_t)total_q * hq * splits * kHeadDim * sizeof(float), 256);
+    return L;
+}
+
+int attn_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                const void *q, int32_t num_q_heads, const int32_t *sel, const int32_t *cnt,
+                int32_t k_max, float sm_scale, void *out, float *lse, int32_t *dev_err, AttnArgs &a) {
+    int rc;
+    if ((rc = check_cache(cache)) || (rc = check_seqs(seqs)) || (rc = check_queries(queries))) return rc;
+    if (queries->total_q > 0 && (!q || !sel || !cnt || !out)) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(sel)) return DSA_ERR_INVALID_ARG;
+    if (k_max < 1 || num_q_heads < 1) return DSA_ERR_INVALID_ARG;
+    if (num_q_heads % cache->num_kv_heads != 0) return DSA_ERR_INVALID_ARG;
+    const int group = num_q_heads / cache->num_kv_heads;
+    if (group > kMaxGroup) return DSA_ERR_UNSUPPORTED;
+    if (!(sm_scale > 0.f)) return DSA_ERR_INVALID_ARG;
+    a = AttnArgs{};
+    a.k_pool = static_cast<const __nv_bfloat16 *>(cache->k_pool);
+    a.v_pool = static_cast<const __nv_bfloat16 *>(cache->v_pool);
+    a.num_pages = cache->num_pages;
+    a.num_kv_heads = cache->num_kv_heads;
+    a.block_table = seqs->block_table;
+    a.max_blocks = seqs->max_blocks;
+    a.seq_lens = seqs->seq_lens;
+    a.num_seqs = seqs->num_seqs;
+    a.cu_q = queries->cu_q;
+    a.q_pos = queries->q_pos;
+    a.total_q = queries->total_q;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.num_q_heads = num_q_heads;
+    a.group = group;
+    a.sel = sel;
+    a.cnt = cnt;
+    a.k_max = k_max;
+    a.scale_log2 = sm_scale * 1.4426950408889634f;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.lse = lse;
+    a.dev_err = dev_err;
+    return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_version(void) { return 100; }
+
+const char *dsa_status_string(int status) {
+    switch (status) {
+        case DSA_OK: return "ok";
+        case DSA_ERR_INVALID_ARG: return "invalid argument";
+        case DSA_ERR_UNSUPPORTED: return "unsupported size";
+        case DSA_ERR_RANGE: return "int32 score range exceeded";
+        case DSA_ERR_WORKSPACE: return "workspace too small";
+        case DSA_ERR_CUDA: return "CUDA error";
+        default: return "unknown status";
+    }
+}
+
+int dsa_kv_append(const dsa_kv_cache *cache, const dsa_seqs *seqs, const int32_t *cu_new,
+                  int32_t total_new, const void *k_new, const void *v_new, const int8_t *kc_new,
+                  int32_t *dev_err, dsa_stream_t stream) {
+    int rc;
+    if ((rc = check_cache(cache)) || (rc = check_seqs(seqs))) return rc;
+    if (total_new < 0) return DSA_ERR_INVALID_ARG;
+    if (total_new == 0) return DSA_OK;
+    if (!cu_new || !k_new || !v_new) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || (kc_new && !aligned16(kc_new))) return DSA_ERR_INVALID_ARG;
+    KvAppendArgs a{};
+    a.k_pool = cache->k_pool;
+    a.v_pool = cache->v_pool;
+    a.kc_pool = cache->kc_pool;
+    a.num_pages = cache->num_pages;
+    a.num_kv_heads = cache->num_kv_heads;
+    a.block_table = seqs->block_table;
+    a.max_blocks = seqs->max_blocks;
+    a.seq_lens = seqs->seq_lens;
+    a.num_seqs = seqs->num_seqs;
+    a.cu_new = cu_new;
+    a.total_new = total_new;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.kc_new = kc_new;
+    a.dev_err = dev_err;
+    return from_cuda(launch_kv_append(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int dsa_index_score(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                    const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads, int32_t w_abs_max,
+                    int32_t *scores, int32_t *dev_err, dsa_stream_t stream) {
+    int rc;
+    if ((rc = check_cache(cache)) || (rc = check_seqs(seqs)) || (rc = check_queries(queries))) return rc;
+    if (num_idx_heads < 1 || w_abs_max < 0) return DSA_ERR_INVALID_ARG;
+    if (num_idx_heads > kMaxIdxHeads) return DSA_ERR_UNSUPPORTED;
+    // |S| <= H * |w| * idx_dim * 128 * 128 must stay below 2^31 for exact int32
+    const long long bound = (long long)num_idx_heads * w_abs_max * kIdxDim * 128LL * 128LL;
+    if (bound >= (1LL << 31)) return DSA_ERR_RANGE;
+    if (queries->total_q == 0) return DSA_OK;
+    if (!q_idx || !w || !scores || !aligned16(q_idx)) return DSA_ERR_INVALID_ARG;
+    IndexScoreArgs a{};
+    a.kc_pool = cache->kc_pool;
+    a.num_pages = cache->num_pages;
+    a.block_table = seqs->block_table;
+    a.max_blocks = seqs->max_blocks;
+    a.seq_lens = seqs->seq_lens;
+    a.num_seqs = seqs->num_seqs;
+    a.cu_q = queries->cu_q;
+    a.q_pos = queries->q_pos;
+    a.total_q = queries->total_q;
+    a.q_idx = q_idx;
+    a.w = w;
+    a.num_idx_heads = num_idx_heads;
+    a.scores = scores;
+    a.dev_err = dev_err;
+    return from_cuda(launch_index_score(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int32_t *scores,
+                    const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt,
+                    int32_t *dev_err, dsa_stream_t stream) {
+    int rc;
+    if ((rc = check_seqs(seqs)) || (rc = check_queries(queries))) return rc;
+    if (k_max < 1) return DSA_ERR_INVALID_ARG;
+    if (queries->total_q == 0) return DSA_OK;
+    if (!scores || !k_per_seq || !sel || !cnt) return DSA_ERR_INVALID_ARG;
+    TopkArgs a{};
+    a.seq_lens = seqs->seq_lens;
+    a.num_seqs = seqs->num_seqs;
+    a.max_blocks = seqs->max_blocks;
+    a.cu_q = queries->cu_q;
+    a.q_pos = queries->q_pos;
+    a.total_q = queries->total_q;
+    a.scores = scores;
+    a.k_per_seq = k_per_seq;
+    a.k_max = k_max;
+    a.sel = sel;
+    a.cnt = cnt;
+    a.dev_err = dev_err;
+    return from_cuda(launch_topk(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t dsa_sparse_attn_decode_workspace_size(int32_t total_q, int32_t num_q_heads, int32_t num_kv_heads,
+                                             int32_t k_max) {
+    if (total_q < 0 || num_q_heads < 1 || num_kv_heads < 1 || k_max < 1) return 0;
+    return decode_layout(total_q, num_q_heads, num_kv_heads, k_max).total;
+}
+
+int dsa_sparse_attn_decode(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                           const void *q, int32_t num_q_heads, const int32_t *sel, const int32_t *cnt,
+                           int32_t k_max, float sm_scale, void *out, float *lse, void *workspace,
+                           size_t workspace_bytes, int32_t *dev_err, dsa_stream_t stream) {
+    AttnArgs a;
+    int rc = attn_common(cache, seqs, queries, q, num_q_heads, sel, cnt, k_max, sm_scale, out, lse, dev_err, a);
+    if (rc) return rc;
+    if (queries->total_q == 0) return DSA_OK;
+    // split each query's selection so that (query, KV head, split) CTAs fill
+    // about two waves of the SMs
+    const long long per_split = (long long)queries->total_q * cache->num_kv_heads;
+    long long want = (2LL * sm_count() + per_split - 1) / per_split;
+    if (want < 1) want = 1;
+    if (want > k_max) want = k_max;
+    const int bps = (int)((k_max + want - 1) / want);
+    const int splits = (k_max + bps - 1) / bps;
+    a.n_splits = splits;
+    a.blocks_per_split = bps;
+    if (splits > 1) {
+        const DecodeLayout L = decode_layout(queries->total_q, num_q_heads, cache->num_kv_heads, splits);
+        if (!workspace || !aligned16(workspace) ||
+            workspace_bytes < dsa_sparse_attn_decode_workspace_size(queries->total_q, num_q_heads,
+                                                                    cache->num_kv_heads, k_max))
+            return DSA_ERR_WORKSPACE;
+        char *ws = static_cast<char *>(workspace);
+        a.counters = reinterpret_cast<int32_t *>(ws + L.counters);
+        a.part_ml = reinterpret_cast<float *>(ws + L.ml);
+        a.part_o = reinterpret_cast<float *>(ws + L.o);
+    }
+    return from_cuda(launch_sparse_attn(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int dsa_sparse_attn_prefill(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                            const void *q, int32_t num_q_heads, const int32_t *sel, const int32_t *cnt,
+                            int32_t k_max, float sm_scale, void *out, float *lse, int32_t *dev_err,
+                            dsa_stream_t stream) {
+    AttnArgs a;
+    int rc = attn_common(cache, seqs, queries, q, num_q_heads, sel, cnt, k_max, sm_scale, out, lse, dev_err, a);
+    if (rc) return rc;
+    if (queries->total_q == 0) return DSA_OK;
+    a.n_splits = 1;
+    a.blocks_per_split = k_max;
+    return from_cuda(launch_sparse_attn(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

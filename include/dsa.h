@@ -1,0 +1,198 @@
+/*
+ * dsa.h -- C ABI of the B200 (sm_100a) library for query-driven dynamic
+ * block-sparse attention over a block-paged KV cache.
+ *
+ * The pipeline follows the pages' statement of the problem:
+ *   append new tokens -> score every visible KV block with a low-precision
+ *   indexer -> keep the Top-K blocks (own block forced) -> exact attention over
+ *   the selected blocks only, with separate decode and prefill paths.
+ * Pages (cited by title and section):
+ *   [P1] "Day-0 Adaptation for Massive LLMs: Overcoming Sparse Attention and
+ *        MXFP4 Expert Weights", section 4 (1) Index Selection, (2) KV Cache
+ *        Layout, (3) Prefill and Decode (decode schematic: select, gather by
+ *        block, attend under a valid mask).
+ *   [P3] "Day-0 Adaptation for Trillion-Parameter Models: Engineering
+ *        Practices and Technical Breakdown", section 4 (4.1 index selection,
+ *        4.2 KV cache layout, 4.3 dual prefill / decode paths).
+ *   [P5] "Day-0 Readiness for Trillion-Parameter Models: Engineering Sparse
+ *        Attention and Expert Weight Compression", sections "Index Selection
+ *        Path", "KV Cache Layout", "Differentiated Adaptation of Prefill and
+ *        Decode".
+ *
+ * Conventions shared by every entry point
+ *  - Every array pointer is DEVICE memory owned by the caller, 16-byte
+ *    aligned.  The library never allocates or frees device memory.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  Host-side validation is synchronous: a non-zero
+ *    status means nothing was launched.
+ *  - Kernels never trap.  A fault they detect in device-resident metadata
+ *    (a page id outside the pool, a position outside its sequence, a
+ *    selection outside the visible range) ORs a DSA_DEV_ERR_* bit into
+ *    *dev_err (an int32 in device memory, may be NULL to ignore) and the
+ *    offending item is skipped; the caller reads the word back when it likes.
+ *  - Sizes in v1: block_size 64, head_dim 128, idx_dim 64; query heads per KV
+ *    head 1..16; indexer heads 1..16.  Anything else is DSA_ERR_UNSUPPORTED.
+ *
+ * KV cache layout [P5 "KV Cache Layout"; P1 4(2) two storage types]:
+ *   k_pool, v_pool : bf16  [num_pages][block_size][num_kv_heads][head_dim]
+ *   kc_pool        : int8  [num_pages][idx_dim]  one coarse key per block
+ *   block_table    : int32 [num_seqs][max_blocks] logical block -> page
+ *
+ * Queries are ragged: sequence s owns queries cu_q[s] .. cu_q[s+1]-1, query t
+ * sits at position q_pos[t] (< seq_lens[s]).  A query sees the logical
+ * blocks 0 .. q_pos[t]/block_size ("visible blocks"); the last of them is its
+ * own block.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t without pulling in the CUDA headers */
+typedef struct CUstream_st *dsa_stream_t;
+
+/* host-side status codes */
+enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1, /* NULL / misaligned pointer, negative or inconsistent size */
+    DSA_ERR_UNSUPPORTED = 2, /* a size this version does not implement (see above) */
+    DSA_ERR_RANGE = 3,       /* int32 scores could overflow for the stated |w| bound */
+    DSA_ERR_WORKSPACE = 4,   /* workspace NULL or smaller than the size query says */
+    DSA_ERR_CUDA = 5         /* a CUDA runtime call failed (launch or attribute) */
+};
+
+/* device-side error bits ORed into *dev_err */
+#define DSA_DEV_ERR_PAGE 1u  /* block_table entry outside [0, num_pages) */
+#define DSA_DEV_ERR_POS 2u   /* position / new-token count outside the sequence or table */
+#define DSA_DEV_ERR_SEL 4u   /* selected block id outside the query's visible blocks */
+#define DSA_DEV_ERR_K 8u     /* k_per_seq[s] outside [1, k_max] */
+#define DSA_DEV_ERR_WAIT 16u /* a bounded in-kernel wait gave up (work of that unit skipped) */
+
+typedef struct {
+    void *k_pool;          /* bf16 [num_pages][block_size][num_kv_heads][head_dim] */
+    void *v_pool;          /* bf16, same shape */
+    int8_t *kc_pool;       /* int8 [num_pages][idx_dim] */
+    int32_t num_pages;
+    int32_t block_size;    /* 64 */
+    int32_t num_kv_heads;
+    int32_t head_dim;      /* 128 */
+    int32_t idx_dim;       /* 64 */
+} dsa_kv_cache;
+
+typedef struct {
+    const int32_t *block_table; /* [num_seqs][max_blocks]; entries past a sequence's end are never read */
+    int32_t max_blocks;
+    const int32_t *seq_lens;    /* [num_seqs] context length INCLUDING any tokens appended this step */
+    int32_t num_seqs;
+} dsa_seqs;
+
+typedef struct {
+    const int32_t *cu_q;   /* [num_seqs + 1] ragged offsets of each sequence's queries */
+    const int32_t *q_pos;  /* [total_q] absolute position of each query token */
+    int32_t total_q;
+} dsa_queries;
+
+/*
+ * dsa_kv_append -- write new tokens into the paged cache [P5 "KV Cache
+ * Layout": prefill writes blocks in batch, decode appends incrementally and
+ * keeps the block table; both share one block-index semantics].
+ *   cu_new  [num_seqs+1]: sequence s appends tokens cu_new[s] .. cu_new[s+1]-1,
+ *           landing at positions seq_lens[s]-n_s .. seq_lens[s]-1.
+ *   k_new, v_new: bf16 [total_new][num_kv_heads][head_dim].
+ *   kc_new: int8 [total_new][idx_dim] or NULL.  Row i is the coarse key of the
+ *           block token i lands in, as that block stands after token i; each
+ *           touched block keeps the row of its last new token.  NULL leaves
+ *           kc_pool untouched.
+ * Device errors: DSA_DEV_ERR_POS (n_s > seq_lens[s] or block >= max_blocks),
+ * DSA_DEV_ERR_PAGE; the token is skipped.
+ */
+int dsa_kv_append(const dsa_kv_cache *cache, const dsa_seqs *seqs, const int32_t *cu_new,
+                  int32_t total_new, const void *k_new, const void *v_new,
+                  const int8_t *kc_new, int32_t *dev_err, dsa_stream_t stream);
+
+/*
+ * dsa_index_score -- block scores of every query against each visible block
+ * [P1 4(1): the inner product of the compressed representation with the
+ * query, in one fused kernel without intermediate writes; P5 "Index
+ * Selection Path": low-precision inputs; P3 4.1].  The pages leave the
+ * formula open; this library computes
+ *     S[t][b] = sum_h w[t][h] * max(0, sum_d q_idx[t][h][d] * kc[page(s,b)][d])
+ * exactly in int32.
+ *   q_idx  int8  [total_q][num_idx_heads][idx_dim]
+ *   w      int32 [total_q][num_idx_heads]; |w| <= w_abs_max (caller's bound)
+ *   scores int32 [total_q][max_blocks]: entries b <= q_pos[t]/block_size are
+ *          written, the rest of the row is left untouched.
+ * DSA_ERR_RANGE when num_idx_heads * w_abs_max * idx_dim * 128 * 128 >= 2^31
+ * (an int32 result could overflow).  Sequences with at least 16 queries take
+ * the tensor-core (tcgen05 int8) path, the others the CUDA-core path; both
+ * give the same integers.  Device errors: DSA_DEV_ERR_PAGE, DSA_DEV_ERR_POS.
+ */
+int dsa_index_score(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                    const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads,
+                    int32_t w_abs_max, int32_t *scores, int32_t *dev_err, dsa_stream_t stream);
+
+/*
+ * dsa_topk_blocks -- per-query block selection [P1 4(1) "Scalable Top-K";
+ * P5 "Index Selection Path": index semantics aligned with the gather].
+ * With n = q_pos[t]/block_size + 1 visible blocks and K = k_per_seq[s]:
+ * if n <= K every visible block is taken; otherwise the own block n-1 plus
+ * the K-1 best of blocks 0..n-2 under (score descending, block id ascending).
+ *   scores   int32 [total_q][max_blocks] as written by dsa_index_score
+ *   k_per_seq int32 [num_seqs], each in [1, k_max]
+ *   sel      int32 [total_q][k_max]: LOGICAL block ids ascending, then -1
+ *   cnt      int32 [total_q]: number of ids written
+ * Device errors: DSA_DEV_ERR_K (that query gets cnt 0), DSA_DEV_ERR_POS.
+ */
+int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int32_t *scores,
+                    const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt,
+                    int32_t *dev_err, dsa_stream_t stream);
+
+/*
+ * Exact attention over the selected blocks [P1 4(3) decode schematic; P3 4:
+ * exact attention on the selected part; P4 "Day-0 Adaptation for Large
+ * Language Models: From Architecture Analysis to Inference Serving", table:
+ * only the token pairs named by the indexes].  For query t and query head h
+ * (KV head h / (num_q_heads/num_kv_heads)), over the tokens j of the blocks
+ * sel[t][0..cnt[t]) with position <= q_pos[t]:
+ *     out[t][h] = sum_j softmax_j(sm_scale * q[t][h].k_j) v_j
+ *     lse[t][h] = ln sum_j exp(sm_scale * q[t][h].k_j)
+ * bf16 inputs, fp32 accumulation, bf16 out.
+ *   q   bf16 [total_q][num_q_heads][head_dim];  out bf16, same shape
+ *   lse fp32 [total_q][num_q_heads] (may be NULL)
+ * The decode entry splits each query's blocks over several CTAs and merges
+ * the partial softmax states; it needs a workspace of
+ * dsa_sparse_attn_decode_workspace_size() bytes, zero-filled before its first
+ * use (each call leaves it zeroed again).  The prefill entry runs one CTA per
+ * (query, KV head) and needs no workspace.
+ * Device errors: DSA_DEV_ERR_SEL, DSA_DEV_ERR_PAGE (that block is skipped).
+ */
+size_t dsa_sparse_attn_decode_workspace_size(int32_t total_q, int32_t num_q_heads,
+                                             int32_t num_kv_heads, int32_t k_max);
+
+int dsa_sparse_attn_decode(const dsa_kv_cache *cache, const dsa_seqs *seqs,
+                           const dsa_queries *queries, const void *q, int32_t num_q_heads,
+                           const int32_t *sel, const int32_t *cnt, int32_t k_max, float sm_scale,
+                           void *out, float *lse, void *workspace, size_t workspace_bytes,
+                           int32_t *dev_err, dsa_stream_t stream);
+
+int dsa_sparse_attn_prefill(const dsa_kv_cache *cache, const dsa_seqs *seqs,
+                            const dsa_queries *queries, const void *q, int32_t num_q_heads,
+                            const int32_t *sel, const int32_t *cnt, int32_t k_max, float sm_scale,
+                            void *out, float *lse, int32_t *dev_err, dsa_stream_t stream);
+
+/* human-readable name of a status code (static string) */
+const char *dsa_status_string(int status);
+
+/* library version, e.g. 100 for 0.1.0 */
+int dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

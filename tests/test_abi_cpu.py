@@ -1,0 +1,122 @@
+"""The C ABI loads on a machine without a GPU, exports every function that
+include/dsa.h declares, and rejects bad arguments on the host before any
+CUDA call (so these run without a device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from dynamic_block_sparse_dsa_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w \*]*?\b(dsa_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_pipeline():
+    names = _declared_functions()
+    for n in ("dsa_kv_append", "dsa_index_score", "dsa_topk_blocks", "dsa_sparse_attn_decode",
+              "dsa_sparse_attn_prefill"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    for n in _declared_functions():
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, f"binding lacks a signature for {n}"
+
+
+def test_status_strings_and_version():
+    lib = _lib.load()
+    assert lib.dsa_version() >= 100
+    assert lib.dsa_status_string(0) == b"ok"
+    assert lib.dsa_status_string(3) == b"int32 score range exceeded"
+
+
+FAKE = 0x10000   # a 16-byte aligned address that is never dereferenced on these paths
+
+
+def _cache(**kw):
+    base = dict(k_pool=FAKE, v_pool=FAKE, kc_pool=FAKE, num_pages=4, block_size=64, num_kv_heads=8,
+                head_dim=128, idx_dim=64)
+    base.update(kw)
+    return _lib.KvCacheC(**base)
+
+
+def _seqs(**kw):
+    base = dict(block_table=FAKE, max_blocks=4, seq_lens=FAKE, num_seqs=1)
+    base.update(kw)
+    return _lib.SeqsC(**base)
+
+
+def _queries(**kw):
+    base = dict(cu_q=FAKE, q_pos=FAKE, total_q=1)
+    base.update(kw)
+    return _lib.QueriesC(**base)
+
+
+def _score(cache, seqs, queries, heads=16, wmax=16, qidx=FAKE):
+    lib = _lib.load()
+    return lib.dsa_index_score(ctypes.byref(cache), ctypes.byref(seqs), ctypes.byref(queries), qidx, FAKE,
+                               heads, wmax, FAKE, None, None)
+
+
+def test_host_validation_codes():
+    c, s, q = _cache(), _seqs(), _queries()
+    assert _score(_cache(block_size=32), s, q) == _lib.DSA_ERR_UNSUPPORTED
+    assert _score(_cache(head_dim=64), s, q) == _lib.DSA_ERR_UNSUPPORTED
+    assert _score(_cache(k_pool=FAKE + 8), s, q) == _lib.DSA_ERR_INVALID_ARG      # misaligned
+    assert _score(_cache(num_pages=0), s, q) == _lib.DSA_ERR_INVALID_ARG
+    assert _score(c, _seqs(block_table=None), q) == _lib.DSA_ERR_INVALID_ARG
+    assert _score(c, s, _queries(total_q=-1)) == _lib.DSA_ERR_INVALID_ARG
+    assert _score(c, s, q, heads=17) == _lib.DSA_ERR_UNSUPPORTED
+    assert _score(c, s, q, heads=0) == _lib.DSA_ERR_INVALID_ARG
+    # 16 heads * |w| 16 * 64 * 128^2 = 2^28 is fine; |w| 128 would overflow int32
+    assert _score(c, s, q, wmax=128) == _lib.DSA_ERR_RANGE
+    assert _score(c, s, q, qidx=FAKE + 4) == _lib.DSA_ERR_INVALID_ARG
+    # nothing to do is fine and launches nothing
+    assert _score(c, s, _queries(total_q=0)) == _lib.DSA_OK
+
+
+def test_attention_validation_codes():
+    lib = _lib.load()
+    c, s, q = _cache(), _seqs(), _queries()
+
+    def dec(cache=c, hq=64, k_max=32, ws=None, ws_bytes=0, scale=0.088):
+        return lib.dsa_sparse_attn_decode(ctypes.byref(cache), ctypes.byref(s), ctypes.byref(q), FAKE, hq,
+                                          FAKE, FAKE, k_max, scale, FAKE, None, ws, ws_bytes, None, None)
+
+    assert dec(hq=60) == _lib.DSA_ERR_INVALID_ARG           # not a multiple of the KV heads
+    assert dec(hq=8 * 17) == _lib.DSA_ERR_UNSUPPORTED       # group of 17
+    assert dec(k_max=0) == _lib.DSA_ERR_INVALID_ARG
+    assert dec(scale=0.0) == _lib.DSA_ERR_INVALID_ARG
+    need = lib.dsa_sparse_attn_decode_workspace_size(8, 64, 8, 32)
+    assert need > 0 and need % 256 == 0
+    assert lib.dsa_sparse_attn_decode_workspace_size(0, 64, 8, 32) == 0
+    assert lib.dsa_sparse_attn_decode_workspace_size(8, 0, 8, 32) == 0
+
+
+def test_topk_and_append_validation_codes():
+    lib = _lib.load()
+    s, q = _seqs(), _queries()
+    assert lib.dsa_topk_blocks(ctypes.byref(s), ctypes.byref(q), FAKE, FAKE, 0, FAKE, FAKE, None,
+                               None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_topk_blocks(ctypes.byref(s), ctypes.byref(_queries(total_q=0)), FAKE, FAKE, 8, FAKE, FAKE,
+                               None, None) == _lib.DSA_OK
+    c = _cache()
+    assert lib.dsa_kv_append(ctypes.byref(c), ctypes.byref(s), FAKE, -1, FAKE, FAKE, None, None,
+                             None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_kv_append(ctypes.byref(c), ctypes.byref(s), FAKE, 1, FAKE + 2, FAKE, None, None,
+                             None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_kv_append(ctypes.byref(c), ctypes.byref(s), FAKE, 0, FAKE, FAKE, None, None,
+                             None) == _lib.DSA_OK

@@ -1,0 +1,234 @@
+"""GPU parity: the CUDA library against the oracle, on the same seeded inputs.
+
+Bar (stated here, used by every case):
+  * scores, selected block ids and counts: bit-exact (integer work);
+  * attention output (bf16, fp32 accumulation): max |gpu - oracle| <= 2e-2 and
+    mean |gpu - oracle| <= 2e-3 against the oracle's float64 result;
+  * lse (fp32): max |gpu - oracle| <= 2e-3.
+Every call goes through the C ABI (libdsa.so) via the Python binding.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import dynamic_block_sparse_dsa_b200 as dsa
+from dynamic_block_sparse_dsa_b200 import workloads as wk
+from oracle.harness import oracle_step
+
+pytestmark = pytest.mark.gpu
+
+OUT_MAX, OUT_MEAN, LSE_MAX = 2e-2, 2e-3, 2e-3
+
+
+def _handles(wl):
+    return (dsa.PagedKVCache(wl.k_pool, wl.v_pool, wl.kc_pool), dsa.SeqBatch(wl.block_table, wl.seq_lens),
+            dsa.QueryBatch(wl.cu_q, wl.q_pos))
+
+
+def gpu_step(wl, decode=True, bufs=None):
+    cache, seqs, queries = _handles(wl)
+    err = torch.zeros(1, dtype=torch.int32, device=wl.device)
+    bufs = dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
+                    q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=wl.spec.k_max,
+                    decode=decode, bufs=bufs, dev_err=err)
+    torch.cuda.synchronize()
+    return bufs, int(err.item())
+
+
+def compare(wl, ref, bufs, check_scores=True):
+    qs = torch.as_tensor(ref["queries"], device=wl.device)
+    sel = bufs["sel"].index_select(0, qs).cpu().numpy()
+    cnt = bufs["cnt"].index_select(0, qs).cpu().numpy()
+    assert np.array_equal(cnt, ref["cnt"]), "selection counts differ"
+    assert np.array_equal(sel, ref["sel"]), "selected block ids differ"
+    if check_scores and "scores" in ref:
+        sc = bufs["scores"].index_select(0, qs).cpu().numpy().astype(np.int64)
+        vis = ref["scores"] != np.iinfo(np.int64).min
+        assert np.array_equal(sc[vis], ref["scores"][vis]), "block scores differ"
+    out = bufs["out"].index_select(0, qs).double().cpu().numpy()
+    lse = bufs["lse"].index_select(0, qs).double().cpu().numpy()
+    d = np.abs(out - ref["out"])
+    assert d.max() <= OUT_MAX and d.mean() <= OUT_MEAN, (d.max(), d.mean())
+    assert np.abs(lse - ref["lse"]).max() <= LSE_MAX
+    return d.max(), d.mean()
+
+
+def _run(spec, seed, device, queries=None, decode=True, scores=True):
+    wl = wk.make_workload(spec, seed=seed, device=device)
+    ref = oracle_step(wl, queries=queries, want_scores=scores)
+    bufs, err = gpu_step(wl, decode=decode)
+    assert err == 0, f"device error bits {err}"
+    return wl, ref, bufs
+
+
+# ----------------------------------------------------------------------------- small, all outputs
+SMALL = {
+    # name: spec overrides (block_size 64, head_dim 128 fixed by the library)
+    "single_partial_block": dict(seq_lens=(37,), n_new=(1,), k_per_seq=(4,), k_max=4),
+    "one_token": dict(seq_lens=(1,), n_new=(1,), k_per_seq=(2,), k_max=2),
+    "k1_only_own": dict(seq_lens=(700, 130), n_new=(1, 1), k_per_seq=(1, 1), k_max=1),
+    "k_covers_all": dict(seq_lens=(300, 511), n_new=(1, 1), k_per_seq=(16, 16), k_max=16),
+    "ragged_prefill_tail": dict(seq_lens=(1000, 250, 64), n_new=(77, 0, 64), k_per_seq=(5, 3, 2), k_max=8),
+    "group16": dict(seq_lens=(900,), n_new=(3,), k_per_seq=(6,), k_max=6, num_q_heads=32, num_kv_heads=2),
+    "group1_mha": dict(seq_lens=(650, 200), n_new=(1, 2), k_per_seq=(4, 4), k_max=4, num_q_heads=4,
+                       num_kv_heads=4),
+    "many_seqs_decode": dict(seq_lens=tuple(range(129, 129 + 40 * 97, 97)), n_new=(1,) * 40,
+                             k_per_seq=(8,) * 40, k_max=8),
+    "prefill_two_chunks": dict(seq_lens=(3000, 2111), n_new=(200, 130), k_per_seq=(12, 7), k_max=12,
+                               occupancy=0.6),
+}
+
+
+def _small_spec(name, q_scale=1.0):
+    kw = dict(num_q_heads=16, num_kv_heads=2, num_idx_heads=16)
+    kw.update(SMALL[name])
+    return wk.WorkloadSpec(name, q_scale=q_scale, **kw)
+
+
+@pytest.mark.parametrize("decode", [True, False], ids=["decode_entry", "prefill_entry"])
+@pytest.mark.parametrize("q_scale", [1.0, 12.0], ids=["plain", "sharp"])
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_small_cases_all_outputs(name, q_scale, decode, cuda_device):
+    wl, ref, bufs = _run(_small_spec(name, q_scale), 100 + len(name), cuda_device, decode=decode)
+    compare(wl, ref, bufs)
+
+
+def test_tiny_decode_workload(cuda_device):
+    wl, ref, bufs = _run(wk.tiny_decode(), 1001, cuda_device)
+    compare(wl, ref, bufs)
+
+
+@pytest.mark.parametrize("q_scale", [1.0, 12.0])
+def test_batched_gqa_decode_workload(q_scale, cuda_device):
+    spec = wk.scaled(wk.batched_gqa_decode(), q_scale=q_scale)
+    wl, ref, bufs = _run(spec, 1002, cuda_device)
+    compare(wl, ref, bufs)
+
+
+@pytest.mark.slow
+def test_decode_1m_workload_all_outputs(cuda_device):
+    wl, ref, bufs = _run(wk.decode_1m(), 1003, cuda_device)
+    compare(wl, ref, bufs)
+    # the planted blocks shape the selection (non-trivial selections)
+    planted = wl.planted.cpu().numpy()
+    hits = [len(set(ref["sel"][s]) & set(planted[s])) for s in range(8)]
+    assert min(hits) >= 1, hits
+
+
+def _sample_queries(wl, n, rng):
+    T = wl.spec.total_q
+    pos = wl.q_pos.cpu().numpy()
+    edge = [0, T - 1] + [i for i in range(T) if pos[i] % 64 in (0, 63)][:8]
+    rest = rng.choice(T, size=min(T, n), replace=False).tolist()
+    return sorted(set(edge + rest))
+
+
+@pytest.mark.slow
+def test_chunked_prefill_workload_sampled(cuda_device):
+    spec = wk.chunked_prefill()
+    wl = wk.make_workload(spec, seed=1004, device=cuda_device)
+    qs = _sample_queries(wl, 40, np.random.default_rng(0))
+    ref = oracle_step(wl, queries=qs, want_scores=True)
+    bufs, err = gpu_step(wl, decode=False)
+    assert err == 0
+    compare(wl, ref, bufs)
+    # properties of every query at full size
+    cnt = bufs["cnt"].cpu().numpy()
+    sel = bufs["sel"].cpu().numpy()
+    own = wl.q_pos.cpu().numpy() // 64
+    assert (cnt == 64).all()
+    assert (sel[:, -1] == own).all()                       # own block last (largest id)
+    assert (np.diff(sel, axis=1) > 0).all()                # strictly ascending
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("decode", [True, False])
+def test_mixed_ragged_workload_sampled(decode, cuda_device):
+    spec = wk.mixed_ragged()
+    wl = wk.make_workload(spec, seed=1005, device=cuda_device)
+    cu = wl.cu_q.cpu().numpy()
+    decode_q = [int(cu[s]) for s in range(spec.num_seqs) if cu[s + 1] - cu[s] == 1]
+    rng = np.random.default_rng(1)
+    prefill_q = [int(x) for s in range(spec.num_seqs) if cu[s + 1] - cu[s] > 1
+                 for x in rng.choice(np.arange(cu[s], cu[s + 1]), size=12, replace=False)]
+    qs = sorted(decode_q + prefill_q)
+    ref = oracle_step(wl, queries=qs, want_scores=True)
+    bufs, err = gpu_step(wl, decode=decode)
+    assert err == 0
+    compare(wl, ref, bufs)
+
+
+# ----------------------------------------------------------------------------- invariants on the GPU
+def test_page_permutation_is_bit_identical(cuda_device):
+    spec = _small_spec("prefill_two_chunks", 8.0)
+    wl = wk.make_workload(spec, seed=7, device=cuda_device)
+    wl2 = wk.make_workload(spec, seed=7, device=cuda_device)
+    perm = torch.randperm(spec.num_pages, generator=torch.Generator().manual_seed(5)).to(cuda_device)
+    inv = torch.empty_like(perm)
+    inv[perm] = torch.arange(len(perm), device=cuda_device)
+    wl2.k_pool = wl.k_pool[inv].contiguous()
+    wl2.v_pool = wl.v_pool[inv].contiguous()
+    wl2.kc_pool = wl.kc_pool[inv].contiguous()
+    bt = wl.block_table.long()
+    wl2.block_table = torch.where(bt >= 0, perm[bt.clamp(min=0)], -1).to(torch.int32).contiguous()
+    b1, e1 = gpu_step(wl)
+    b2, e2 = gpu_step(wl2)
+    assert e1 == e2 == 0
+    for k in ("sel", "cnt", "out", "lse"):
+        assert torch.equal(b1[k], b2[k]), k
+
+
+def test_v_all_ones_gives_ones(cuda_device):
+    spec = _small_spec("ragged_prefill_tail", 16.0)
+    wl = wk.make_workload(spec, seed=8, device=cuda_device)
+    wl.v_pool.fill_(1.0)
+    wl.v_new.fill_(1.0)
+    for decode in (True, False):
+        b, e = gpu_step(wl, decode=decode)
+        assert e == 0
+        assert torch.all(b["out"] == 1.0)
+
+
+def test_repeat_calls_reuse_workspace(cuda_device):
+    # the split-KV workspace counters must be left at zero for the next call
+    spec = _small_spec("many_seqs_decode", 8.0)
+    wl = wk.make_workload(spec, seed=9, device=cuda_device)
+    b, e = gpu_step(wl)
+    first = b["out"].clone()
+    for _ in range(3):
+        b, e = gpu_step(wl, bufs=b)
+        assert e == 0
+        assert torch.equal(b["out"], first)
+    assert int(b["workspace"][:4 * spec.total_q * spec.num_kv_heads].view(torch.int32).abs().sum()) == 0
+
+
+# ----------------------------------------------------------------------------- device error flags
+def test_bad_page_sets_flag_without_fault(cuda_device):
+    spec = _small_spec("k_covers_all")
+    wl = wk.make_workload(spec, seed=10, device=cuda_device)
+    wl.block_table[0, 1] = spec.num_pages + 5
+    _, err = gpu_step(wl)
+    assert err & dsa._lib.DEV_ERR_PAGE
+
+
+def test_bad_position_and_k_set_flags(cuda_device):
+    spec = _small_spec("k_covers_all")
+    wl = wk.make_workload(spec, seed=11, device=cuda_device)
+    wl.q_pos[1] = int(wl.seq_lens[1]) + 3          # past the end of its sequence
+    wl.k_per_seq[0] = 0
+    b, err = gpu_step(wl)
+    assert err & dsa._lib.DEV_ERR_POS
+    assert err & dsa._lib.DEV_ERR_K
+    assert int(b["cnt"][0]) == 0 and int(b["cnt"][1]) == 0
+
+
+def test_host_validation_raises(cuda_device):
+    spec = _small_spec("one_token")
+    wl = wk.make_workload(spec, seed=12, device=cuda_device)
+    cache, seqs, queries = _handles(wl)
+    with pytest.raises(dsa.DsaError):
+        dsa.index_score(cache, seqs, queries, wl.q_idx, wl.w, w_abs_max=1 << 12)
+    with pytest.raises(ValueError):
+        dsa.index_score(cache, seqs, queries, wl.q_idx.cpu(), wl.w)
