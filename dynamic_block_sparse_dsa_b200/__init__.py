@@ -31,7 +31,7 @@ from ._lib import DsaError, load
 __all__ = [
     "PagedKVCache", "SeqBatch", "QueryBatch", "DsaError", "load",
     "kv_append", "index_score", "topk_blocks", "sparse_attn_decode", "sparse_attn_prefill",
-    "decode_workspace_size", "step",
+    "decode_workspace_size", "sparse_attn_decode_noalloc", "step",
 ]
 
 BLOCK_SIZE = 64
@@ -188,6 +188,26 @@ def sparse_attn_decode(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch,
         ctypes.byref(c), ctypes.byref(s), ctypes.byref(qq), _ptr(q), q.shape[1], _ptr(sel), _ptr(cnt),
         k_max, scale, _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), _ptr(dev_err),
         _stream(stream)))
+    return out, lse
+
+
+def sparse_attn_decode_noalloc(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, q: torch.Tensor,
+                               sel: torch.Tensor, cnt: torch.Tensor, sm_scale: Optional[float] = None,
+                               out=None, lse=None, dev_err: Optional[torch.Tensor] = None, stream=None):
+    """Decode attention that allocates nothing on the device: for callers that
+    cannot call cudaMalloc (an engine plugin's enqueue path, a runtime that owns
+    all device memory).  The split-KV scratch is a fixed 16 MiB array inside
+    the library; problems needing more are rejected, and calls that overlap on
+    the GPU share that array and race.  ``out``/``lse`` are allocated by torch
+    here only when not given."""
+    lib = load()
+    _expect(q, torch.bfloat16, "q")
+    out, lse = _attn_out(q, out, lse)
+    scale = 1.0 / math.sqrt(q.shape[2]) if sm_scale is None else float(sm_scale)
+    c, s, qq = cache.ctype(), seqs.ctype(), queries.ctype()
+    _lib.check("dsa_sparse_attn_decode_noalloc", lib.dsa_sparse_attn_decode_noalloc(
+        ctypes.byref(c), ctypes.byref(s), ctypes.byref(qq), _ptr(q), q.shape[1], _ptr(sel), _ptr(cnt),
+        sel.shape[1], scale, _ptr(out), _ptr(lse), _ptr(dev_err), _stream(stream)))
     return out, lse
 
 

@@ -185,6 +185,35 @@ int dsa_sparse_attn_prefill(const dsa_kv_cache *cache, const dsa_seqs *seqs,
                             const int32_t *sel, const int32_t *cnt, int32_t k_max, float sm_scale,
                             void *out, float *lse, int32_t *dev_err, dsa_stream_t stream);
 
+/*
+ * dsa_sparse_attn_decode_noalloc -- the decode attention above for callers
+ * that cannot allocate device memory.  The pages have no counterpart to this
+ * call; it exists for callers such as an engine plugin whose enqueue path must
+ * not allocate or synchronise, or a runtime that owns all device memory
+ * itself, which therefore cannot hand over a workspace from cudaMalloc.
+ * Arguments are those of dsa_sparse_attn_decode without the workspace: the
+ * split-KV scratch lives in a fixed array of DSA_NOALLOC_SCRATCH_BYTES inside
+ * the library, held on every GPU that loads the library until the process
+ * exits.  The call allocates nothing.
+ *  - Limit: dsa_sparse_attn_decode_workspace_size(total_q, num_q_heads,
+ *    num_kv_heads, k_max) must be <= DSA_NOALLOC_SCRATCH_BYTES (e.g. 8 decode
+ *    queries x 64 heads x Top-K 32 needs about 8.5 MiB); larger problems get
+ *    DSA_ERR_WORKSPACE and nothing is launched.
+ *  - The first call on each device (with that device current) looks up the
+ *    scratch array's device address; make that first call before any stream
+ *    capture.
+ *  - Every call first zeroes the scratch's split counters on `stream`.  All
+ *    calls share the one array, so calls that overlap on the GPU (other
+ *    streams or threads) race; the caller must serialise them.
+ */
+#define DSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+int dsa_sparse_attn_decode_noalloc(const dsa_kv_cache *cache, const dsa_seqs *seqs,
+                                   const dsa_queries *queries, const void *q, int32_t num_q_heads,
+                                   const int32_t *sel, const int32_t *cnt, int32_t k_max,
+                                   float sm_scale, void *out, float *lse, int32_t *dev_err,
+                                   dsa_stream_t stream);
+
 /* human-readable name of a status code (static string) */
 const char *dsa_status_string(int status);
 

@@ -1,0 +1,60 @@
+"""The allocation-free decode entry point against the regular one.
+
+dsa_sparse_attn_decode_noalloc serves callers that cannot call cudaMalloc
+(an engine plugin's enqueue path, a runtime that owns all device memory): its
+split-KV scratch is a fixed array inside the library.  Two calls in a row --
+the second one finds the first one's leftovers in that shared array -- must
+match dsa_sparse_attn_decode on the same selection, within the parity
+tolerance of the other GPU tests.  This file is collected last on purpose.
+"""
+import numpy as np
+import pytest
+import torch
+
+import dynamic_block_sparse_dsa_b200 as dsa
+from dynamic_block_sparse_dsa_b200 import workloads as wk
+
+pytestmark = pytest.mark.gpu
+
+OUT_MAX, OUT_MEAN, LSE_MAX = 2e-2, 2e-3, 2e-3
+
+
+def _setup(spec, seed, device):
+    wl = wk.make_workload(spec, seed=seed, device=device)
+    cache = dsa.PagedKVCache(wl.k_pool, wl.v_pool, wl.kc_pool)
+    seqs = dsa.SeqBatch(wl.block_table, wl.seq_lens)
+    queries = dsa.QueryBatch(wl.cu_q, wl.q_pos)
+    scores = dsa.index_score(cache, seqs, queries, wl.q_idx, wl.w)
+    sel, cnt = dsa.topk_blocks(seqs, queries, scores, wl.k_per_seq, spec.k_max)
+    return wl, cache, seqs, queries, sel, cnt
+
+
+@pytest.mark.parametrize("name,spec", [
+    ("decode_8x32_blocks", wk.WorkloadSpec("na1", seq_lens=(1 << 16,) * 8, n_new=(1,) * 8, k_per_seq=(32,) * 8,
+                                           k_max=32, q_scale=8.0)),
+    ("ragged_small", wk.WorkloadSpec("na2", seq_lens=(900, 70, 4000), n_new=(1, 1, 1), k_per_seq=(8, 2, 16),
+                                     k_max=16, num_q_heads=16, num_kv_heads=2)),
+])
+def test_noalloc_matches_regular_decode_twice(name, spec, cuda_device):
+    wl, cache, seqs, queries, sel, cnt = _setup(spec, 77, cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    ref_out, ref_lse = dsa.sparse_attn_decode(cache, seqs, queries, wl.q, sel, cnt, dev_err=err)
+    for _ in range(2):
+        out = torch.full_like(wl.q, float("nan"))
+        lse = torch.full(wl.q.shape[:2], float("nan"), dtype=torch.float32, device=cuda_device)
+        dsa.sparse_attn_decode_noalloc(cache, seqs, queries, wl.q, sel, cnt, out=out, lse=lse, dev_err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        d = (out.double() - ref_out.double()).abs()
+        assert float(d.max()) <= OUT_MAX and float(d.mean()) <= OUT_MEAN
+        assert float((lse - ref_lse).abs().max()) <= LSE_MAX
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
+    spec = wk.WorkloadSpec("na3", seq_lens=(5000,) * 64, n_new=(1,) * 64, k_per_seq=(64,) * 64, k_max=64)
+    wl, cache, seqs, queries, sel, cnt = _setup(spec, 78, cuda_device)
+    need = dsa.decode_workspace_size(spec.total_q, spec.num_q_heads, spec.num_kv_heads, spec.k_max)
+    assert need > 16 << 20
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.sparse_attn_decode_noalloc(cache, seqs, queries, wl.q, sel, cnt)
+    assert e.value.status == dsa._lib.DSA_ERR_WORKSPACE
