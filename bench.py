@@ -163,15 +163,20 @@ def run_ours(args, world, rank, device):
     seqs = dsa.SeqBatch(wl.block_table, wl.seq_lens)
     queries = dsa.QueryBatch(wl.cu_q, wl.q_pos)
     decode = all(n == 1 for n in spec.n_new)
+    fused = decode and spec.k_max <= 64   # score + Top-K in one pass for decode batches
     err = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.Stream(device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
 
     def front(b):
         dsa.kv_append(cache, seqs, queries.cu_q, wl.k_new, wl.v_new, wl.kc_new, dev_err=err)
-        dsa.index_score(cache, seqs, queries, wl.q_idx, wl.w, 16, scores=b["scores"], dev_err=err)
-        dsa.topk_blocks(seqs, queries, b["scores"], wl.k_per_seq, spec.k_max, sel=b["sel"], cnt=b["cnt"],
-                        dev_err=err)
+        if fused:
+            dsa.select_blocks(cache, seqs, queries, wl.q_idx, wl.w, wl.k_per_seq, spec.k_max, 16, sel=b["sel"],
+                              cnt=b["cnt"], workspace=b["select_ws"], dev_err=err)
+        else:
+            dsa.index_score(cache, seqs, queries, wl.q_idx, wl.w, 16, scores=b["scores"], dev_err=err)
+            dsa.topk_blocks(seqs, queries, b["scores"], wl.k_per_seq, spec.k_max, sel=b["sel"], cnt=b["cnt"],
+                            dev_err=err)
 
     def attn(b):
         if decode:
@@ -184,7 +189,7 @@ def run_ours(args, world, rank, device):
     with torch.cuda.stream(stream):
         bufs = dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
                         q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=spec.k_max, decode=decode,
-                        dev_err=err)
+                        fused_select=fused, dev_err=err)
     torch.cuda.synchronize(device)
     if int(err.item()) != 0:
         raise RuntimeError(f"device error bits {int(err.item())} in the first step")
@@ -256,7 +261,7 @@ def run_ours(args, world, rank, device):
                 dev_in[k].copy_(t, non_blocking=True)
             dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
                      q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=spec.k_max, decode=decode,
-                     bufs=bufs, dev_err=err)
+                     fused_select=fused, bufs=bufs, dev_err=err)
             host_out.copy_(bufs["out"], non_blocking=True)
             host_lse.copy_(bufs["lse"], non_blocking=True)
             e_e.record()
@@ -276,13 +281,14 @@ def run_ours(args, world, rank, device):
                    "top_k": spec.k_max, "block_size": spec.block_size,
                    "heads_q_kv_idx": [spec.num_q_heads, spec.num_kv_heads, spec.num_idx_heads],
                    "global_batch": spec.num_seqs * world, "parallelism": f"dp{world} (independent sequences)",
-                   "l2": "flushed by a 512 MiB write before every timed step", "graph": "one CUDA graph per step"},
+                   "l2": "flushed by a 512 MiB write before every timed step", "graph": "one CUDA graph per step",
+                   "select": "fused score+top-k" if fused else "index_score then topk_blocks"},
         "roofline": roofline,
         "step_roofline": step_roof,
         "attn_ms_mean": round(attn_mean_s * 1e3, 5),
         "step_ms_median": round(statistics.median(step_ms), 5),
         "e2e": e2e,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": (3 if fused else 4) * args.steps,
         "clocks": clk.summary(),
     }
     return res, wl

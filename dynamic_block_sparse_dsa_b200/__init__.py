@@ -30,8 +30,8 @@ from ._lib import DsaError, load
 
 __all__ = [
     "PagedKVCache", "SeqBatch", "QueryBatch", "DsaError", "load",
-    "kv_append", "index_score", "topk_blocks", "sparse_attn_decode", "sparse_attn_prefill",
-    "decode_workspace_size", "sparse_attn_decode_noalloc", "step",
+    "kv_append", "index_score", "topk_blocks", "select_blocks", "sparse_attn_decode", "sparse_attn_prefill",
+    "decode_workspace_size", "select_workspace_size", "sparse_attn_decode_noalloc", "step",
 ]
 
 BLOCK_SIZE = 64
@@ -157,6 +157,35 @@ def topk_blocks(seqs: SeqBatch, queries: QueryBatch, scores: torch.Tensor, k_per
     return sel, cnt
 
 
+def select_workspace_size(total_q: int) -> int:
+    return int(load().dsa_select_blocks_workspace_size(total_q))
+
+
+def select_blocks(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, q_idx: torch.Tensor,
+                  w: torch.Tensor, k_per_seq: torch.Tensor, k_max: int, w_abs_max: int = 16,
+                  sel: Optional[torch.Tensor] = None, cnt: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None, stream=None):
+    """index_score + topk_blocks fused (no score matrix): (sel, cnt).  ``workspace``
+    is a zero-initialised uint8 tensor of select_workspace_size() bytes (allocated here if None)."""
+    lib = load()
+    _expect(q_idx, torch.int8, "q_idx")
+    _expect(w, torch.int32, "w")
+    dev = q_idx.device
+    T = queries.total_q
+    if sel is None:
+        sel = torch.empty((T, k_max), dtype=torch.int32, device=dev)
+    if cnt is None:
+        cnt = torch.empty((T,), dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = torch.zeros(select_workspace_size(T), dtype=torch.uint8, device=dev)
+    c, s, q = cache.ctype(), seqs.ctype(), queries.ctype()
+    _lib.check("dsa_select_blocks", lib.dsa_select_blocks(
+        ctypes.byref(c), ctypes.byref(s), ctypes.byref(q), _ptr(q_idx), _ptr(w), q_idx.shape[1], int(w_abs_max),
+        _ptr(k_per_seq), int(k_max), _ptr(sel), _ptr(cnt), _ptr(workspace), workspace.numel(), _ptr(dev_err),
+        _stream(stream)))
+    return sel, cnt
+
+
 def decode_workspace_size(total_q: int, num_q_heads: int, num_kv_heads: int, k_max: int) -> int:
     return int(load().dsa_sparse_attn_decode_workspace_size(total_q, num_q_heads, num_kv_heads, k_max))
 
@@ -226,9 +255,10 @@ def sparse_attn_prefill(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch
 
 
 def step(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, *, k_new, v_new, kc_new, q, q_idx, w,
-         k_per_seq, k_max: int, w_abs_max: int = 16, decode: bool = True, bufs: Optional[dict] = None,
-         dev_err: Optional[torch.Tensor] = None, stream=None):
-    """One pass of the hot path: append -> index_score -> topk_blocks -> attention.
+         k_per_seq, k_max: int, w_abs_max: int = 16, decode: bool = True, fused_select: bool = False,
+         bufs: Optional[dict] = None, dev_err: Optional[torch.Tensor] = None, stream=None):
+    """One pass of the hot path: append -> index_score -> topk_blocks -> attention
+    (with ``fused_select`` the middle two are the single select_blocks call).
 
     ``bufs`` (optional, reused across calls) holds the scores / sel / cnt /
     out / lse / workspace tensors; missing ones are allocated.  Returns bufs.
@@ -243,10 +273,16 @@ def step(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, *, k_new, v_n
         b["lse"] = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
         b["workspace"] = torch.zeros(decode_workspace_size(T, q.shape[1], cache.num_kv_heads, k_max),
                                      dtype=torch.uint8, device=dev)
+        b["select_ws"] = torch.zeros(select_workspace_size(T), dtype=torch.uint8, device=dev)
     kv_append(cache, seqs, queries.cu_q, k_new, v_new, kc_new, dev_err=dev_err, stream=stream)
-    index_score(cache, seqs, queries, q_idx, w, w_abs_max, scores=b["scores"], dev_err=dev_err, stream=stream)
-    topk_blocks(seqs, queries, b["scores"], k_per_seq, k_max, sel=b["sel"], cnt=b["cnt"], dev_err=dev_err,
-                stream=stream)
+    if fused_select:
+        select_blocks(cache, seqs, queries, q_idx, w, k_per_seq, k_max, w_abs_max, sel=b["sel"], cnt=b["cnt"],
+                      workspace=b["select_ws"], dev_err=dev_err, stream=stream)
+    else:
+        index_score(cache, seqs, queries, q_idx, w, w_abs_max, scores=b["scores"], dev_err=dev_err,
+                    stream=stream)
+        topk_blocks(seqs, queries, b["scores"], k_per_seq, k_max, sel=b["sel"], cnt=b["cnt"], dev_err=dev_err,
+                    stream=stream)
     if decode:
         sparse_attn_decode(cache, seqs, queries, q, b["sel"], b["cnt"], out=b["out"], lse=b["lse"],
                            workspace=b["workspace"], dev_err=dev_err, stream=stream)

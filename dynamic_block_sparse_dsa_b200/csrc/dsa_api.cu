@@ -35,24 +35,56 @@ int check_queries(const dsa_queries *q) {
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
 
 int sm_count() {
-    int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n > 0 ? n : 148;
+    static int cached[64] = {};
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (dev >= 0 && dev < 64) cached[dev] = n;
+    return n;
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// decode workspace: [counters int32 T*Hkv][m,l f32 T*Hq*S*2][O f32 T*Hq*S*128], S <= k_max
+// decode workspace: [split counters int32 T*Hkv][partials f32 2*kAttnMaxCtas*G*kAttnPartStride]
 struct DecodeLayout {
-    size_t counters, ml, o, total;
+    size_t counters, part, total;
 };
-DecodeLayout decode_layout(int total_q, int hq, int hkv, int splits) {
+DecodeLayout decode_layout(int total_q, int hq, int hkv) {
     DecodeLayout L;
     L.counters = 0;
-    L.ml = align_up((size_t)total_q * hkv * sizeof(int32_t), 256);
-    L.o = align_up(L.ml + (size_t)total_q * hq * splits * 2 * sizeof(float), 256);
-    L.total = align_up(L.o + (size_t)total_q * hq * splits * kHeadDim * sizeof(float), 256);
+    L.part = align_up((size_t)total_q * hkv * sizeof(int32_t), 256);
+    L.total = align_up(L.part + (size_t)2 * kAttnMaxCtas * (hq / hkv) * kAttnPartStride * sizeof(float), 256);
     return L;
+}
+
+// select workspace: [counters int32 T][candidates uint2 T*kSelMaxChunks*(kSelMaxK-1)]
+struct SelectLayout {
+    size_t counters, cand, total;
+};
+SelectLayout select_layout(int total_q) {
+    SelectLayout L;
+    L.counters = 0;
+    L.cand = align_up((size_t)total_q * sizeof(int32_t), 256);
+    L.total = align_up(L.cand + (size_t)total_q * kSelMaxChunks * (kSelMaxK - 1) * sizeof(uint2), 256);
+    return L;
+}
+
+// grid of the persistent attention kernel: one CTA per SM, never more CTAs
+// than work items so that every CTA owns a non-empty range
+void attn_schedule(AttnArgs &a, bool allow_split) {
+    const long long pairs = (long long)a.total_q * a.num_kv_heads;
+    a.total_units = pairs * a.k_max;
+    long long C = sm_count();
+    if (C > kAttnMaxCtas) C = kAttnMaxCtas;
+    // whole (query, KV head) pairs per CTA when there are plenty of them (or
+    // when no workspace is available); otherwise split pairs across CTAs
+    a.pair_aligned = (!allow_split || pairs >= 16 * C) ? 1 : 0;
+    const long long items = a.pair_aligned ? pairs : a.total_units;
+    if (C > items) C = items;
+    // a pair may be split over at most ~60 CTAs (the kernel merges <= 63 partials)
+    if (C > pairs * 60) C = pairs * 60;
+    a.num_ctas = (int)C;
 }
 
 int attn_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
@@ -67,6 +99,10 @@ int attn_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queri
     const int group = num_q_heads / cache->num_kv_heads;
     if (group > kMaxGroup) return DSA_ERR_UNSUPPORTED;
     if (!(sm_scale > 0.f)) return DSA_ERR_INVALID_ARG;
+    // TMA coordinates are int32: pool rows (page*64+token) and query rows (t*Hq+h)
+    if ((long long)cache->num_pages * kBlockSize >= (1LL << 31) ||
+        (long long)queries->total_q * num_q_heads >= (1LL << 31))
+        return DSA_ERR_UNSUPPORTED;
     a = AttnArgs{};
     a.k_pool = static_cast<const __nv_bfloat16 *>(cache->k_pool);
     a.v_pool = static_cast<const __nv_bfloat16 *>(cache->v_pool);
@@ -174,6 +210,7 @@ int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int3
     int rc;
     if ((rc = check_seqs(seqs)) || (rc = check_queries(queries))) return rc;
     if (k_max < 1) return DSA_ERR_INVALID_ARG;
+    if (seqs->max_blocks > topk_max_blocks()) return DSA_ERR_UNSUPPORTED;
     if (queries->total_q == 0) return DSA_OK;
     if (!scores || !k_per_seq || !sel || !cnt) return DSA_ERR_INVALID_ARG;
     TopkArgs a{};
@@ -192,10 +229,55 @@ int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int3
     return from_cuda(launch_topk(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t dsa_select_blocks_workspace_size(int32_t total_q) {
+    if (total_q <= 0) return 0;
+    return select_layout(total_q).total;
+}
+
+int dsa_select_blocks(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                      const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads, int32_t w_abs_max,
+                      const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt, void *workspace,
+                      size_t workspace_bytes, int32_t *dev_err, dsa_stream_t stream) {
+    int rc;
+    if ((rc = check_cache(cache)) || (rc = check_seqs(seqs)) || (rc = check_queries(queries))) return rc;
+    if (num_idx_heads < 1 || w_abs_max < 0 || k_max < 1) return DSA_ERR_INVALID_ARG;
+    if (num_idx_heads > kMaxIdxHeads || k_max > kSelMaxK || seqs->max_blocks > kSelMaxChunks * 4096)
+        return DSA_ERR_UNSUPPORTED;
+    const long long bound = (long long)num_idx_heads * w_abs_max * kIdxDim * 128LL * 128LL;
+    if (bound >= (1LL << 31)) return DSA_ERR_RANGE;
+    if (queries->total_q == 0) return DSA_OK;
+    if (!q_idx || !w || !k_per_seq || !sel || !cnt || !aligned16(q_idx)) return DSA_ERR_INVALID_ARG;
+    const SelectLayout L = select_layout(queries->total_q);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < L.total) return DSA_ERR_WORKSPACE;
+    SelectArgs a{};
+    a.kc_pool = cache->kc_pool;
+    a.num_pages = cache->num_pages;
+    a.block_table = seqs->block_table;
+    a.max_blocks = seqs->max_blocks;
+    a.seq_lens = seqs->seq_lens;
+    a.num_seqs = seqs->num_seqs;
+    a.cu_q = queries->cu_q;
+    a.q_pos = queries->q_pos;
+    a.total_q = queries->total_q;
+    a.q_idx = q_idx;
+    a.w = w;
+    a.num_idx_heads = num_idx_heads;
+    a.k_per_seq = k_per_seq;
+    a.k_max = k_max;
+    a.sel = sel;
+    a.cnt = cnt;
+    char *ws = static_cast<char *>(workspace);
+    a.counters = reinterpret_cast<int32_t *>(ws + L.counters);
+    a.cand = reinterpret_cast<uint2 *>(ws + L.cand);
+    a.dev_err = dev_err;
+    return from_cuda(launch_select_blocks(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t dsa_sparse_attn_decode_workspace_size(int32_t total_q, int32_t num_q_heads, int32_t num_kv_heads,
                                              int32_t k_max) {
-    if (total_q < 0 || num_q_heads < 1 || num_kv_heads < 1 || k_max < 1) return 0;
-    return decode_layout(total_q, num_q_heads, num_kv_heads, k_max).total;
+    if (total_q <= 0 || num_q_heads < 1 || num_kv_heads < 1 || k_max < 1 || num_q_heads % num_kv_heads)
+        return 0;
+    return decode_layout(total_q, num_q_heads, num_kv_heads).total;
 }
 
 int dsa_sparse_attn_decode(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
@@ -206,27 +288,12 @@ int dsa_sparse_attn_decode(const dsa_kv_cache *cache, const dsa_seqs *seqs, cons
     int rc = attn_common(cache, seqs, queries, q, num_q_heads, sel, cnt, k_max, sm_scale, out, lse, dev_err, a);
     if (rc) return rc;
     if (queries->total_q == 0) return DSA_OK;
-    // split each query's selection so that (query, KV head, split) CTAs fill
-    // about two waves of the SMs
-    const long long per_split = (long long)queries->total_q * cache->num_kv_heads;
-    long long want = (2LL * sm_count() + per_split - 1) / per_split;
-    if (want < 1) want = 1;
-    if (want > k_max) want = k_max;
-    const int bps = (int)((k_max + want - 1) / want);
-    const int splits = (k_max + bps - 1) / bps;
-    a.n_splits = splits;
-    a.blocks_per_split = bps;
-    if (splits > 1) {
-        const DecodeLayout L = decode_layout(queries->total_q, num_q_heads, cache->num_kv_heads, splits);
-        if (!workspace || !aligned16(workspace) ||
-            workspace_bytes < dsa_sparse_attn_decode_workspace_size(queries->total_q, num_q_heads,
-                                                                    cache->num_kv_heads, k_max))
-            return DSA_ERR_WORKSPACE;
-        char *ws = static_cast<char *>(workspace);
-        a.counters = reinterpret_cast<int32_t *>(ws + L.counters);
-        a.part_ml = reinterpret_cast<float *>(ws + L.ml);
-        a.part_o = reinterpret_cast<float *>(ws + L.o);
-    }
+    const DecodeLayout L = decode_layout(queries->total_q, num_q_heads, cache->num_kv_heads);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < L.total) return DSA_ERR_WORKSPACE;
+    char *ws = static_cast<char *>(workspace);
+    a.counters = reinterpret_cast<int32_t *>(ws + L.counters);
+    a.part = reinterpret_cast<float *>(ws + L.part);
+    attn_schedule(a, true);
     return from_cuda(launch_sparse_attn(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -238,8 +305,7 @@ int dsa_sparse_attn_prefill(const dsa_kv_cache *cache, const dsa_seqs *seqs, con
     int rc = attn_common(cache, seqs, queries, q, num_q_heads, sel, cnt, k_max, sm_scale, out, lse, dev_err, a);
     if (rc) return rc;
     if (queries->total_q == 0) return DSA_OK;
-    a.n_splits = 1;
-    a.blocks_per_split = k_max;
+    attn_schedule(a, false);   // whole pairs per CTA: no partial states, no workspace
     return from_cuda(launch_sparse_attn(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -52,6 +52,31 @@ struct TopkArgs {
     int32_t *dev_err;
 };
 
+// fused score + Top-K (decode-oriented): candidate workspace layout
+constexpr int kSelMaxChunks = 32;   // chunks per query
+constexpr int kSelMaxK = 64;        // largest k_max of the fused path
+struct SelectArgs {
+    const int8_t *kc_pool;
+    int num_pages;
+    const int32_t *block_table;
+    int max_blocks;
+    const int32_t *seq_lens;
+    int num_seqs;
+    const int32_t *cu_q;
+    const int32_t *q_pos;
+    int total_q;
+    const int8_t *q_idx;     // [T][H][64]
+    const int32_t *w;        // [T][H]
+    int num_idx_heads;
+    const int32_t *k_per_seq;
+    int k_max;
+    int32_t *sel;            // [T][k_max]
+    int32_t *cnt;            // [T]
+    uint2 *cand;             // [T][kSelMaxChunks][kSelMaxK-1] (order key, block id)
+    int32_t *counters;       // [T] chunk CTAs done per query
+    int32_t *dev_err;
+};
+
 struct AttnArgs {
     const __nv_bfloat16 *k_pool, *v_pool;
     int num_pages, num_kv_heads;
@@ -71,17 +96,27 @@ struct AttnArgs {
     float scale_log2;        // sm_scale * log2(e)
     __nv_bfloat16 *out;      // [T][Hq][128]
     float *lse;              // [T][Hq] or null
-    int n_splits;            // CTAs per (query, kv head)
-    int blocks_per_split;
-    float *part_o;           // [T][Hq][n_splits][128]
-    float *part_ml;          // [T][Hq][n_splits][2]
-    int32_t *counters;       // [T][Hkv]
+    // persistent schedule: work unit u = (query t, KV head, selection slot j),
+    // u = (t * Hkv + kvh) * k_max + j; CTA c owns [c*U/C, (c+1)*U/C), rounded to
+    // whole (t, kvh) pairs when pair_aligned
+    long long total_units;   // U
+    int num_ctas;            // C (= gridDim.x)
+    int pair_aligned;
+    float *part;             // [2*C][group][kAttnPartStride] partial (o[128], m, l) of split pairs
+    int32_t *counters;       // [T*Hkv] units merged so far per split pair
     int32_t *dev_err;
 };
 
 cudaError_t launch_kv_append(const KvAppendArgs &a, cudaStream_t stream);
 cudaError_t launch_index_score(const IndexScoreArgs &a, cudaStream_t stream);
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream);
+cudaError_t launch_select_blocks(const SelectArgs &a, cudaStream_t stream);
+int topk_max_blocks();   // longest block table the standalone Top-K kernel accepts
+// the K/V pool and Q tensor maps are built by the launcher from AttnArgs
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream);
+// largest grid the attention kernel uses (sizes the partial-state workspace)
+constexpr int kAttnMaxCtas = 256;
+// floats per partial-state row: o[128], m, l, padded to a 16-byte multiple
+constexpr int kAttnPartStride = 132;
 
 }  // namespace dsa

@@ -1,0 +1,104 @@
+// dsa_tma.cuh -- mbarrier and TMA (cp.async.bulk.tensor) helpers for sm_100a.
+//
+// Every wait is bounded: a wait that has not completed after kWaitLimitCycles
+// SM clock cycles gives up and reports false, so that a kernel can flag
+// DSA_DEV_ERR_WAIT and wind down instead of hanging the GPU.
+#pragma once
+
+#include <cuda.h>
+
+#include "dsa_common.cuh"
+
+namespace dsa {
+
+// clock64 is a cheap per-SM cycle counter (unlike %globaltimer, which is slow
+// to read in a spin loop); 2^32 cycles is about 2 s at the boost clock.
+constexpr long long kWaitLimitCycles = 1ll << 32;
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+// make initialised barriers visible to the async (TMA) proxy
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// wait for the phase with the given parity to complete; false on timeout or
+// when *abort becomes non-zero (another role of the CTA gave up)
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+#pragma unroll 1
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > kWaitLimitCycles) return false;
+    }
+}
+
+// wait until *word == value (a shared-memory word another warp writes);
+// false on timeout or when *abort becomes non-zero
+__device__ __forceinline__ bool wait_value(const volatile int *word, int value, const volatile int *abort) {
+    if (*word == value) return true;
+    const long long t0 = clock64();
+#pragma unroll 1
+    while (*word != value) {
+        if (*abort) return false;
+        if (clock64() - t0 > kWaitLimitCycles) return false;
+    }
+    return true;
+}
+
+// 2-D / 3-D tiled TMA loads into shared memory, completing on an mbarrier
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y, int z,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+        "%4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// named barrier over a subset of the CTA's warps
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// byte offset of 16-byte chunk c (0..7) of row r in a 128B-swizzled tile of
+// 128-byte rows (the layout a SWIZZLE_128B TMA box writes; base 1024-aligned)
+__device__ __forceinline__ uint32_t swz128(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
+
+}  // namespace dsa

@@ -15,6 +15,7 @@
 // query rows, which every thread of the CTA reads from shared memory as
 // broadcasts.  Queries of the sequence are taken in batches of kQBatch.
 #include "dsa_kernels.h"
+#include "indexer_core.cuh"
 
 namespace dsa {
 
@@ -47,12 +48,7 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_dp4a_kernel(IndexSc
     if (b < n_blocks && b < a.max_blocks) {
         const int page = __ldg(a.block_table + (size_t)s * a.max_blocks + b);
         if (page >= 0 && page < a.num_pages) {
-            const int4 *src = reinterpret_cast<const int4 *>(a.kc_pool + (size_t)page * kIdxDim);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                int4 v = __ldg(src + i);
-                kc[4 * i + 0] = v.x; kc[4 * i + 1] = v.y; kc[4 * i + 2] = v.z; kc[4 * i + 3] = v.w;
-            }
+            load_coarse_key(a.kc_pool, page, kc);
             have = true;
         } else {
             set_err(a.dev_err, DSA_DEV_ERR_PAGE);
@@ -83,19 +79,7 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_dp4a_kernel(IndexSc
         if (!have) continue;
         for (int qi = 0; qi < nq; ++qi) {
             if (b > s_own[qi]) continue;
-            int total = 0;
-            for (int h = 0; h < H; ++h) {
-                int dot = 0;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int4 qv = s_q[qi][h][i];
-                    dot = __dp4a(kc[4 * i + 0], qv.x, dot);
-                    dot = __dp4a(kc[4 * i + 1], qv.y, dot);
-                    dot = __dp4a(kc[4 * i + 2], qv.z, dot);
-                    dot = __dp4a(kc[4 * i + 3], qv.w, dot);
-                }
-                total += s_w[qi][h] * max(dot, 0);
-            }
+            const int total = block_score(kc, s_q[qi], s_w[qi], H);
             a.scores[(size_t)(qb + qi) * a.max_blocks + b] = total;
         }
     }

@@ -2,338 +2,658 @@
 //
 // "Day-0 Adaptation for Massive LLMs: Overcoming Sparse Attention and MXFP4
 // Expert Weights", section 4(3): decode gathers the selected KV blocks on chip
-// by their indices and attends under a valid mask; the cost is the gather of
+// by their indices and attends under a valid mask; its cost is the gather of
 // non-contiguous blocks.  "Day-0 Adaptation for Trillion-Parameter Models:
 // Engineering Practices and Technical Breakdown", section 4.3: decode needs a
 // dedicated gather kernel.  "Day-0 Readiness ...", section "KV Cache Layout":
-// read whole blocks by block id, never per token.
+// read whole blocks by block id, never token by token.
 //
-// One CTA = (split of the selection, KV head, query).  The CTA streams its
-// selected blocks' K and V page slices -- 64 tokens x 256 bytes each, token
-// stride num_kv_heads*256 bytes -- through a 3-stage cp.async ring of 16-byte
-// copies into XOR-swizzled shared memory, and runs the GQA group of query
-// heads (rows of an m16 tile) against them on the tensor cores with
-// mma.m16n8k16 bf16 / fp32 accumulate:
-//   S = Q K^T  (A = Q from registers, B = K via ldmatrix),
-//   online softmax in fp32 (base-2 exponent, causal mask inside the own block),
-//   O += P V   (P re-used from the S accumulators as the A operand, B = V via
-//               ldmatrix.trans).
-// Each of the 4 warps takes 16 of the 64 tokens of every block; their softmax
-// states are merged through shared memory at the end.  With n_splits > 1 the
-// CTA writes its partial state (m, l, unnormalised O) to the workspace and the
-// last CTA of the (query, KV head) -- elected by an atomic counter, no waiting
-// -- merges the partials and resets the counter.
+// Design (B200): a persistent grid of one CTA per SM.  The work is the list of
+// units u = (query t, KV head, selection slot j) -- one 64-token page slice of
+// K and of V (16 KiB each) -- and CTA c takes the contiguous range
+// [c*U/C, (c+1)*U/C), so every SM streams the same number of bytes whatever
+// the batch looks like.  Inside the CTA:
+//   * a producer warp walks the range and, for each selected block, issues four
+//     boxes of a 3-D TMA tensor map over the pool (K and V, two 128-byte halves
+//     each, SWIZZLE_128B, no multicast) into a 5-stage shared-memory ring
+//     guarded by full/empty mbarriers; it also TMA-loads the 16-row query tile
+//     of each (query, KV head) pair into a 2-slot ring;
+//   * four consumer warps take whole blocks round-robin.  Each runs the GQA
+//     group of query heads (rows of an m16 tile) against its 64 tokens on the
+//     tensor cores with mma.m16n8k16 bf16/fp32: S = Q K^T, online softmax in
+//     fp32 with base-2 exponents and the causal mask of the own block, then
+//     O += P V with P reused from the S accumulators as the A operand;
+//   * at the end of each pair the four warps' softmax states are merged in a
+//     fixed order through shared memory.  A pair that lies wholly inside the
+//     CTA is written straight out; a pair split across CTAs leaves a partial
+//     (m, l, unnormalised O) in the workspace and the CTA completing its units
+//     -- counted with an atomic, no waiting -- merges the partials.
+// All waits are bounded (DSA_DEV_ERR_WAIT on timeout, no hang).
 #include "dsa_kernels.h"
+#include "dsa_tma.cuh"
 
 namespace dsa {
 
 namespace {
-constexpr int kAttnThreads = 128;
-constexpr int kStages = 3;
-constexpr int kTileBytes = kBlockSize * kHeadDim * 2;       // 16 KiB: one K or V page slice
-constexpr int kQBytes = 16 * kHeadDim * 2;                  // 4 KiB: 16 padded query rows
-constexpr int kSmemBytes = kQBytes + kStages * 2 * kTileBytes;
+constexpr int kConsumerWarps = 4;
+constexpr int kAttnThreads = (kConsumerWarps + 1) * 32;
+constexpr int kStages = 5;
+constexpr int kHalf = kBlockSize * 128;            // 8 KiB: 64 rows x 128 B (one swizzled half)
+constexpr int kStageBytes = 4 * kHalf;             // K lo, K hi, V lo, V hi
+constexpr int kQHalf = 16 * 128;                   // 16 query rows x 128 B
+constexpr int kQSlotBytes = 2 * kQHalf;
+constexpr int kSegSlots = 2;                       // query tile + pair facts, double buffered
+constexpr int kMergeStride = 132;                  // floats per merge row (padded against bank conflicts)
+constexpr int kMaxSmemSeqs = 2048;                 // cu_q entries cached in shared memory
+constexpr int kOffQ = kStages * kStageBytes;
+constexpr int kOffMergeO = kOffQ + kSegSlots * kQSlotBytes;
+constexpr int kOffMergeML = kOffMergeO + kConsumerWarps * 16 * kMergeStride * 4;
+constexpr int kOffCuq = kOffMergeML + kConsumerWarps * 16 * 2 * 4;
+constexpr int kOffBars = kOffCuq + (kMaxSmemSeqs + 1) * 4 + 4;
+constexpr int kNumBars = 2 * kStages + 2 * kSegSlots;
+constexpr int kOffWords = kOffBars + kNumBars * 8;
+// int words after the barriers
+constexpr int kWAbort = 0, kWLast = 1, kWNever = 2;
+constexpr int kWFill = 4;                           // [kStages] item index the stage was last armed for
+constexpr int kWItemBlk = kWFill + kStages;         // [kStages] logical block of that item
+constexpr int kWItemSeg = kWItemBlk + kStages;      // [kStages] segment of that item
+constexpr int kWSegEndCnt = kWItemSeg + kStages;    // [kSegSlots] items issued when the segment ended
+constexpr int kWSegEndTag = kWSegEndCnt + kSegSlots;  // [kSegSlots] which segment that count belongs to
+constexpr int kWSegInfo = kWSegEndTag + kSegSlots;  // [kSegSlots][4]: t, kvh, p, n_vis
+constexpr int kNumWords = kWSegInfo + 4 * kSegSlots;
+constexpr int kSmemBytes = kOffWords + kNumWords * 4 + 1024;   // + slack to align the base to 1 KiB
 constexpr float kLn2 = 0.6931471805599453f;
+// most CTAs whose ranges can cover one pair (the host keeps K*C/U + 2 below it)
+constexpr int kMaxSplitSlots = 63;
 
-// byte offset of 16-byte chunk c of row r in a [rows][256 B] tile, XOR-swizzled
-__device__ __forceinline__ uint32_t swz(int r, int c) { return r * 256 + ((c ^ (r & 7)) << 4); }
-
-struct BlockRef {
-    int blk;        // logical block id, -1 if unusable
-    int page;
-    uint32_t err;   // DSA_DEV_ERR_* bit explaining an unusable block
+struct Smem {
+    uint32_t base;   // 1 KiB aligned shared address
+    __device__ uint32_t stage(int s) const { return base + s * kStageBytes; }
+    __device__ uint32_t qslot(int s) const { return base + kOffQ + s * kQSlotBytes; }
+    __device__ uint32_t full(int s) const { return base + kOffBars + 8 * s; }
+    __device__ uint32_t empty(int s) const { return base + kOffBars + 8 * (kStages + s); }
+    __device__ uint32_t qfull(int s) const { return base + kOffBars + 8 * (2 * kStages + s); }
+    __device__ uint32_t qempty(int s) const { return base + kOffBars + 8 * (2 * kStages + kSegSlots + s); }
 };
 
-__device__ __forceinline__ BlockRef block_ref(const AttnArgs &a, int t, int s, int j, int n_vis) {
-    BlockRef r{-1, -1, 0u};
-    const int b = __ldg(a.sel + (size_t)t * a.k_max + j);
-    if (b < 0 || b >= n_vis) { r.err = DSA_DEV_ERR_SEL; return r; }
-    const int page = __ldg(a.block_table + (size_t)s * a.max_blocks + b);
-    if (page < 0 || page >= a.num_pages) { r.err = DSA_DEV_ERR_PAGE; return r; }
-    r.blk = b;
-    r.page = page;
-    return r;
+__device__ __forceinline__ long long range_begin(const AttnArgs &a, int c) {
+    if (a.pair_aligned) {
+        const long long pairs = a.total_units / a.k_max;
+        return (long long)c * pairs / a.num_ctas * a.k_max;
+    }
+    return (long long)c * a.total_units / a.num_ctas;
+}
+
+// sequence of query t: last s with cu_q[s] <= t, from the shared-memory copy when it fits
+__device__ __forceinline__ int seq_of(const AttnArgs &a, const int *s_cuq, int t) {
+    if (a.num_seqs + 1 > kMaxSmemSeqs) return find_seq(a.cu_q, a.num_seqs, t);
+    int lo = 0, hi = a.num_seqs - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_cuq[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
 }
 }  // namespace
 
-__global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ int s_last;
+template <int NT>   // query-head n-tiles of 8: the GQA group is <= 8 * NT
+__global__ void __launch_bounds__(kAttnThreads, 1)
+sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_q, AttnArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    Smem sm{(raw + 1023u) & ~1023u};
+    uint8_t *gbase = smem_raw + (sm.base - raw);   // generic pointer of the aligned base
+    volatile int *W = reinterpret_cast<volatile int *>(gbase + kOffWords);
+    volatile int *s_abort = W + kWAbort;
+    const volatile int *s_never = W + kWNever;      // stays 0: a wait that ignores the abort flag
+    int *s_cuq = reinterpret_cast<int *>(gbase + kOffCuq);
 
-    const int t = blockIdx.x, kvh = blockIdx.y, split = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, c = lane & 3;
+    const int c = blockIdx.x;
+    const long long u0 = range_begin(a, c), u1 = range_begin(a, c + 1);
     const int G = a.group;
-    const int h0 = kvh * G;
+    const long long K = a.k_max;
 
-    const int s = find_seq(a.cu_q, a.num_seqs, t);
-    const int p = __ldg(a.q_pos + t);
-    const int len = __ldg(a.seq_lens + s);
-    int n_sel = __ldg(a.cnt + t);
-    const int n_vis = p / kBlockSize + 1;
-    bool bad_query = (p < 0 || p >= len || n_vis > a.max_blocks);
-    if (n_sel < 0 || n_sel > a.k_max) {
-        if (tid == 0 && split == 0 && kvh == 0) set_err(a.dev_err, DSA_DEV_ERR_SEL);
-        n_sel = 0;
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(sm.full(s), 1);
+            mbar_init(sm.empty(s), 1);
+        }
+        for (int s = 0; s < kSegSlots; ++s) {
+            mbar_init(sm.qfull(s), 1);
+            mbar_init(sm.qempty(s), 1);
+        }
+        for (int k = 0; k < kNumWords; ++k) W[k] = 0;
+        for (int s = 0; s < kStages; ++s) W[kWFill + s] = -1;
+        for (int s = 0; s < kSegSlots; ++s) W[kWSegEndTag + s] = -1;
+        fence_barrier_init();
     }
-    if (bad_query) {
-        if (tid == 0 && split == 0 && kvh == 0) set_err(a.dev_err, DSA_DEV_ERR_POS);
-        n_sel = 0;
-    }
-    const int j0 = split * a.blocks_per_split;
-    const int j1 = min(n_sel, j0 + a.blocks_per_split);
+    __syncthreads();
 
-    const uint32_t sQ = smem_u32(smem);
-    const uint32_t sKV = sQ + kQBytes;
-    const size_t row_elems = (size_t)a.num_kv_heads * kHeadDim;   // one token row of the pool
-
-    // ---- query tile: rows 0..G-1 real, the rest zero
-    for (int e = tid; e < 16 * 16; e += kAttnThreads) {
-        const int r = e >> 4, ch = e & 15;
-        const __nv_bfloat16 *src = a.q + ((size_t)t * a.num_q_heads + h0 + min(r, G - 1)) * kHeadDim + ch * 8;
-        if (r < G) cp_async_16(sQ + swz(r, ch), src);
-        else cp_async_16_zero(sQ + swz(r, ch), src);
-    }
-
-    auto load_block = [&](int j, int stage) {
-        const BlockRef br = block_ref(a, t, s, j, n_vis);
-        const uint32_t dk = sKV + stage * 2 * kTileBytes;
-        const uint32_t dv = dk + kTileBytes;
-        if (br.blk < 0) {
-            // unusable block: flag it and zero the stage so that the masked
-            // products see finite values (0 * stale NaN would poison O)
-            if (tid == 0) set_err(a.dev_err, br.err);
-#pragma unroll
-            for (int i = 0; i < (kBlockSize * 16) / kAttnThreads; ++i) {
-                const int e = tid + i * kAttnThreads;
-                cp_async_16_zero(dk + swz(e >> 4, e & 15), a.k_pool);
-                cp_async_16_zero(dv + swz(e >> 4, e & 15), a.v_pool);
+    if (warp == kConsumerWarps) {
+        // ================================================================ producer warp
+        // The warp resolves 32 units per round trip (one lane per unit: pair
+        // facts, selected block, page), then lane 0 publishes them in order:
+        // a segment header (pair facts + TMA of the query tile) when a
+        // (query, KV head) pair starts, one stage fill per usable block, and a
+        // segment end marker (item count) when the pair's units are done.
+        if (a.num_seqs + 1 <= kMaxSmemSeqs)
+            for (int k = lane; k <= a.num_seqs; k += 32) s_cuq[k] = __ldg(a.cu_q + k);
+        __syncwarp();
+        if (lane == 0) {
+            prefetch_tensormap(&tm_k);
+            prefetch_tensormap(&tm_v);
+            prefetch_tensormap(&tm_q);
+        }
+        int item = 0, seg = 0;
+        uint32_t err_bits = 0;
+        bool stop = false;
+        for (long long base = u0; base < u1 && !stop; base += 32) {
+            const long long uu = base + lane;
+            const bool in = uu < u1;
+            int t = 0, kvh = 0, s = 0, p = 0, n_vis = 0, blk = -1, page = -1;
+            if (in) {
+                const long long pair = uu / K;
+                const int j = (int)(uu - pair * K);
+                t = (int)(pair / a.num_kv_heads);
+                kvh = (int)(pair % a.num_kv_heads);
+                s = seq_of(a, s_cuq, t);
+                p = __ldg(a.q_pos + t);
+                const int len = __ldg(a.seq_lens + s);
+                int n_sel = __ldg(a.cnt + t);
+                const int b = __ldg(a.sel + (size_t)t * a.k_max + j);
+                n_vis = p / kBlockSize + 1;
+                if (p < 0 || p >= len || n_vis > a.max_blocks || n_sel < 0 || n_sel > a.k_max) n_sel = 0;
+                if (j < n_sel) {
+                    if (b < 0 || b >= n_vis) {
+                        err_bits |= DSA_DEV_ERR_SEL;
+                    } else {
+                        const int pg = __ldg(a.block_table + (size_t)s * a.max_blocks + b);
+                        if (pg < 0 || pg >= a.num_pages) err_bits |= DSA_DEV_ERR_PAGE;
+                        else { blk = b; page = pg; }
+                    }
+                }
             }
-            return;
+            const long long chunk_end = min(u1, base + 32);
+            long long v = base;
+            while (v < chunk_end) {
+                const int lf = (int)(v - base);
+                const long long pair = v / K;
+                const long long seg_stop = min(u1, (pair + 1) * K);
+                const long long run_end = min(chunk_end, seg_stop);
+                const int ll = (int)(run_end - 1 - base);
+                const int pt = __shfl_sync(0xffffffffu, t, lf);
+                const int pkvh = __shfl_sync(0xffffffffu, kvh, lf);
+                const int pp = __shfl_sync(0xffffffffu, p, lf);
+                const int pnv = __shfl_sync(0xffffffffu, n_vis, lf);
+                if (v == u0 || v == pair * K) {
+                    // ---- segment header: pair facts + query tile into slot seg % 2
+                    const int qs = seg % kSegSlots;
+                    if (lane == 0) {
+                        bool ok = !*s_abort &&
+                                  (seg < kSegSlots || mbar_wait(sm.qempty(qs), ((seg / kSegSlots) - 1) & 1, s_abort));
+                        if (ok) {
+                            W[kWSegInfo + 4 * qs + 0] = pt;
+                            W[kWSegInfo + 4 * qs + 1] = pkvh;
+                            W[kWSegInfo + 4 * qs + 2] = pp;
+                            W[kWSegInfo + 4 * qs + 3] = pnv;
+                            __threadfence_block();
+                            mbar_arrive_expect_tx(sm.qfull(qs), kQSlotBytes);
+                            const int qrow = pt * a.num_q_heads + pkvh * G;
+                            tma_load_2d(sm.qslot(qs), &tm_q, 0, qrow, sm.qfull(qs));
+                            tma_load_2d(sm.qslot(qs) + kQHalf, &tm_q, 64, qrow, sm.qfull(qs));
+                        } else {
+                            *s_abort = 1;
+                        }
+                    }
+                    __syncwarp();
+                }
+                // ---- the run's usable blocks, in unit order
+                unsigned todo = __ballot_sync(0xffffffffu, in && lane >= lf && lane <= ll && blk >= 0);
+                while (todo) {
+                    const int src = __ffs(todo) - 1;
+                    todo &= todo - 1;
+                    const int ib = __shfl_sync(0xffffffffu, blk, src);
+                    const int ipg = __shfl_sync(0xffffffffu, page, src);
+                    if (lane == 0 && !*s_abort) {
+                        const int st = item % kStages;
+                        if (item >= kStages && !mbar_wait(sm.empty(st), ((item / kStages) - 1) & 1, s_abort)) {
+                            *s_abort = 1;
+                        } else {
+                            W[kWItemBlk + st] = ib;
+                            W[kWItemSeg + st] = seg;
+                            __threadfence_block();
+                            W[kWFill + st] = item;
+                            const uint32_t dst = sm.stage(st);
+                            mbar_arrive_expect_tx(sm.full(st), kStageBytes);
+                            const int z = ipg * kBlockSize;
+                            tma_load_3d(dst, &tm_k, 0, pkvh, z, sm.full(st));
+                            tma_load_3d(dst + kHalf, &tm_k, 64, pkvh, z, sm.full(st));
+                            tma_load_3d(dst + 2 * kHalf, &tm_v, 0, pkvh, z, sm.full(st));
+                            tma_load_3d(dst + 3 * kHalf, &tm_v, 64, pkvh, z, sm.full(st));
+                        }
+                    }
+                    ++item;
+                    __syncwarp();
+                }
+                if (run_end == seg_stop) {
+                    // ---- segment end marker
+                    if (lane == 0) {
+                        const int qs = seg % kSegSlots;
+                        W[kWSegEndCnt + qs] = item;
+                        __threadfence_block();
+                        W[kWSegEndTag + qs] = seg;
+                    }
+                    ++seg;
+                }
+                v = run_end;
+            }
+            stop = __shfl_sync(0xffffffffu, (int)*s_abort, 0) != 0;
         }
-        const __nv_bfloat16 *kb = a.k_pool + ((size_t)br.page * kBlockSize * a.num_kv_heads + kvh) * kHeadDim;
-        const __nv_bfloat16 *vb = a.v_pool + ((size_t)br.page * kBlockSize * a.num_kv_heads + kvh) * kHeadDim;
-#pragma unroll
-        for (int i = 0; i < (kBlockSize * 16) / kAttnThreads; ++i) {
-            const int e = tid + i * kAttnThreads;
-            const int r = e >> 4, ch = e & 15;
-            const size_t off = (size_t)r * row_elems + ch * 8;
-            cp_async_16(dk + swz(r, ch), kb + off);
-            cp_async_16(dv + swz(r, ch), vb + off);
+        err_bits = __reduce_or_sync(0xffffffffu, err_bits);
+        if (lane == 0) {
+            if (err_bits) set_err(a.dev_err, err_bits);
+            if (*s_abort) {
+                set_err(a.dev_err, DSA_DEV_ERR_WAIT);
+                // let the copies already issued land before the CTA exits: the
+                // last fill of each stage is the only one that can be in flight
+                for (int st = 0; st < kStages; ++st) {
+                    const int k = W[kWFill + st];
+                    if (k >= 0) mbar_wait(sm.full(st), (k / kStages) & 1, s_never);
+                }
+            }
         }
-    };
-
-#pragma unroll
-    for (int i = 0; i < kStages - 1; ++i) {
-        if (j0 + i < j1) load_block(j0 + i, i);
-        cp_async_commit();
+        return;
     }
 
-    // Q fragments stay in registers for the whole CTA
-    uint32_t qa[8][4];
-    float o[16][4];
-    float m_run[2] = {-INFINITY, -INFINITY};
-    float l_run[2] = {0.f, 0.f};
-#pragma unroll
-    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    // ==================================================================== consumer warps
+    const int g = lane >> 2, cq = lane & 3;
+    float *s_mo = reinterpret_cast<float *>(gbase + kOffMergeO);    // [4][16][kMergeStride]
+    float *s_ml = reinterpret_cast<float *>(gbase + kOffMergeML);   // [4][16][2]
 
-    bool q_loaded = false;
-    for (int j = j0; j < j1; ++j) {
-        cp_async_wait<kStages - 2>();
-        __syncthreads();
-        {
-            const int jn = j + kStages - 1;
-            if (jn < j1) load_block(jn, (jn - j0) % kStages);
-            cp_async_commit();
+    long long u = u0;
+    long long pair = u0 / K;
+    int cursor = 0, seg = 0;
+    while (u < u1) {
+        const long long seg_begin = u;
+        const long long seg_end = min(u1, (pair + 1) * K);
+        const int qs = seg % kSegSlots;
+        bool ok = !*s_abort && mbar_wait(sm.qfull(qs), (seg / kSegSlots) & 1, s_abort);
+        if (!ok) *s_abort = 1;
+        const int pt = W[kWSegInfo + 4 * qs + 0];
+        const int pkvh = W[kWSegInfo + 4 * qs + 1];
+        const int pp = W[kWSegInfo + 4 * qs + 2];
+        const int pnv = W[kWSegInfo + 4 * qs + 3];
+
+        // Q^T fragments (B operand of S^T = K Q^T): k = dims, n = query heads
+        uint32_t qb[8][NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int kp = 0; kp < 4; ++kp) {
+                qb[2 * kp][nt][0] = qb[2 * kp][nt][1] = qb[2 * kp + 1][nt][0] = qb[2 * kp + 1][nt][1] = 0u;
+                if (ok) {
+                    const int r = 8 * nt + (lane & 7);
+                    const int ch = 4 * kp + (lane >> 3);
+                    ldmatrix_x4(sm.qslot(qs) + (ch >> 3) * kQHalf + swz128(r, ch & 7), qb[2 * kp][nt][0],
+                                qb[2 * kp][nt][1], qb[2 * kp + 1][nt][0], qb[2 * kp + 1][nt][1]);
+                }
+            }
+        // O^T accumulators: dims 16*dm + g (+8) x heads 8*nt + 2*cq (+1)
+        float o[8][NT][4];
+        float m_run[NT][2], l_run[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            m_run[nt][0] = m_run[nt][1] = -INFINITY;
+            l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+            for (int dm = 0; dm < 8; ++dm) o[dm][nt][0] = o[dm][nt][1] = o[dm][nt][2] = o[dm][nt][3] = 0.f;
         }
-        if (!q_loaded) {
+
+        // this warp's items of the segment: indices cursor.. with index % 4 == warp
+        int ui = cursor + ((warp - cursor % kConsumerWarps) + kConsumerWarps) % kConsumerWarps;
+        while (true) {
+            const int st = ui % kStages;
+            // wait for item ui to be armed, or for this segment to end before it
+            bool done = false;
+            const long long t0 = clock64();
+            while (true) {
+                if (W[kWFill + st] == ui) {
+                    __threadfence_block();
+                    done = W[kWItemSeg + st] != seg;   // armed for a later segment: this one is over
+                    break;
+                }
+                if (W[kWSegEndTag + qs] == seg) {
+                    __threadfence_block();
+                    if (ui >= W[kWSegEndCnt + qs]) { done = true; break; }
+                }
+                if (*s_abort || clock64() - t0 > kWaitLimitCycles) { *s_abort = 1; done = true; break; }
+            }
+            __syncwarp();
+            if (done) break;
+            if (!mbar_wait(sm.full(st), (ui / kStages) & 1, s_abort)) {
+                *s_abort = 1;
+                break;
+            }
+            __syncwarp();
+            const int blk = W[kWItemBlk + st];
+            const uint32_t tk = sm.stage(st), tv = tk + 2 * kHalf;
+            // ---- S^T = K Q^T: 4 m-tiles of 16 tokens x NT n-tiles of 8 heads
+            float sc[4][NT][4];
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) sc[mt][nt][0] = sc[mt][nt][1] = sc[mt][nt][2] = sc[mt][nt][3] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                const int r = (lane & 7) + 8 * ((lane >> 3) & 1);
                 const int ch = 2 * kk + (lane >> 4);
-                ldmatrix_x4(sQ + swz(r, ch), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+                const uint32_t half = tk + (ch >> 3) * kHalf;
+#pragma unroll
+                for (int mt = 0; mt < 4; ++mt) {
+                    const int r = 16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1);
+                    uint32_t ka[4];
+                    ldmatrix_x4(half + swz128(r, ch & 7), ka[0], ka[1], ka[2], ka[3]);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sc[mt][nt], ka, qb[kk][nt][0], qb[kk][nt][1]);
+                }
             }
-            q_loaded = true;
+            // ---- causal mask (own block only), scale, online softmax per head column
+            const int lim = (blk == pnv - 1) ? pp - blk * kBlockSize : kBlockSize - 1;
+            float alpha[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+                for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int tok = 16 * mt + g + 8 * (k >> 1);
+                        const float x = tok <= lim ? sc[mt][nt][k] * a.scale_log2 : -INFINITY;
+                        sc[mt][nt][k] = x;
+                        mx[k & 1] = fmaxf(mx[k & 1], x);
+                    }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 4));
+                    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 8));
+                    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 16));
+                    const float m_new = fmaxf(m_run[nt][h], mx[h]);
+                    alpha[nt][h] = (m_new == -INFINITY) ? 1.f : exp2f(m_run[nt][h] - m_new);
+                    m_run[nt][h] = m_new;
+                }
+                float rs[2] = {0.f, 0.f};
+#pragma unroll
+                for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float mr = m_run[nt][k & 1];
+                        const float pv = (mr == -INFINITY) ? 0.f : exp2f(sc[mt][nt][k] - mr);
+                        sc[mt][nt][k] = pv;
+                        rs[k & 1] += pv;
+                    }
+                l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + rs[0];
+                l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + rs[1];
+#pragma unroll
+                for (int dm = 0; dm < 8; ++dm) {
+                    o[dm][nt][0] *= alpha[nt][0]; o[dm][nt][1] *= alpha[nt][1];
+                    o[dm][nt][2] *= alpha[nt][0]; o[dm][nt][3] *= alpha[nt][1];
+                }
+            }
+            // ---- O^T += V^T P^T: k-steps of 16 tokens; P^T fragments by movmatrix
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt) {
+                uint32_t pb[NT][2];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    pb[nt][0] = movmatrix_trans(pack_bf16x2(sc[mt][nt][0], sc[mt][nt][1]));
+                    pb[nt][1] = movmatrix_trans(pack_bf16x2(sc[mt][nt][2], sc[mt][nt][3]));
+                }
+                const int r = 16 * mt + (lane & 7) + 8 * (lane >> 4);
+#pragma unroll
+                for (int dm = 0; dm < 8; ++dm) {
+                    const int ch = 2 * dm + ((lane >> 3) & 1);
+                    uint32_t va[4];
+                    ldmatrix_x4_trans(tv + (ch >> 3) * kHalf + swz128(r, ch & 7), va[0], va[1], va[2], va[3]);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[dm][nt], va, pb[nt][0], pb[nt][1]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sm.empty(st));
+            ui += kConsumerWarps;
         }
-        const BlockRef br = block_ref(a, t, s, j, n_vis);
-        const int stage = (j - j0) % kStages;
-        const uint32_t tk = sKV + stage * 2 * kTileBytes;
-        const uint32_t tv = tk + kTileBytes;
-        const int tok0 = warp * 16;
+        // the segment's item count (published by the producer before it moves on)
+        {
+            const long long t0 = clock64();
+            while (W[kWSegEndTag + qs] != seg) {
+                if (*s_abort || clock64() - t0 > kWaitLimitCycles) { *s_abort = 1; break; }
+            }
+            __threadfence_block();
+        }
+        const int next_cursor = W[kWSegEndTag + qs] == seg ? W[kWSegEndCnt + qs] : cursor;
 
-        // ---- S = Q K^T for this warp's 16 tokens (two n8 tiles)
-        float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        // ---- end of this pair's units in the CTA: merge the four warps' states
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-            const int r = tok0 + (lane & 7) + 8 * (lane >> 4);
-            const int ch = 2 * kk + ((lane >> 3) & 1);
-            uint32_t b0, b1, b2, b3;
-            ldmatrix_x4(tk + swz(r, ch), b0, b1, b2, b3);
-            mma_bf16_16816(sc[0], qa[kk], b0, b1);
-            mma_bf16_16816(sc[1], qa[kk], b2, b3);
-        }
-        // ---- mask, scale, online softmax (rows g and g+8 of the head tile)
-        float mx[2] = {-INFINITY, -INFINITY};
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int pos = br.blk * kBlockSize + tok0 + nt * 8 + 2 * c + (e & 1);
-                const bool ok = br.blk >= 0 && pos <= p;
-                const float x = ok ? sc[nt][e] * a.scale_log2 : -INFINITY;
-                sc[nt][e] = x;
-                mx[e >> 1] = fmaxf(mx[e >> 1], x);
-            }
-        float alpha[2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-            mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-            const float m_new = fmaxf(m_run[r], mx[r]);
-            // all tokens so far masked: keep zero state, avoid (-inf) - (-inf)
-            alpha[r] = (m_new == -INFINITY) ? 1.f : exp2f(m_run[r] - m_new);
-            m_run[r] = m_new;
-        }
-        float rs[2] = {0.f, 0.f};
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float mr = m_run[e >> 1];
-                const float pv = (mr == -INFINITY) ? 0.f : exp2f(sc[nt][e] - mr);
-                sc[nt][e] = pv;
-                rs[e >> 1] += pv;
+            for (int h = 0; h < 2; ++h) {
+                l_run[nt][h] += __shfl_xor_sync(0xffffffffu, l_run[nt][h], 4);
+                l_run[nt][h] += __shfl_xor_sync(0xffffffffu, l_run[nt][h], 8);
+                l_run[nt][h] += __shfl_xor_sync(0xffffffffu, l_run[nt][h], 16);
             }
 #pragma unroll
-        for (int r = 0; r < 2; ++r) l_run[r] = l_run[r] * alpha[r] + rs[r];
+        for (int nt = 0; nt < NT; ++nt) {
+            const int h0 = 8 * nt + 2 * cq;
+            float *row0 = s_mo + (warp * 16 + h0) * kMergeStride;
+            float *row1 = row0 + kMergeStride;
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            o[n][0] *= alpha[0]; o[n][1] *= alpha[0];
-            o[n][2] *= alpha[1]; o[n][3] *= alpha[1];
+            for (int dm = 0; dm < 8; ++dm) {
+                const int d = 16 * dm + g;
+                row0[d] = o[dm][nt][0];
+                row1[d] = o[dm][nt][1];
+                row0[d + 8] = o[dm][nt][2];
+                row1[d + 8] = o[dm][nt][3];
+            }
+            if (g == 0) {
+                s_ml[(warp * 16 + h0) * 2] = m_run[nt][0];
+                s_ml[(warp * 16 + h0) * 2 + 1] = l_run[nt][0];
+                s_ml[(warp * 16 + h0 + 1) * 2] = m_run[nt][1];
+                s_ml[(warp * 16 + h0 + 1) * 2 + 1] = l_run[nt][1];
+            }
         }
-        // ---- O += P V
-        uint32_t pa[4];
-        pa[0] = pack_bf16x2(sc[0][0], sc[0][1]);
-        pa[1] = pack_bf16x2(sc[0][2], sc[0][3]);
-        pa[2] = pack_bf16x2(sc[1][0], sc[1][1]);
-        pa[3] = pack_bf16x2(sc[1][2], sc[1][3]);
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-            const int r = tok0 + (lane & 7) + 8 * ((lane >> 3) & 1);
-            const int ch = 2 * n + (lane >> 4);
-            uint32_t b0, b1, b2, b3;
-            ldmatrix_x4_trans(tv + swz(r, ch), b0, b1, b2, b3);
-            mma_bf16_16816(o[2 * n], pa, b0, b1);
-            mma_bf16_16816(o[2 * n + 1], pa, b2, b3);
-        }
-    }
-    cp_async_wait<0>();
-    __syncthreads();
+        __syncwarp();
+        named_barrier(1, kConsumerWarps * 32);
+        // every warp has read this slot's query tile, pair facts and end count
+        if (tid == 0) mbar_arrive(sm.qempty(qs));
 
-    // ---- merge the 4 warps' softmax states through shared memory
+        const bool whole = seg_begin == pair * K && seg_end == (pair + 1) * K;
+        const size_t out_row = (size_t)pt * a.num_q_heads + (size_t)pkvh * G;
+        const int slot = 2 * c + (seg == 0 ? 0 : 1);
+        for (int e = tid; e < G * 32; e += kConsumerWarps * 32) {
+            const int r = e >> 5, d0 = (e & 31) * 4;
+            float M = -INFINITY;
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 1);
-        l_run[r] += __shfl_xor_sync(0xffffffffu, l_run[r], 2);
-    }
-    float *s_o = reinterpret_cast<float *>(smem + kQBytes);      // [4][16][128]
-    float *s_m = s_o + 4 * 16 * kHeadDim;                          // [4][16]
-    float *s_l = s_m + 4 * 16;                                     // [4][16]
+            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, s_ml[(w * 16 + r) * 2]);
+            float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (M != -INFINITY) {
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {
-        float *row0 = s_o + (warp * 16 + g) * kHeadDim + n * 8 + 2 * c;
-        float *row1 = s_o + (warp * 16 + g + 8) * kHeadDim + n * 8 + 2 * c;
-        row0[0] = o[n][0]; row0[1] = o[n][1];
-        row1[0] = o[n][2]; row1[1] = o[n][3];
-    }
-    if (c == 0) {
-        s_m[warp * 16 + g] = m_run[0];
-        s_m[warp * 16 + g + 8] = m_run[1];
-        s_l[warp * 16 + g] = l_run[0];
-        s_l[warp * 16 + g + 8] = l_run[1];
-    }
-    __syncthreads();
-
-    // thread -> (row r, 4 consecutive dims); G rows x 32 dim-quads
-    const size_t unit = (size_t)t * a.num_q_heads + h0;   // first head row of this CTA
-    for (int e = tid; e < G * 32; e += kAttnThreads) {
-        const int r = e >> 5, d0 = (e & 31) * 4;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, s_m[w * 16 + r]);
-        float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float f = exp2f(s_m[w * 16 + r] - M);
-                L += s_l[w * 16 + r] * f;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) acc[k] += s_o[(w * 16 + r) * kHeadDim + d0 + k] * f;
+                for (int w = 0; w < kConsumerWarps; ++w) {
+                    const float f = exp2f(s_ml[(w * 16 + r) * 2] - M);
+                    L += s_ml[(w * 16 + r) * 2 + 1] * f;
+                    const float4 v = *reinterpret_cast<const float4 *>(s_mo + (w * 16 + r) * kMergeStride + d0);
+                    acc[0] += v.x * f; acc[1] += v.y * f; acc[2] += v.z * f; acc[3] += v.w * f;
+                }
+            }
+            if (whole) {
+                const float inv = L > 0.f ? 1.f / L : 0.f;
+                *reinterpret_cast<uint2 *>(a.out + (out_row + r) * kHeadDim + d0) =
+                    make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+                if (a.lse && d0 == 0) a.lse[out_row + r] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+            } else {
+                float *dst = a.part + ((size_t)slot * G + r) * kAttnPartStride;
+                *reinterpret_cast<float4 *>(dst + d0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                if (d0 == 0) { dst[128] = M; dst[129] = L; }
             }
         }
-        if (a.n_splits == 1) {
-            const float inv = L > 0.f ? 1.f / L : 0.f;
-            __nv_bfloat16 *dst = a.out + (unit + r) * kHeadDim + d0;
-            *reinterpret_cast<uint2 *>(dst) =
-                make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
-            if (a.lse && d0 == 0) a.lse[unit + r] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
-        } else {
-            const size_t pi = (unit + r) * a.n_splits + split;
-            *reinterpret_cast<float4 *>(a.part_o + pi * kHeadDim + d0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            if (d0 == 0) *reinterpret_cast<float2 *>(a.part_ml + pi * 2) = make_float2(M, L);
-        }
-    }
-    if (a.n_splits == 1) return;
-
-    // ---- the last CTA of this (query, KV head) merges the splits
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const int old = atomicAdd(a.counters + (size_t)t * a.num_kv_heads + kvh, 1);
-        s_last = (old == a.n_splits - 1);
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    for (int e = tid; e < G * 32; e += kAttnThreads) {
-        const int r = e >> 5, d0 = (e & 31) * 4;
-        const size_t pb = (unit + r) * a.n_splits;
-        float M = -INFINITY;
-        for (int sp = 0; sp < a.n_splits; ++sp) M = fmaxf(M, __ldcg(a.part_ml + (pb + sp) * 2));
-        float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (M != -INFINITY) {
-            for (int sp = 0; sp < a.n_splits; ++sp) {
-                const float2 ml = __ldcg(reinterpret_cast<const float2 *>(a.part_ml + (pb + sp) * 2));
-                if (ml.x == -INFINITY) continue;
-                const float f = exp2f(ml.x - M);
-                L += ml.y * f;
-                const float4 ov = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (pb + sp) * kHeadDim + d0));
-                acc[0] += ov.x * f; acc[1] += ov.y * f; acc[2] += ov.z * f; acc[3] += ov.w * f;
+        if (!whole) {
+            __threadfence();
+            __syncwarp();
+            named_barrier(1, kConsumerWarps * 32);
+            if (tid == 0) {
+                const int covered = (int)(seg_end - seg_begin);
+                const int old = atomicAdd(a.counters + pair, covered);
+                W[kWLast] = (old + covered == a.k_max);
+            }
+            __syncwarp();
+            named_barrier(1, kConsumerWarps * 32);
+            if (W[kWLast]) {
+                __threadfence();
+                // the CTAs covering this pair are this CTA's neighbours: walk
+                // out from c while their ranges still overlap the pair.  The
+                // per-warp merge buffers are free now and hold the slot list,
+                // each partial's (m, l) and its merge weight.
+                int *s_slot = reinterpret_cast<int *>(s_ml);        // [1 + kMaxSplitSlots]
+                float *s_pml = s_mo;                                 // [kMaxSplitSlots][16][2]
+                float *s_w = s_mo + kMaxSplitSlots * 32;             // [kMaxSplitSlots][16] weights
+                float *s_inv = s_w + kMaxSplitSlots * 16;            // [16] 1/L
+                float *s_lse = s_inv + 16;                           // [16]
+                if (tid == 0) {
+                    const long long p_lo = pair * K, p_hi = p_lo + K;
+                    int cf = c, cl = c;
+                    while (cf > 0 && range_begin(a, cf) > p_lo) --cf;
+                    while (cl + 1 < a.num_ctas && range_begin(a, cl + 1) < p_hi) ++cl;
+                    int n = 0;
+                    for (int cc = cf; cc <= cl && n < kMaxSplitSlots; ++cc, ++n)
+                        s_slot[1 + n] = 2 * cc + (range_begin(a, cc) >= p_lo ? 0 : 1);
+                    s_slot[0] = n;
+                }
+                __syncwarp();
+                named_barrier(1, kConsumerWarps * 32);
+                const int n_slots = s_slot[0];
+                // (m, l) of every partial row, all loads in flight at once
+                for (int e = tid; e < n_slots * G; e += kConsumerWarps * 32) {
+                    const int k = e / G, r = e % G;
+                    const float *src = a.part + ((size_t)s_slot[1 + k] * G + r) * kAttnPartStride;
+                    const float2 ml = __ldcg(reinterpret_cast<const float2 *>(src + 128));
+                    s_pml[(k * 16 + r) * 2] = ml.x;
+                    s_pml[(k * 16 + r) * 2 + 1] = ml.y;
+                }
+                __syncwarp();
+                named_barrier(1, kConsumerWarps * 32);
+                if (tid < G) {
+                    const int r = tid;
+                    float M = -INFINITY;
+                    for (int k = 0; k < n_slots; ++k) M = fmaxf(M, s_pml[(k * 16 + r) * 2]);
+                    float L = 0.f;
+                    for (int k = 0; k < n_slots; ++k) {
+                        const float mk = s_pml[(k * 16 + r) * 2];
+                        const float f = (M == -INFINITY || mk == -INFINITY) ? 0.f : exp2f(mk - M);
+                        s_w[k * 16 + r] = f;
+                        L += s_pml[(k * 16 + r) * 2 + 1] * f;
+                    }
+                    s_inv[r] = L > 0.f ? 1.f / L : 0.f;
+                    s_lse[r] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+                }
+                __syncwarp();
+                named_barrier(1, kConsumerWarps * 32);
+                for (int e = tid; e < G * 32; e += kConsumerWarps * 32) {
+                    const int r = e >> 5, d0 = (e & 31) * 4;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    for (int k0 = 0; k0 < n_slots; k0 += 4) {
+                        float4 v[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            v[k] = (k0 + k < n_slots)
+                                       ? __ldcg(reinterpret_cast<const float4 *>(
+                                             a.part + ((size_t)s_slot[1 + k0 + k] * G + r) * kAttnPartStride + d0))
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float f = (k0 + k < n_slots) ? s_w[(k0 + k) * 16 + r] : 0.f;
+                            acc[0] += v[k].x * f; acc[1] += v[k].y * f; acc[2] += v[k].z * f; acc[3] += v[k].w * f;
+                        }
+                    }
+                    const float inv = s_inv[r];
+                    *reinterpret_cast<uint2 *>(a.out + (out_row + r) * kHeadDim + d0) = make_uint2(
+                        pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+                    if (a.lse && d0 == 0) a.lse[out_row + r] = s_lse[r];
+                }
+                if (tid == 0) a.counters[pair] = 0;
             }
         }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        __nv_bfloat16 *dst = a.out + (unit + r) * kHeadDim + d0;
-        *reinterpret_cast<uint2 *>(dst) =
-            make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
-        if (a.lse && d0 == 0) a.lse[unit + r] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+        __syncwarp();
+        named_barrier(1, kConsumerWarps * 32);   // merge buffers free again
+        cursor = next_cursor;
+        u = seg_end;
+        ++pair;
+        ++seg;
     }
-    if (tid == 0) a.counters[(size_t)t * a.num_kv_heads + kvh] = 0;
 }
 
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+}  // namespace
+
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream) {
-    if (a.total_q == 0) return cudaSuccess;
-    // the shared-memory opt-in is a per-device function attribute
-    static unsigned long long attr_done = 0;
+    if (a.total_q == 0 || a.num_ctas == 0) return cudaSuccess;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    // K / V pool: dims (head_dim, kv_head, page*64+token), boxes of 64 dims x 1 head x 64 tokens
+    CUtensorMap tk, tv, tq;
+    const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)a.num_kv_heads,
+                                (cuuint64_t)a.num_pages * kBlockSize};
+    const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)a.num_kv_heads * kHeadDim * 2};
+    const cuuint32_t box[3] = {64, 1, kBlockSize};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(a.k_pool), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    if (enc(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(a.v_pool), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    // Q: rows (query, head), boxes of 64 dims x 16 rows; rows past the end read as zero
+    const cuuint64_t qdims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)a.total_q * a.num_q_heads};
+    const cuuint64_t qstr[1] = {(cuuint64_t)kHeadDim * 2};
+    const cuuint32_t qbox[2] = {64, 16};
+    if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(a.q), qdims, qstr, qbox, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+
+    static unsigned long long attr_done = 0;   // the shared-memory opt-in is per device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !(attr_done & (1ull << dev))) {
-        e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        e = cudaFuncSetAttribute(sparse_attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(sparse_attn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_done |= 1ull << dev;
     }
-    dim3 grid(a.total_q, a.num_kv_heads, a.n_splits);
-    sparse_attn_kernel<<<grid, kAttnThreads, kSmemBytes, stream>>>(a);
+    if (a.group <= 8)
+        sparse_attn_kernel<1><<<a.num_ctas, kAttnThreads, kSmemBytes, stream>>>(tk, tv, tq, a);
+    else
+        sparse_attn_kernel<2><<<a.num_ctas, kAttnThreads, kSmemBytes, stream>>>(tk, tv, tq, a);
     return cudaGetLastError();
 }
 

@@ -106,6 +106,13 @@ def decode_1m(batch: int = 8) -> WorkloadSpec:
                         k_per_seq=(32,) * batch, k_max=32, plant=32)
 
 
+def decode_128k(batch: int = 8) -> WorkloadSpec:
+    """decode_1m's shape at a 131,072-token context (2,048 blocks): the same
+    Top-K 32 attention work with a 4 GiB pool, small enough for profiling."""
+    return WorkloadSpec("decode_128k", seq_lens=(1 << 17,) * batch, n_new=(1,) * batch,
+                        k_per_seq=(32,) * batch, k_max=32, plant=32)
+
+
 def chunked_prefill(prefix: int = 131072, chunk: int = 4096) -> WorkloadSpec:
     """4096 new query tokens at positions 131072..135167 after a 128K prefix; K = 64."""
     return WorkloadSpec("chunked_prefill", seq_lens=(prefix + chunk,), n_new=(chunk,),
@@ -135,6 +142,7 @@ NAMED = {
     "tiny_decode": tiny_decode,
     "batched_gqa_decode": batched_gqa_decode,
     "decode_1m": decode_1m,
+    "decode_128k": decode_128k,
     "chunked_prefill": chunked_prefill,
     "mixed_ragged": mixed_ragged,
 }

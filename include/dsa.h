@@ -146,11 +146,33 @@ int dsa_index_score(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_q
  *   k_per_seq int32 [num_seqs], each in [1, k_max]
  *   sel      int32 [total_q][k_max]: LOGICAL block ids ascending, then -1
  *   cnt      int32 [total_q]: number of ids written
+ * max_blocks <= 32768 (a 2M-token context) in v1; longer tables use
+ * dsa_select_blocks.
  * Device errors: DSA_DEV_ERR_K (that query gets cnt 0), DSA_DEV_ERR_POS.
  */
 int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int32_t *scores,
                     const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt,
                     int32_t *dev_err, dsa_stream_t stream);
+
+/*
+ * dsa_select_blocks -- dsa_index_score and dsa_topk_blocks in one pass, with
+ * no score matrix in memory [P1 4(1): one fused scoring kernel with no
+ * intermediate written to memory, block-wise reduction + partial selection;
+ * P5 "Differentiated Adaptation of Prefill and Decode": fuse selection in
+ * decode].  Same arguments and the same sel / cnt results as the two calls;
+ * k_max <= 64 and max_blocks <= 131072 (an 8M-token context) in v1.  Each
+ * query's visible blocks are scored in chunks by separate CTAs that keep their
+ * local Top-(K-1); the last CTA of the query merges them.  Needs a workspace
+ * of dsa_select_blocks_workspace_size(total_q) bytes, zero-filled before its
+ * first use (each call leaves its counters at zero again).
+ * Device errors: DSA_DEV_ERR_PAGE, DSA_DEV_ERR_POS, DSA_DEV_ERR_K.
+ */
+size_t dsa_select_blocks_workspace_size(int32_t total_q);
+
+int dsa_select_blocks(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                      const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads, int32_t w_abs_max,
+                      const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt,
+                      void *workspace, size_t workspace_bytes, int32_t *dev_err, dsa_stream_t stream);
 
 /*
  * Exact attention over the selected blocks [P1 4(3) decode schematic; P3 4:
@@ -164,11 +186,13 @@ int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int3
  * bf16 inputs, fp32 accumulation, bf16 out.
  *   q   bf16 [total_q][num_q_heads][head_dim];  out bf16, same shape
  *   lse fp32 [total_q][num_q_heads] (may be NULL)
- * The decode entry splits each query's blocks over several CTAs and merges
- * the partial softmax states; it needs a workspace of
- * dsa_sparse_attn_decode_workspace_size() bytes, zero-filled before its first
- * use (each call leaves it zeroed again).  The prefill entry runs one CTA per
- * (query, KV head) and needs no workspace.
+ * Both entries run one persistent CTA per SM over the list of (query, KV
+ * head, selected block) units, split evenly.  The decode entry may split a
+ * (query, KV head) pair across CTAs and merge the partial softmax states; it
+ * needs a workspace of dsa_sparse_attn_decode_workspace_size() bytes (32
+ * bytes per (query, KV head) plus a fixed part), zero-filled before its first
+ * use (each call leaves it zeroed again).  The prefill entry keeps every pair
+ * inside one CTA and needs no workspace.
  * Device errors: DSA_DEV_ERR_SEL, DSA_DEV_ERR_PAGE (that block is skipped).
  */
 size_t dsa_sparse_attn_decode_workspace_size(int32_t total_q, int32_t num_q_heads,
@@ -196,8 +220,9 @@ int dsa_sparse_attn_prefill(const dsa_kv_cache *cache, const dsa_seqs *seqs,
  * the library, held on every GPU that loads the library until the process
  * exits.  The call allocates nothing.
  *  - Limit: dsa_sparse_attn_decode_workspace_size(total_q, num_q_heads,
- *    num_kv_heads, k_max) must be <= DSA_NOALLOC_SCRATCH_BYTES (e.g. 8 decode
- *    queries x 64 heads x Top-K 32 needs about 8.5 MiB); larger problems get
+ *    num_kv_heads, k_max) must be <= DSA_NOALLOC_SCRATCH_BYTES (with 8 query
+ *    heads per KV head that is about 2.1 MiB plus 4 bytes per (query, KV head),
+ *    so up to roughly 3.6 million (query, KV head) pairs); larger problems get
  *    DSA_ERR_WORKSPACE and nothing is launched.
  *  - The first call on each device (with that device current) looks up the
  *    scratch array's device address; make that first call before any stream

@@ -27,23 +27,23 @@ def _handles(wl):
             dsa.QueryBatch(wl.cu_q, wl.q_pos))
 
 
-def gpu_step(wl, decode=True, bufs=None):
+def gpu_step(wl, decode=True, bufs=None, fused=False):
     cache, seqs, queries = _handles(wl)
     err = torch.zeros(1, dtype=torch.int32, device=wl.device)
     bufs = dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
                     q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=wl.spec.k_max,
-                    decode=decode, bufs=bufs, dev_err=err)
+                    decode=decode, fused_select=fused, bufs=bufs, dev_err=err)
     torch.cuda.synchronize()
     return bufs, int(err.item())
 
 
-def compare(wl, ref, bufs, check_scores=True):
+def compare(wl, ref, bufs, check_scores=True, fused=False):
     qs = torch.as_tensor(ref["queries"], device=wl.device)
     sel = bufs["sel"].index_select(0, qs).cpu().numpy()
     cnt = bufs["cnt"].index_select(0, qs).cpu().numpy()
     assert np.array_equal(cnt, ref["cnt"]), "selection counts differ"
     assert np.array_equal(sel, ref["sel"]), "selected block ids differ"
-    if check_scores and "scores" in ref:
+    if check_scores and not fused and "scores" in ref:
         sc = bufs["scores"].index_select(0, qs).cpu().numpy().astype(np.int64)
         vis = ref["scores"] != np.iinfo(np.int64).min
         assert np.array_equal(sc[vis], ref["scores"][vis]), "block scores differ"
@@ -55,10 +55,10 @@ def compare(wl, ref, bufs, check_scores=True):
     return d.max(), d.mean()
 
 
-def _run(spec, seed, device, queries=None, decode=True, scores=True):
+def _run(spec, seed, device, queries=None, decode=True, scores=True, fused=False):
     wl = wk.make_workload(spec, seed=seed, device=device)
     ref = oracle_step(wl, queries=queries, want_scores=scores)
-    bufs, err = gpu_step(wl, decode=decode)
+    bufs, err = gpu_step(wl, decode=decode, fused=fused)
     assert err == 0, f"device error bits {err}"
     return wl, ref, bufs
 
@@ -87,30 +87,34 @@ def _small_spec(name, q_scale=1.0):
     return wk.WorkloadSpec(name, q_scale=q_scale, **kw)
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["score_topk", "fused_select"])
 @pytest.mark.parametrize("decode", [True, False], ids=["decode_entry", "prefill_entry"])
 @pytest.mark.parametrize("q_scale", [1.0, 12.0], ids=["plain", "sharp"])
 @pytest.mark.parametrize("name", sorted(SMALL))
-def test_small_cases_all_outputs(name, q_scale, decode, cuda_device):
-    wl, ref, bufs = _run(_small_spec(name, q_scale), 100 + len(name), cuda_device, decode=decode)
-    compare(wl, ref, bufs)
+def test_small_cases_all_outputs(name, q_scale, decode, fused, cuda_device):
+    wl, ref, bufs = _run(_small_spec(name, q_scale), 100 + len(name), cuda_device, decode=decode, fused=fused)
+    compare(wl, ref, bufs, fused=fused)
 
 
-def test_tiny_decode_workload(cuda_device):
-    wl, ref, bufs = _run(wk.tiny_decode(), 1001, cuda_device)
-    compare(wl, ref, bufs)
+@pytest.mark.parametrize("fused", [False, True], ids=["score_topk", "fused_select"])
+def test_tiny_decode_workload(fused, cuda_device):
+    wl, ref, bufs = _run(wk.tiny_decode(), 1001, cuda_device, fused=fused)
+    compare(wl, ref, bufs, fused=fused)
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["score_topk", "fused_select"])
 @pytest.mark.parametrize("q_scale", [1.0, 12.0])
-def test_batched_gqa_decode_workload(q_scale, cuda_device):
+def test_batched_gqa_decode_workload(q_scale, fused, cuda_device):
     spec = wk.scaled(wk.batched_gqa_decode(), q_scale=q_scale)
-    wl, ref, bufs = _run(spec, 1002, cuda_device)
-    compare(wl, ref, bufs)
+    wl, ref, bufs = _run(spec, 1002, cuda_device, fused=fused)
+    compare(wl, ref, bufs, fused=fused)
 
 
 @pytest.mark.slow
-def test_decode_1m_workload_all_outputs(cuda_device):
-    wl, ref, bufs = _run(wk.decode_1m(), 1003, cuda_device)
-    compare(wl, ref, bufs)
+@pytest.mark.parametrize("fused", [False, True], ids=["score_topk", "fused_select"])
+def test_decode_1m_workload_all_outputs(fused, cuda_device):
+    wl, ref, bufs = _run(wk.decode_1m(), 1003, cuda_device, fused=fused)
+    compare(wl, ref, bufs, fused=fused)
     # the planted blocks shape the selection (non-trivial selections)
     planted = wl.planted.cpu().numpy()
     hits = [len(set(ref["sel"][s]) & set(planted[s])) for s in range(8)]
@@ -144,8 +148,8 @@ def test_chunked_prefill_workload_sampled(cuda_device):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("decode", [True, False])
-def test_mixed_ragged_workload_sampled(decode, cuda_device):
+@pytest.mark.parametrize("decode,fused", [(True, False), (False, False), (True, True)])
+def test_mixed_ragged_workload_sampled(decode, fused, cuda_device):
     spec = wk.mixed_ragged()
     wl = wk.make_workload(spec, seed=1005, device=cuda_device)
     cu = wl.cu_q.cpu().numpy()
@@ -155,9 +159,9 @@ def test_mixed_ragged_workload_sampled(decode, cuda_device):
                  for x in rng.choice(np.arange(cu[s], cu[s + 1]), size=12, replace=False)]
     qs = sorted(decode_q + prefill_q)
     ref = oracle_step(wl, queries=qs, want_scores=True)
-    bufs, err = gpu_step(wl, decode=decode)
+    bufs, err = gpu_step(wl, decode=decode, fused=fused)
     assert err == 0
-    compare(wl, ref, bufs)
+    compare(wl, ref, bufs, fused=fused)
 
 
 # ----------------------------------------------------------------------------- invariants on the GPU
@@ -205,20 +209,22 @@ def test_repeat_calls_reuse_workspace(cuda_device):
 
 
 # ----------------------------------------------------------------------------- device error flags
-def test_bad_page_sets_flag_without_fault(cuda_device):
+@pytest.mark.parametrize("fused", [False, True])
+def test_bad_page_sets_flag_without_fault(fused, cuda_device):
     spec = _small_spec("k_covers_all")
     wl = wk.make_workload(spec, seed=10, device=cuda_device)
     wl.block_table[0, 1] = spec.num_pages + 5
-    _, err = gpu_step(wl)
+    _, err = gpu_step(wl, fused=fused)
     assert err & dsa._lib.DEV_ERR_PAGE
 
 
-def test_bad_position_and_k_set_flags(cuda_device):
+@pytest.mark.parametrize("fused", [False, True])
+def test_bad_position_and_k_set_flags(fused, cuda_device):
     spec = _small_spec("k_covers_all")
     wl = wk.make_workload(spec, seed=11, device=cuda_device)
     wl.q_pos[1] = int(wl.seq_lens[1]) + 3          # past the end of its sequence
     wl.k_per_seq[0] = 0
-    b, err = gpu_step(wl)
+    b, err = gpu_step(wl, fused=fused)
     assert err & dsa._lib.DEV_ERR_POS
     assert err & dsa._lib.DEV_ERR_K
     assert int(b["cnt"][0]) == 0 and int(b["cnt"][1]) == 0
@@ -232,3 +238,20 @@ def test_host_validation_raises(cuda_device):
         dsa.index_score(cache, seqs, queries, wl.q_idx, wl.w, w_abs_max=1 << 12)
     with pytest.raises(ValueError):
         dsa.index_score(cache, seqs, queries, wl.q_idx.cpu(), wl.w)
+
+
+def test_fused_select_equals_score_then_topk_on_ties(cuda_device):
+    # all-equal coarse keys: every candidate ties, so the selection is decided
+    # by the lowest-id rule alone, across chunk boundaries of the fused path
+    spec = wk.WorkloadSpec("ties", seq_lens=(40000, 1500), n_new=(1, 3), k_per_seq=(33, 64), k_max=64,
+                           num_q_heads=16, num_kv_heads=2)
+    wl = wk.make_workload(spec, seed=31, device=cuda_device)
+    wl.kc_pool.fill_(3)
+    wl.kc_new.fill_(3)
+    b1, e1 = gpu_step(wl, fused=False)
+    b2, e2 = gpu_step(wl, fused=True)
+    assert e1 == e2 == 0
+    assert torch.equal(b1["sel"], b2["sel"]) and torch.equal(b1["cnt"], b2["cnt"])
+    own = (wl.q_pos // 64).cpu()
+    sel = b1["sel"].cpu()
+    assert sel[0, :32].tolist() == list(range(32)) and int(sel[0, 32]) == int(own[0])

@@ -51,10 +51,17 @@ def test_noalloc_matches_regular_decode_twice(name, spec, cuda_device):
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
-    spec = wk.WorkloadSpec("na3", seq_lens=(5000,) * 64, n_new=(1,) * 64, k_per_seq=(64,) * 64, k_max=64)
-    wl, cache, seqs, queries, sel, cnt = _setup(spec, 78, cuda_device)
-    need = dsa.decode_workspace_size(spec.total_q, spec.num_q_heads, spec.num_kv_heads, spec.k_max)
+    # 600,000 queries x 8 KV heads need more than the fixed 16 MiB scratch; the
+    # call must refuse before touching any memory (the pointers are dummies)
+    import ctypes
+    lib = dsa._lib.load()
+    L = dsa._lib
+    fake = 0x10000
+    cache = L.KvCacheC(fake, fake, fake, 4, 64, 8, 128, 64)
+    seqs = L.SeqsC(fake, 4, fake, 1)
+    queries = L.QueriesC(fake, fake, 600000)
+    need = lib.dsa_sparse_attn_decode_workspace_size(600000, 64, 8, 32)
     assert need > 16 << 20
-    with pytest.raises(dsa.DsaError) as e:
-        dsa.sparse_attn_decode_noalloc(cache, seqs, queries, wl.q, sel, cnt)
-    assert e.value.status == dsa._lib.DSA_ERR_WORKSPACE
+    rc = lib.dsa_sparse_attn_decode_noalloc(ctypes.byref(cache), ctypes.byref(seqs), ctypes.byref(queries),
+                                            fake, 64, fake, fake, 32, 0.088, fake, None, None, None)
+    assert rc == L.DSA_ERR_WORKSPACE
