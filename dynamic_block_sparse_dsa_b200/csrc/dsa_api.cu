@@ -58,7 +58,7 @@ DecodeLayout decode_layout(int total_q, int hq, int hkv) {
     return L;
 }
 
-// select workspace: [counters int32 T][candidates uint2 T*kSelMaxChunks*(kSelMaxK-1)]
+// select workspace: [counters int32 T][candidate keys u64 T*kSelMaxChunks*(kSelMaxK-1)]
 struct SelectLayout {
     size_t counters, cand, total;
 };
@@ -66,7 +66,7 @@ SelectLayout select_layout(int total_q) {
     SelectLayout L;
     L.counters = 0;
     L.cand = align_up((size_t)total_q * sizeof(int32_t), 256);
-    L.total = align_up(L.cand + (size_t)total_q * kSelMaxChunks * (kSelMaxK - 1) * sizeof(uint2), 256);
+    L.total = align_up(L.cand + (size_t)total_q * kSelMaxChunks * (kSelMaxK - 1) * sizeof(unsigned long long), 256);
     return L;
 }
 
@@ -210,7 +210,7 @@ int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int3
     int rc;
     if ((rc = check_seqs(seqs)) || (rc = check_queries(queries))) return rc;
     if (k_max < 1) return DSA_ERR_INVALID_ARG;
-    if (seqs->max_blocks > topk_max_blocks()) return DSA_ERR_UNSUPPORTED;
+    if (k_max > kSelMaxK || seqs->max_blocks > topk_max_blocks()) return DSA_ERR_UNSUPPORTED;
     if (queries->total_q == 0) return DSA_OK;
     if (!scores || !k_per_seq || !sel || !cnt) return DSA_ERR_INVALID_ARG;
     TopkArgs a{};
@@ -268,7 +268,7 @@ int dsa_select_blocks(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa
     a.cnt = cnt;
     char *ws = static_cast<char *>(workspace);
     a.counters = reinterpret_cast<int32_t *>(ws + L.counters);
-    a.cand = reinterpret_cast<uint2 *>(ws + L.cand);
+    a.cand = reinterpret_cast<unsigned long long *>(ws + L.cand);
     a.dev_err = dev_err;
     return from_cuda(launch_select_blocks(a, reinterpret_cast<cudaStream_t>(stream)));
 }

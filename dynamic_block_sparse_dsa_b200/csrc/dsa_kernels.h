@@ -72,7 +72,7 @@ struct SelectArgs {
     int k_max;
     int32_t *sel;            // [T][k_max]
     int32_t *cnt;            // [T]
-    uint2 *cand;             // [T][kSelMaxChunks][kSelMaxK-1] (order key, block id)
+    unsigned long long *cand;   // [T][kSelMaxChunks][kSelMaxK-1] 64-bit selection keys, sorted descending
     int32_t *counters;       // [T] chunk CTAs done per query
     int32_t *dev_err;
 };

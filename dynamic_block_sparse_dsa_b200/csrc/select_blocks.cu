@@ -11,33 +11,54 @@
 // Grid: (query, chunk of 256*E candidate blocks).  Each CTA scores its chunk
 // with the CUDA-core int8 indexer (one thread per E consecutive blocks: page
 // id, 64-byte coarse key, dp4a), keeps the chunk's local Top-(K-1) in id order
-// (exact radix select on register-resident keys) and writes it to the
-// workspace.  The last CTA of the query -- elected with an atomic counter,
-// nothing waits -- merges the chunks' candidates with the same selection,
-// appends the query's own block and writes the ascending selection.  Result
-// is identical to dsa_index_score followed by dsa_topk_blocks.
+// (warp-level bitonic Top-64 on unique 64-bit keys, then a merge tree over
+// the warps) and writes it to the workspace.  The last CTA of the query --
+// elected with an atomic counter, nothing waits -- merges the chunks' sorted
+// lists the same way, appends the query's own block and writes the ascending
+// selection.  Result is identical to dsa_index_score followed by
+// dsa_topk_blocks.
 #include "dsa_kernels.h"
 #include "indexer_core.cuh"
-#include "select_core.cuh"
+#include "warp_topk.cuh"
 
 namespace dsa {
 
 namespace {
 constexpr int kSelThreads = 256;
-constexpr int kMergeE = kSelMaxChunks * (kSelMaxK - 1) / kSelThreads + 1;   // candidates per thread
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kCuqCache = 1024;   // cu_q entries staged in shared memory
 }  // namespace
 
 template <int E>
 __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a) {
-    __shared__ SelectSmem sh;
     __shared__ int4 s_q[kMaxIdxHeads][kIdxDim / 16];
     __shared__ int s_w[kMaxIdxHeads];
+    __shared__ int s_cuq[kCuqCache + 1];
+    __shared__ key64 s_lists[kSelWarps * 64];
     __shared__ int s_last;
     constexpr int CH = kSelThreads * E;
-    const int t = blockIdx.x, c = blockIdx.y, tid = threadIdx.x;
+    const int t = blockIdx.x, c = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = a.num_idx_heads;
 
-    const int s = find_seq(a.cu_q, a.num_seqs, t);
+    // ---- query facts: the sequence from a shared-memory copy of cu_q
+    const bool cached = a.num_seqs + 1 <= kCuqCache;
+    if (cached)
+        for (int i = tid; i <= a.num_seqs; i += kSelThreads) s_cuq[i] = __ldg(a.cu_q + i);
+    for (int e = tid; e < H * 4; e += kSelThreads)
+        s_q[e >> 2][e & 3] = __ldg(reinterpret_cast<const int4 *>(a.q_idx + (size_t)t * H * kIdxDim) + e);
+    if (tid < H) s_w[tid] = __ldg(a.w + (size_t)t * H + tid);
+    __syncthreads();
+    int s;
+    if (cached) {
+        int lo = 0, hi = a.num_seqs - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_cuq[mid] <= t) lo = mid; else hi = mid - 1;
+        }
+        s = lo;
+    } else {
+        s = find_seq(a.cu_q, a.num_seqs, t);
+    }
     const int p = __ldg(a.q_pos + t);
     const int len = __ldg(a.seq_lens + s);
     const int K = __ldg(a.k_per_seq + s);
@@ -68,27 +89,20 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     const int n_chunks = (own + CH - 1) / CH;   // candidates: blocks 0 .. own-1
     if (c >= n_chunks) return;
 
-    // ---- score this chunk (E consecutive blocks per thread)
-    for (int e = tid; e < H * 4; e += kSelThreads)
-        s_q[e >> 2][e & 3] = __ldg(reinterpret_cast<const int4 *>(a.q_idx + (size_t)t * H * kIdxDim) + e);
-    if (tid < H) s_w[tid] = __ldg(a.w + (size_t)t * H + tid);
-    __syncthreads();
-    uint32_t key[E];
-    bool valid[E];
+    // ---- score this chunk: E consecutive blocks per thread
+    key64 key[E];
     uint32_t err_bits = 0;
     const int b0 = c * CH + tid * E;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const int b = b0 + e;
-        valid[e] = false;
         key[e] = 0;
         if (b < own) {
             const int page = __ldg(a.block_table + (size_t)s * a.max_blocks + b);
             if (page >= 0 && page < a.num_pages) {
                 int kc[16];
                 load_coarse_key(a.kc_pool, page, kc);
-                key[e] = order_key(block_score(kc, s_q, s_w, H));
-                valid[e] = true;
+                key[e] = make_key64(block_score(kc, s_q, s_w, H), (uint32_t)b);
             } else {
                 err_bits |= DSA_DEV_ERR_PAGE;
             }
@@ -96,32 +110,23 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     }
     if (err_bits) set_err(a.dev_err, err_bits);
 
-    // ---- local Top-kk of the chunk, written in id order
-    int nv = 0;
+    // ---- chunk Top-64: per warp, then a merge tree over the warps
+    key64 acc[2];
 #pragma unroll
-    for (int e = 0; e < E; ++e) nv += valid[e];
-    int n_valid;
-    cta_exclusive_scan<kSelThreads>(nv, sh, &n_valid);
-    const int kl = min(kk, n_valid);
-    bool take[E];
-    if (kl == n_valid) {
-#pragma unroll
-        for (int e = 0; e < E; ++e) take[e] = valid[e];
-    } else {
-        cta_select<kSelThreads, E>(key, valid, kl, take, sh);
+    for (int g = 0; g < (E + 1) / 2; ++g) {
+        key64 v[2] = {key[2 * g], 2 * g + 1 < E ? key[2 * g + 1] : 0ull};
+        warp_sort64_desc(v);
+        if (g == 0) { acc[0] = v[0]; acc[1] = v[1]; }
+        else warp_merge64_desc(acc, v);
     }
-    int nt = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) nt += take[e];
-    int tot;
-    int pos = cta_exclusive_scan<kSelThreads>(nt, sh, &tot);
-    uint2 *cand = a.cand + ((size_t)t * kSelMaxChunks + c) * (kSelMaxK - 1);
-#pragma unroll
-    for (int e = 0; e < E; ++e)
-        if (take[e]) cand[pos++] = make_uint2(key[e], (uint32_t)(b0 + e));
-    for (int i = kl + tid; i < kk; i += kSelThreads) cand[i] = make_uint2(0u, 0xffffffffu);   // padding
+    cta_merge_top64<kSelWarps>(acc, s_lists);
+    key64 *cand = a.cand + ((size_t)t * kSelMaxChunks + c) * (kSelMaxK - 1);
+    if (warp == 0) {
+        if (lane < kk) cand[lane] = acc[0];
+        if (32 + lane < kk) cand[32 + lane] = acc[1];
+    }
 
-    // ---- the last chunk CTA of this query merges
+    // ---- the last chunk CTA of this query merges the chunks' lists
     __threadfence();
     __syncthreads();
     if (tid == 0) {
@@ -131,50 +136,29 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-
-    const int n_cand = n_chunks * kk;
-    uint32_t mk[kMergeE];
-    uint32_t mid[kMergeE];
-    bool mv[kMergeE];
-#pragma unroll
-    for (int e = 0; e < kMergeE; ++e) {
-        const int i = tid * kMergeE + e;
-        mv[e] = false;
-        mk[e] = 0;
-        mid[e] = 0;
-        if (i < n_cand) {
-            const int ci = i / kk, j = i - ci * kk;
-            const uint2 v = __ldcg(a.cand + ((size_t)t * kSelMaxChunks + ci) * (kSelMaxK - 1) + j);
-            mk[e] = v.x;
-            mid[e] = v.y;
-            mv[e] = v.y != 0xffffffffu;
+    acc[0] = acc[1] = 0ull;
+    for (int ci = warp; ci < n_chunks; ci += kSelWarps) {
+        const key64 *src = a.cand + ((size_t)t * kSelMaxChunks + ci) * (kSelMaxK - 1);
+        const key64 b[2] = {lane < kk ? __ldcg(src + lane) : 0ull, 32 + lane < kk ? __ldcg(src + 32 + lane) : 0ull};
+        if (ci == warp) { acc[0] = b[0]; acc[1] = b[1]; }
+        else warp_merge64_desc(acc, b);
+    }
+    cta_merge_top64<kSelWarps>(acc, s_lists);
+    if (warp == 0) {
+        // the winners (non-zero keys among the first kk) in ascending block order
+        const bool v0 = lane < kk && acc[0] != 0ull, v1 = 32 + lane < kk && acc[1] != 0ull;
+        const int km = __popc(__ballot_sync(0xffffffffu, v0)) + __popc(__ballot_sync(0xffffffffu, v1));
+        uint32_t ids[2] = {v0 ? key64_id(acc[0]) : 0xffffffffu, v1 ? key64_id(acc[1]) : 0xffffffffu};
+        warp_sort64_asc_u32(ids);
+        if (lane < km) out[lane] = (int32_t)ids[0];
+        if (32 + lane < km) out[32 + lane] = (int32_t)ids[1];
+        if (lane == 0) {
+            out[km] = own;              // the own block: the largest visible id, last in order
+            a.cnt[t] = km + 1;
+            a.counters[t] = 0;          // ready for the next call
         }
+        for (int i = km + 1 + lane; i < a.k_max; i += 32) out[i] = -1;
     }
-    nv = 0;
-#pragma unroll
-    for (int e = 0; e < kMergeE; ++e) nv += mv[e];
-    cta_exclusive_scan<kSelThreads>(nv, sh, &n_valid);
-    const int km = min(kk, n_valid);
-    bool mt[kMergeE];
-    if (km == n_valid) {
-#pragma unroll
-        for (int e = 0; e < kMergeE; ++e) mt[e] = mv[e];
-    } else {
-        cta_select<kSelThreads, kMergeE>(mk, mv, km, mt, sh);
-    }
-    nt = 0;
-#pragma unroll
-    for (int e = 0; e < kMergeE; ++e) nt += mt[e];
-    pos = cta_exclusive_scan<kSelThreads>(nt, sh, &tot);
-#pragma unroll
-    for (int e = 0; e < kMergeE; ++e)
-        if (mt[e]) out[pos++] = (int32_t)mid[e];
-    if (tid == 0) {
-        out[km] = own;              // the own block: the largest visible id, last in order
-        a.cnt[t] = km + 1;
-        a.counters[t] = 0;          // ready for the next call
-    }
-    for (int i = km + 1 + tid; i < a.k_max; i += kSelThreads) out[i] = -1;
 }
 
 cudaError_t launch_select_blocks(const SelectArgs &a, cudaStream_t stream) {

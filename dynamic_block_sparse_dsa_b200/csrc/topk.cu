@@ -7,24 +7,24 @@
 // Selection Path": the indices follow the gather's semantics; here they are
 // logical block ids, ascending, -1 padded.
 //
-// One CTA of 1024 threads per query.  The candidates (blocks 0..n-2; the own
-// block n-1 is always kept) are loaded once into registers, E consecutive
-// blocks per thread, and the K-1 winners under (score descending, block id
-// ascending) are found by the radix selection of select_core.cuh; a prefix
-// count over the threads writes them in ascending id order without a sort.
+// One CTA of 1024 threads per query.  Each warp streams groups of 64
+// candidates (coalesced loads), sorts each group with a warp bitonic network
+// and folds it into its running Top-64 (warp_topk.cuh); a merge tree over the
+// 32 warps leaves the query's Top-64 in warp 0, which appends the own block
+// and writes the winners in ascending block order.
 #include "dsa_kernels.h"
-#include "select_core.cuh"
+#include "warp_topk.cuh"
 
 namespace dsa {
 
 namespace {
 constexpr int kTopkThreads = 1024;
+constexpr int kTopkWarps = kTopkThreads / 32;
 }  // namespace
 
-template <int E>
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
-    __shared__ SelectSmem sh;
-    const int t = blockIdx.x, tid = threadIdx.x;
+    __shared__ key64 s_lists[kTopkWarps * 64];
+    const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int32_t *out = a.sel + (size_t)t * a.k_max;
     const int s = find_seq(a.cu_q, a.num_seqs, t);
     const int p = __ldg(a.q_pos + t);
@@ -49,43 +49,37 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     const int n = n_vis - 1;   // candidates 0..n-1 (n >= K)
     const int kk = K - 1;
     const int32_t *row = a.scores + (size_t)t * a.max_blocks;
-    uint32_t key[E];
-    bool valid[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const int b = tid * E + e;
-        valid[e] = b < n;
-        key[e] = valid[e] ? order_key(__ldg(row + b)) : 0u;
+    key64 acc[2] = {0ull, 0ull};
+    bool first = true;
+    for (int g0 = warp * 64; g0 < n; g0 += kTopkWarps * 64) {
+        const int i0 = g0 + lane, i1 = g0 + 32 + lane;
+        key64 v[2] = {i0 < n ? make_key64(__ldg(row + i0), (uint32_t)i0) : 0ull,
+                      i1 < n ? make_key64(__ldg(row + i1), (uint32_t)i1) : 0ull};
+        warp_sort64_desc(v);
+        if (first) { acc[0] = v[0]; acc[1] = v[1]; first = false; }
+        else warp_merge64_desc(acc, v);
     }
-    bool take[E];
-    cta_select<kTopkThreads, E>(key, valid, kk, take, sh);
-    int nt = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) nt += take[e];
-    int tot;
-    int pos = cta_exclusive_scan<kTopkThreads>(nt, sh, &tot);
-#pragma unroll
-    for (int e = 0; e < E; ++e)
-        if (take[e]) out[pos++] = tid * E + e;
-    if (tid == 0) {
-        out[kk] = n;   // the own block, the largest visible id
-        a.cnt[t] = K;
+    cta_merge_top64<kTopkWarps>(acc, s_lists);
+    if (warp == 0) {
+        const bool v0 = lane < kk, v1 = 32 + lane < kk;
+        uint32_t ids[2] = {v0 ? key64_id(acc[0]) : 0xffffffffu, v1 ? key64_id(acc[1]) : 0xffffffffu};
+        warp_sort64_asc_u32(ids);
+        if (v0) out[lane] = (int32_t)ids[0];
+        if (v1) out[32 + lane] = (int32_t)ids[1];
+        if (lane == 0) {
+            out[kk] = n;   // the own block, the largest visible id
+            a.cnt[t] = K;
+        }
+        for (int i = K + lane; i < a.k_max; i += 32) out[i] = -1;
     }
-    for (int i = K + tid; i < a.k_max; i += kTopkThreads) out[i] = -1;
 }
 
-int topk_max_blocks() { return kTopkThreads * 32; }
+int topk_max_blocks() { return 1 << 20; }
 
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
     if (a.total_q == 0) return cudaSuccess;
-    const int e = (a.max_blocks + kTopkThreads - 1) / kTopkThreads;
-    if (e <= 1) topk_kernel<1><<<a.total_q, kTopkThreads, 0, stream>>>(a);
-    else if (e <= 2) topk_kernel<2><<<a.total_q, kTopkThreads, 0, stream>>>(a);
-    else if (e <= 4) topk_kernel<4><<<a.total_q, kTopkThreads, 0, stream>>>(a);
-    else if (e <= 8) topk_kernel<8><<<a.total_q, kTopkThreads, 0, stream>>>(a);
-    else if (e <= 16) topk_kernel<16><<<a.total_q, kTopkThreads, 0, stream>>>(a);
-    else if (e <= 32) topk_kernel<32><<<a.total_q, kTopkThreads, 0, stream>>>(a);
-    else return cudaErrorInvalidValue;   // the host rejects longer tables first
+    if (a.k_max > 64) return cudaErrorInvalidValue;   // the host rejects these first
+    topk_kernel<<<a.total_q, kTopkThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -146,8 +146,7 @@ int dsa_index_score(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_q
  *   k_per_seq int32 [num_seqs], each in [1, k_max]
  *   sel      int32 [total_q][k_max]: LOGICAL block ids ascending, then -1
  *   cnt      int32 [total_q]: number of ids written
- * max_blocks <= 32768 (a 2M-token context) in v1; longer tables use
- * dsa_select_blocks.
+ * k_max <= 64 in v1.
  * Device errors: DSA_DEV_ERR_K (that query gets cnt 0), DSA_DEV_ERR_POS.
  */
 int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int32_t *scores,
