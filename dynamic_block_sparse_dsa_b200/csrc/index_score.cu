@@ -29,6 +29,8 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_dp4a_kernel(IndexSc
     __shared__ int s_w[kQBatch][kMaxIdxHeads];
     __shared__ int s_own[kQBatch];
 
+    pdl_trigger();
+    pdl_wait();   // coarse keys may come from the preceding append
     const int s = blockIdx.y;
     const int q0 = __ldg(a.cu_q + s), q1 = __ldg(a.cu_q + s + 1);
     if (q1 <= q0) return;
@@ -88,8 +90,7 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_dp4a_kernel(IndexSc
 cudaError_t launch_index_score(const IndexScoreArgs &a, cudaStream_t stream) {
     if (a.total_q == 0 || a.num_seqs == 0) return cudaSuccess;
     dim3 grid((a.max_blocks + kScoreThreads - 1) / kScoreThreads, a.num_seqs);
-    index_score_dp4a_kernel<<<grid, kScoreThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(index_score_dp4a_kernel, grid, dim3(kScoreThreads), 0, stream, a);
 }
 
 }  // namespace dsa

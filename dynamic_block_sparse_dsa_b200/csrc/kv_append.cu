@@ -12,6 +12,7 @@
 namespace dsa {
 
 __global__ void __launch_bounds__(128) kv_append_kernel(KvAppendArgs a) {
+    pdl_trigger();   // the next kernel may start its prologue; it waits for us before reading
     const int i = blockIdx.x;
     const int s = find_seq(a.cu_new, a.num_seqs, i);
     const int first = __ldg(a.cu_new + s), last = __ldg(a.cu_new + s + 1);

@@ -8,9 +8,11 @@
 // Prefill and Decode": fuse index selection for decode to cut launches and
 // write-backs.
 //
-// Grid: (query, chunk of 256*E candidate blocks).  Each CTA scores its chunk
-// with the CUDA-core int8 indexer (one thread per E consecutive blocks: page
-// id, 64-byte coarse key, dp4a), keeps the chunk's local Top-(K-1) in id order
+// Grid: (query, chunk of 512*G candidate blocks).  Each CTA scores its chunk
+// with the int8 indexer on the tensor cores (mma.m16n8k32 s8, coarse keys as
+// the M operand loaded straight into fragments, 64 blocks per warp step; a
+// CUDA-core dp4a version measured ALU-bound at the 1M-token decode shape),
+// keeps the chunk's local Top-(K-1)
 // (warp-level bitonic Top-64 on unique 64-bit keys, then a merge tree over
 // the warps) and writes it to the workspace.  The last CTA of the query --
 // elected with an atomic counter, nothing waits -- merges the chunks' sorted
@@ -29,24 +31,27 @@ constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kCuqCache = 1024;   // cu_q entries staged in shared memory
 }  // namespace
 
-template <int E>
+template <int G>   // 64-block groups per warp: a chunk is kSelWarps * 64 * G blocks
 __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a) {
     __shared__ int4 s_q[kMaxIdxHeads][kIdxDim / 16];
     __shared__ int s_w[kMaxIdxHeads];
     __shared__ int s_cuq[kCuqCache + 1];
     __shared__ key64 s_lists[kSelWarps * 64];
     __shared__ int s_last;
-    constexpr int CH = kSelThreads * E;
+    constexpr int CH = kSelWarps * 64 * G;
     const int t = blockIdx.x, c = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, cq = lane & 3;
     const int H = a.num_idx_heads;
 
+    pdl_trigger();
     // ---- query facts: the sequence from a shared-memory copy of cu_q
     const bool cached = a.num_seqs + 1 <= kCuqCache;
     if (cached)
         for (int i = tid; i <= a.num_seqs; i += kSelThreads) s_cuq[i] = __ldg(a.cu_q + i);
-    for (int e = tid; e < H * 4; e += kSelThreads)
-        s_q[e >> 2][e & 3] = __ldg(reinterpret_cast<const int4 *>(a.q_idx + (size_t)t * H * kIdxDim) + e);
-    if (tid < H) s_w[tid] = __ldg(a.w + (size_t)t * H + tid);
+    for (int e = tid; e < kMaxIdxHeads * 4; e += kSelThreads)   // heads past H read as zero
+        s_q[e >> 2][e & 3] = (e >> 2) < H
+            ? __ldg(reinterpret_cast<const int4 *>(a.q_idx + (size_t)t * H * kIdxDim) + e) : make_int4(0, 0, 0, 0);
+    if (tid < kMaxIdxHeads) s_w[tid] = tid < H ? __ldg(a.w + (size_t)t * H + tid) : 0;
     __syncthreads();
     int s;
     if (cached) {
@@ -67,6 +72,7 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     const bool bad_pos = p < 0 || p >= len || n_vis > a.max_blocks;
     const bool bad_k = K < 1 || K > a.k_max;
     if (bad_pos || bad_k) {
+        pdl_wait();
         if (c == 0) {
             if (tid == 0) {
                 set_err(a.dev_err, bad_k ? DSA_DEV_ERR_K : DSA_DEV_ERR_POS);
@@ -79,6 +85,7 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     const int own = n_vis - 1;
     const int kk = K - 1;
     if (n_vis <= K || kk == 0) {   // every visible block, or only the own block
+        pdl_wait();
         if (c == 0) {
             const int n = n_vis <= K ? n_vis : 1;
             for (int i = tid; i < a.k_max; i += kSelThreads) out[i] = i < n ? (n == 1 ? own : i) : -1;
@@ -89,36 +96,65 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     const int n_chunks = (own + CH - 1) / CH;   // candidates: blocks 0 .. own-1
     if (c >= n_chunks) return;
 
-    // ---- score this chunk: E consecutive blocks per thread
-    key64 key[E];
-    uint32_t err_bits = 0;
-    const int b0 = c * CH + tid * E;
+    // ---- score this chunk on the int8 tensor cores, 64 blocks per warp step
+    int qb[2][2][2], wl[2][2];
+    {
+        const int *qi = reinterpret_cast<const int *>(s_q);
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-        const int b = b0 + e;
-        key[e] = 0;
-        if (b < own) {
-            const int page = __ldg(a.block_table + (size_t)s * a.max_blocks + b);
-            if (page >= 0 && page < a.num_pages) {
-                int kc[16];
-                load_coarse_key(a.kc_pool, page, kc);
-                key[e] = make_key64(block_score(kc, s_q, s_w, H), (uint32_t)b);
-            } else {
-                err_bits |= DSA_DEV_ERR_PAGE;
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int ks = 0; ks < 2; ++ks) {
+                qb[nt][ks][0] = qi[(8 * nt + g) * 16 + 8 * ks + cq];
+                qb[nt][ks][1] = qi[(8 * nt + g) * 16 + 8 * ks + 4 + cq];
             }
+            wl[nt][0] = s_w[8 * nt + 2 * cq];
+            wl[nt][1] = s_w[8 * nt + 2 * cq + 1];
         }
+    }
+    const int32_t *table = a.block_table + (size_t)s * a.max_blocks;
+    key64 acc[2] = {0ull, 0ull};
+    uint32_t err_bits = 0;
+#pragma unroll 1
+    for (int gi = 0; gi < G; ++gi) {
+        const int base = c * CH + (warp * G + gi) * 64;
+        key64 v[2] = {0ull, 0ull};
+        if (base < own) {
+            // all of the group's page ids, then all of its coarse-key fragments,
+            // in flight before the first tensor-core op
+            int pg[4][2];
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int b = base + 16 * mt + g + 8 * h;
+                    int page = b < own ? __ldg(table + b) : -1;
+                    if (b < own && (page < 0 || page >= a.num_pages)) { err_bits |= DSA_DEV_ERR_PAGE; page = -1; }
+                    pg[mt][h] = page;
+                }
+            if (gi == 0) pdl_wait();   // coarse keys may come from the preceding append
+            Tile16 f[4];
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt) tile16_load(a.kc_pool, pg[mt][0], pg[mt][1], f[mt]);
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt) {
+                int s_g, s_g8;
+                tile16_scores(f[mt], qb, wl, s_g, s_g8);
+                if (mt == cq) {   // lane (g, cq) keeps blocks 16*cq + g and 16*cq + g + 8
+                    const int b = base + 16 * mt + g;
+                    v[0] = pg[mt][0] >= 0 ? make_key64(s_g, (uint32_t)b) : 0ull;
+                    v[1] = pg[mt][1] >= 0 ? make_key64(s_g8, (uint32_t)(b + 8)) : 0ull;
+                }
+            }
+        } else if (gi == 0) {
+            pdl_wait();
+        }
+        warp_sort64_desc(v);
+        if (gi == 0) { acc[0] = v[0]; acc[1] = v[1]; }
+        else warp_merge64_desc(acc, v);
     }
     if (err_bits) set_err(a.dev_err, err_bits);
 
-    // ---- chunk Top-64: per warp, then a merge tree over the warps
-    key64 acc[2];
-#pragma unroll
-    for (int g = 0; g < (E + 1) / 2; ++g) {
-        key64 v[2] = {key[2 * g], 2 * g + 1 < E ? key[2 * g + 1] : 0ull};
-        warp_sort64_desc(v);
-        if (g == 0) { acc[0] = v[0]; acc[1] = v[1]; }
-        else warp_merge64_desc(acc, v);
-    }
+    // ---- chunk Top-64 over the warps, kept sorted in the workspace
     cta_merge_top64<kSelWarps>(acc, s_lists);
     key64 *cand = a.cand + ((size_t)t * kSelMaxChunks + c) * (kSelMaxK - 1);
     if (warp == 0) {
@@ -136,13 +172,21 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    acc[0] = acc[1] = 0ull;
-    for (int ci = warp; ci < n_chunks; ci += kSelWarps) {
+    constexpr int kPer = (kSelMaxChunks + kSelWarps - 1) / kSelWarps;   // lists per warp
+    key64 lists[kPer][2];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {   // every load in flight before the first merge
+        const int ci = warp + k * kSelWarps;
         const key64 *src = a.cand + ((size_t)t * kSelMaxChunks + ci) * (kSelMaxK - 1);
-        const key64 b[2] = {lane < kk ? __ldcg(src + lane) : 0ull, 32 + lane < kk ? __ldcg(src + 32 + lane) : 0ull};
-        if (ci == warp) { acc[0] = b[0]; acc[1] = b[1]; }
-        else warp_merge64_desc(acc, b);
+        const bool in = ci < n_chunks;
+        lists[k][0] = in && lane < kk ? __ldcg(src + lane) : 0ull;
+        lists[k][1] = in && 32 + lane < kk ? __ldcg(src + 32 + lane) : 0ull;
     }
+    acc[0] = lists[0][0];
+    acc[1] = lists[0][1];
+#pragma unroll
+    for (int k = 1; k < kPer; ++k)
+        if (warp + k * kSelWarps < n_chunks) warp_merge64_desc(acc, lists[k]);
     cta_merge_top64<kSelWarps>(acc, s_lists);
     if (warp == 0) {
         // the winners (non-zero keys among the first kk) in ascending block order
@@ -165,18 +209,16 @@ cudaError_t launch_select_blocks(const SelectArgs &a, cudaStream_t stream) {
     if (a.total_q == 0) return cudaSuccess;
     // the chunk size keeps every query at <= kSelMaxChunks chunks
     const int need = (a.max_blocks + kSelMaxChunks - 1) / kSelMaxChunks;   // blocks per chunk
-    const int e = (need + kSelThreads - 1) / kSelThreads;
-    auto go = [&](auto kern, int E) {
-        const int chunks = (a.max_blocks + kSelThreads * E - 1) / (kSelThreads * E);
-        kern<<<dim3(a.total_q, chunks), kSelThreads, 0, stream>>>(a);
+    const int gr = (need + kSelWarps * 64 - 1) / (kSelWarps * 64);
+    auto go = [&](auto kern, int G) {
+        const int chunks = (a.max_blocks + kSelWarps * 64 * G - 1) / (kSelWarps * 64 * G);
+        return launch_pdl(kern, dim3(a.total_q, chunks), dim3(kSelThreads), 0, stream, a);
     };
-    if (e <= 1) go(select_blocks_kernel<1>, 1);
-    else if (e <= 2) go(select_blocks_kernel<2>, 2);
-    else if (e <= 4) go(select_blocks_kernel<4>, 4);
-    else if (e <= 8) go(select_blocks_kernel<8>, 8);
-    else if (e <= 16) go(select_blocks_kernel<16>, 16);
-    else return cudaErrorInvalidValue;   // the host rejects contexts this long first
-    return cudaGetLastError();
+    if (gr <= 1) return go(select_blocks_kernel<1>, 1);
+    if (gr <= 2) return go(select_blocks_kernel<2>, 2);
+    if (gr <= 4) return go(select_blocks_kernel<4>, 4);
+    if (gr <= 8) return go(select_blocks_kernel<8>, 8);
+    return cudaErrorInvalidValue;   // the host rejects contexts this long first
 }
 
 }  // namespace dsa

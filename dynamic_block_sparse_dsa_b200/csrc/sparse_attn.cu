@@ -15,7 +15,8 @@
 // the batch looks like.  Inside the CTA:
 //   * a producer warp walks the range and, for each selected block, issues four
 //     boxes of a 3-D TMA tensor map over the pool (K and V, two 128-byte halves
-//     each, SWIZZLE_128B, no multicast) into a 5-stage shared-memory ring
+//     each, SWIZZLE_128B, no multicast) into a 6-stage (5 for 16-head groups)
+//     shared-memory ring
 //     guarded by full/empty mbarriers; it also TMA-loads the 16-row query tile
 //     of each (query, KV head) pair into a 2-slot ring;
 //   * four consumer warps take whole blocks round-robin.  Each runs the GQA
@@ -37,43 +38,56 @@ namespace dsa {
 namespace {
 constexpr int kConsumerWarps = 4;
 constexpr int kAttnThreads = (kConsumerWarps + 1) * 32;
-constexpr int kStages = 5;
 constexpr int kHalf = kBlockSize * 128;            // 8 KiB: 64 rows x 128 B (one swizzled half)
 constexpr int kStageBytes = 4 * kHalf;             // K lo, K hi, V lo, V hi
 constexpr int kQHalf = 16 * 128;                   // 16 query rows x 128 B
 constexpr int kQSlotBytes = 2 * kQHalf;
 constexpr int kSegSlots = 2;                       // query tile + pair facts, double buffered
 constexpr int kMergeStride = 132;                  // floats per merge row (padded against bank conflicts)
-constexpr int kMaxSmemSeqs = 2048;                 // cu_q entries cached in shared memory
-constexpr int kOffQ = kStages * kStageBytes;
-constexpr int kOffMergeO = kOffQ + kSegSlots * kQSlotBytes;
-constexpr int kOffMergeML = kOffMergeO + kConsumerWarps * 16 * kMergeStride * 4;
-constexpr int kOffCuq = kOffMergeML + kConsumerWarps * 16 * 2 * 4;
-constexpr int kOffBars = kOffCuq + (kMaxSmemSeqs + 1) * 4 + 4;
-constexpr int kNumBars = 2 * kStages + 2 * kSegSlots;
-constexpr int kOffWords = kOffBars + kNumBars * 8;
+constexpr int kMaxSmemSeqs = 256;                  // cu_q entries cached in shared memory
 // int words after the barriers
 constexpr int kWAbort = 0, kWLast = 1, kWNever = 2;
-constexpr int kWFill = 4;                           // [kStages] item index the stage was last armed for
-constexpr int kWItemBlk = kWFill + kStages;         // [kStages] logical block of that item
-constexpr int kWItemSeg = kWItemBlk + kStages;      // [kStages] segment of that item
-constexpr int kWSegEndCnt = kWItemSeg + kStages;    // [kSegSlots] items issued when the segment ended
+constexpr int kWFill = 4;                           // [kMaxStages] item index the stage was last armed for
+constexpr int kMaxStages = 8;
+constexpr int kWItemBlk = kWFill + kMaxStages;      // [kMaxStages] logical block of that item
+constexpr int kWItemSeg = kWItemBlk + kMaxStages;   // [kMaxStages] segment of that item
+constexpr int kWSegEndCnt = kWItemSeg + kMaxStages; // [kSegSlots] items issued when the segment ended
 constexpr int kWSegEndTag = kWSegEndCnt + kSegSlots;  // [kSegSlots] which segment that count belongs to
 constexpr int kWSegInfo = kWSegEndTag + kSegSlots;  // [kSegSlots][4]: t, kvh, p, n_vis
 constexpr int kNumWords = kWSegInfo + 4 * kSegSlots;
-constexpr int kSmemBytes = kOffWords + kNumWords * 4 + 1024;   // + slack to align the base to 1 KiB
 constexpr float kLn2 = 0.6931471805599453f;
-// most CTAs whose ranges can cover one pair (the host keeps K*C/U + 2 below it)
+// most CTAs whose ranges can cover one pair (the host caps the split at 60)
 constexpr int kMaxSplitSlots = 63;
 
+// shared-memory plan for NT head tiles: a group of <= 8 heads leaves room for
+// a sixth ring stage; 16-head groups need the larger merge buffer
+template <int NT>
+struct Plan {
+    static constexpr int kStages = NT == 1 ? 6 : 5;
+    static constexpr int kMergeRows = 8 * NT;
+    static constexpr int kOffQ = kStages * kStageBytes;
+    static constexpr int kOffMergeO = kOffQ + kSegSlots * kQSlotBytes;
+    static constexpr int kOffMergeML = kOffMergeO + kConsumerWarps * kMergeRows * kMergeStride * 4;
+    static constexpr int kOffCuq = kOffMergeML + kConsumerWarps * 16 * 2 * 4;
+    static constexpr int kOffRb = (kOffCuq + (kMaxSmemSeqs + 1) * 4 + 4 + 7) / 8 * 8;
+    static constexpr int kOffBars = kOffRb + (kAttnMaxCtas + 1) * 8;
+    static constexpr int kNumBars = 2 * kStages + 2 * kSegSlots;
+    static constexpr int kOffWords = kOffBars + kNumBars * 8;
+    static constexpr int kSmemBytes = kOffWords + kNumWords * 4 + 1024;   // + slack to align the base to 1 KiB
+    static_assert(kStages <= kMaxStages, "stage words");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+template <int NT>
 struct Smem {
+    using P = Plan<NT>;
     uint32_t base;   // 1 KiB aligned shared address
     __device__ uint32_t stage(int s) const { return base + s * kStageBytes; }
-    __device__ uint32_t qslot(int s) const { return base + kOffQ + s * kQSlotBytes; }
-    __device__ uint32_t full(int s) const { return base + kOffBars + 8 * s; }
-    __device__ uint32_t empty(int s) const { return base + kOffBars + 8 * (kStages + s); }
-    __device__ uint32_t qfull(int s) const { return base + kOffBars + 8 * (2 * kStages + s); }
-    __device__ uint32_t qempty(int s) const { return base + kOffBars + 8 * (2 * kStages + kSegSlots + s); }
+    __device__ uint32_t qslot(int s) const { return base + P::kOffQ + s * kQSlotBytes; }
+    __device__ uint32_t full(int s) const { return base + P::kOffBars + 8 * s; }
+    __device__ uint32_t empty(int s) const { return base + P::kOffBars + 8 * (P::kStages + s); }
+    __device__ uint32_t qfull(int s) const { return base + P::kOffBars + 8 * (2 * P::kStages + s); }
+    __device__ uint32_t qempty(int s) const { return base + P::kOffBars + 8 * (2 * P::kStages + kSegSlots + s); }
 };
 
 __device__ __forceinline__ long long range_begin(const AttnArgs &a, int c) {
@@ -100,17 +114,22 @@ template <int NT>   // query-head n-tiles of 8: the GQA group is <= 8 * NT
 __global__ void __launch_bounds__(kAttnThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ CUtensorMap tm_q, AttnArgs a) {
+    using P = Plan<NT>;
+    constexpr int kStages = P::kStages;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
-    Smem sm{(raw + 1023u) & ~1023u};
+    Smem<NT> sm{(raw + 1023u) & ~1023u};
     uint8_t *gbase = smem_raw + (sm.base - raw);   // generic pointer of the aligned base
-    volatile int *W = reinterpret_cast<volatile int *>(gbase + kOffWords);
+    volatile int *W = reinterpret_cast<volatile int *>(gbase + P::kOffWords);
     volatile int *s_abort = W + kWAbort;
     const volatile int *s_never = W + kWNever;      // stays 0: a wait that ignores the abort flag
-    int *s_cuq = reinterpret_cast<int *>(gbase + kOffCuq);
+    int *s_cuq = reinterpret_cast<int *>(gbase + P::kOffCuq);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
+    // every CTA's range start, once (64-bit divisions are slow; lookups are not)
+    long long *s_rb = reinterpret_cast<long long *>(gbase + P::kOffRb);
+    for (int i = tid; i <= a.num_ctas; i += kAttnThreads) s_rb[i] = range_begin(a, i);
     const long long u0 = range_begin(a, c), u1 = range_begin(a, c + 1);
     const int G = a.group;
     const long long K = a.k_max;
@@ -129,6 +148,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         for (int s = 0; s < kSegSlots; ++s) W[kWSegEndTag + s] = -1;
         fence_barrier_init();
     }
+    pdl_trigger();
     __syncthreads();
 
     if (warp == kConsumerWarps) {
@@ -146,6 +166,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             prefetch_tensormap(&tm_v);
             prefetch_tensormap(&tm_q);
         }
+        pdl_wait();   // the selection and the appended tokens come from the kernels before
         int item = 0, seg = 0;
         uint32_t err_bits = 0;
         bool stop = false;
@@ -268,9 +289,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     }
 
     // ==================================================================== consumer warps
+    pdl_wait();
     const int g = lane >> 2, cq = lane & 3;
-    float *s_mo = reinterpret_cast<float *>(gbase + kOffMergeO);    // [4][16][kMergeStride]
-    float *s_ml = reinterpret_cast<float *>(gbase + kOffMergeML);   // [4][16][2]
+    float *s_mo = reinterpret_cast<float *>(gbase + P::kOffMergeO);   // [4][kMergeRows][kMergeStride]
+    float *s_ml = reinterpret_cast<float *>(gbase + P::kOffMergeML);  // [4][16][2]
 
     long long u = u0;
     long long pair = u0 / K;
@@ -445,7 +467,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int h0 = 8 * nt + 2 * cq;
-            float *row0 = s_mo + (warp * 16 + h0) * kMergeStride;
+            float *row0 = s_mo + (warp * P::kMergeRows + h0) * kMergeStride;
             float *row1 = row0 + kMergeStride;
 #pragma unroll
             for (int dm = 0; dm < 8; ++dm) {
@@ -481,7 +503,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 for (int w = 0; w < kConsumerWarps; ++w) {
                     const float f = exp2f(s_ml[(w * 16 + r) * 2] - M);
                     L += s_ml[(w * 16 + r) * 2 + 1] * f;
-                    const float4 v = *reinterpret_cast<const float4 *>(s_mo + (w * 16 + r) * kMergeStride + d0);
+                    const float4 v = *reinterpret_cast<const float4 *>(s_mo + (w * P::kMergeRows + r) * kMergeStride + d0);
                     acc[0] += v.x * f; acc[1] += v.y * f; acc[2] += v.z * f; acc[3] += v.w * f;
                 }
             }
@@ -497,87 +519,68 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             }
         }
         if (!whole) {
-            __threadfence();
+            // publish the partial: the barrier orders every thread's stores
+            // before thread 0's release-add on the pair's counter; the CTA that
+            // completes the count acquires them all and merges.
             __syncwarp();
             named_barrier(1, kConsumerWarps * 32);
             if (tid == 0) {
                 const int covered = (int)(seg_end - seg_begin);
-                const int old = atomicAdd(a.counters + pair, covered);
+                const int old = atomic_add_acq_rel_gpu(a.counters + pair, covered);
                 W[kWLast] = (old + covered == a.k_max);
             }
             __syncwarp();
             named_barrier(1, kConsumerWarps * 32);
             if (W[kWLast]) {
-                __threadfence();
-                // the CTAs covering this pair are this CTA's neighbours: walk
-                // out from c while their ranges still overlap the pair.  The
-                // per-warp merge buffers are free now and hold the slot list,
-                // each partial's (m, l) and its merge weight.
-                int *s_slot = reinterpret_cast<int *>(s_ml);        // [1 + kMaxSplitSlots]
-                float *s_pml = s_mo;                                 // [kMaxSplitSlots][16][2]
-                float *s_w = s_mo + kMaxSplitSlots * 32;             // [kMaxSplitSlots][16] weights
-                float *s_inv = s_w + kMaxSplitSlots * 16;            // [16] 1/L
-                float *s_lse = s_inv + 16;                           // [16]
-                if (tid == 0) {
-                    const long long p_lo = pair * K, p_hi = p_lo + K;
-                    int cf = c, cl = c;
-                    while (cf > 0 && range_begin(a, cf) > p_lo) --cf;
-                    while (cl + 1 < a.num_ctas && range_begin(a, cl + 1) < p_hi) ++cl;
-                    int n = 0;
-                    for (int cc = cf; cc <= cl && n < kMaxSplitSlots; ++cc, ++n)
-                        s_slot[1 + n] = 2 * cc + (range_begin(a, cc) >= p_lo ? 0 : 1);
-                    s_slot[0] = n;
-                }
-                __syncwarp();
-                named_barrier(1, kConsumerWarps * 32);
-                const int n_slots = s_slot[0];
-                // (m, l) of every partial row, all loads in flight at once
-                for (int e = tid; e < n_slots * G; e += kConsumerWarps * 32) {
-                    const int k = e / G, r = e % G;
-                    const float *src = a.part + ((size_t)s_slot[1 + k] * G + r) * kAttnPartStride;
-                    const float2 ml = __ldcg(reinterpret_cast<const float2 *>(src + 128));
-                    s_pml[(k * 16 + r) * 2] = ml.x;
-                    s_pml[(k * 16 + r) * 2 + 1] = ml.y;
-                }
-                __syncwarp();
-                named_barrier(1, kConsumerWarps * 32);
-                if (tid < G) {
-                    const int r = tid;
-                    float M = -INFINITY;
-                    for (int k = 0; k < n_slots; ++k) M = fmaxf(M, s_pml[(k * 16 + r) * 2]);
-                    float L = 0.f;
-                    for (int k = 0; k < n_slots; ++k) {
-                        const float mk = s_pml[(k * 16 + r) * 2];
-                        const float f = (M == -INFINITY || mk == -INFINITY) ? 0.f : exp2f(mk - M);
-                        s_w[k * 16 + r] = f;
-                        L += s_pml[(k * 16 + r) * 2 + 1] * f;
-                    }
-                    s_inv[r] = L > 0.f ? 1.f / L : 0.f;
-                    s_lse[r] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
-                }
-                __syncwarp();
-                named_barrier(1, kConsumerWarps * 32);
+                // CTAs covering the pair: closed form from the split, then a
+                // fix-up step in case of rounding
+                // the pair's CTAs are this CTA's neighbours (ranges are contiguous)
+                const long long p_lo = pair * K, p_hi = p_lo + K;
+                int cf = c, cl = c;
+                while (cf > 0 && s_rb[cf] > p_lo) --cf;
+                while (cl + 1 < a.num_ctas && s_rb[cl + 1] < p_hi) ++cl;
+                const int n_slots = min(cl - cf + 1, kMaxSplitSlots);
+                // every partial of the row in flight at once, then combine
                 for (int e = tid; e < G * 32; e += kConsumerWarps * 32) {
                     const int r = e >> 5, d0 = (e & 31) * 4;
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    float M = -INFINITY, L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
                     for (int k0 = 0; k0 < n_slots; k0 += 4) {
-                        float4 v[4];
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            v[k] = (k0 + k < n_slots)
-                                       ? __ldcg(reinterpret_cast<const float4 *>(
-                                             a.part + ((size_t)s_slot[1 + k0 + k] * G + r) * kAttnPartStride + d0))
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                        float2 ml[4];
+                        float4 ov[4];
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            const float f = (k0 + k < n_slots) ? s_w[(k0 + k) * 16 + r] : 0.f;
-                            acc[0] += v[k].x * f; acc[1] += v[k].y * f; acc[2] += v[k].z * f; acc[3] += v[k].w * f;
+                            const int cc = cf + k0 + k;
+                            if (k0 + k < n_slots) {
+                                const int sl = 2 * cc + (s_rb[cc] >= p_lo ? 0 : 1);
+                                const float *src = a.part + ((size_t)sl * G + r) * kAttnPartStride;
+                                ml[k] = __ldcg(reinterpret_cast<const float2 *>(src + 128));
+                                ov[k] = __ldcg(reinterpret_cast<const float4 *>(src + d0));
+                            } else {
+                                ml[k] = make_float2(-INFINITY, 0.f);
+                                ov[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            }
+                        }
+                        float Mn = M;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) Mn = fmaxf(Mn, ml[k].x);
+                        if (Mn != -INFINITY) {
+                            const float fo = M == -INFINITY ? 0.f : exp2f(M - Mn);   // rescale what we have
+                            L *= fo;
+                            acc[0] *= fo; acc[1] *= fo; acc[2] *= fo; acc[3] *= fo;
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const float f = ml[k].x == -INFINITY ? 0.f : exp2f(ml[k].x - Mn);
+                                L += ml[k].y * f;
+                                acc[0] += ov[k].x * f; acc[1] += ov[k].y * f;
+                                acc[2] += ov[k].z * f; acc[3] += ov[k].w * f;
+                            }
+                            M = Mn;
                         }
                     }
-                    const float inv = s_inv[r];
+                    const float inv = L > 0.f ? 1.f / L : 0.f;
                     *reinterpret_cast<uint2 *>(a.out + (out_row + r) * kHeadDim + d0) = make_uint2(
                         pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
-                    if (a.lse && d0 == 0) a.lse[out_row + r] = s_lse[r];
+                    if (a.lse && d0 == 0) a.lse[out_row + r] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
                 }
                 if (tid == 0) a.counters[pair] = 0;
             }
@@ -644,17 +647,19 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !(attr_done & (1ull << dev))) {
-        e = cudaFuncSetAttribute(sparse_attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        e = cudaFuncSetAttribute(sparse_attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Plan<1>::kSmemBytes);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(sparse_attn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+            e = cudaFuncSetAttribute(sparse_attn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Plan<2>::kSmemBytes);
         if (e != cudaSuccess) return e;
         if (dev < 64) attr_done |= 1ull << dev;
     }
     if (a.group <= 8)
-        sparse_attn_kernel<1><<<a.num_ctas, kAttnThreads, kSmemBytes, stream>>>(tk, tv, tq, a);
-    else
-        sparse_attn_kernel<2><<<a.num_ctas, kAttnThreads, kSmemBytes, stream>>>(tk, tv, tq, a);
-    return cudaGetLastError();
+        return launch_pdl(sparse_attn_kernel<1>, dim3(a.num_ctas), dim3(kAttnThreads), Plan<1>::kSmemBytes, stream,
+                          tk, tv, tq, a);
+    return launch_pdl(sparse_attn_kernel<2>, dim3(a.num_ctas), dim3(kAttnThreads), Plan<2>::kSmemBytes, stream, tk,
+                      tv, tq, a);
 }
 
 }  // namespace dsa

@@ -24,6 +24,8 @@ constexpr int kTopkWarps = kTopkThreads / 32;
 
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     __shared__ key64 s_lists[kTopkWarps * 64];
+    pdl_trigger();
+    pdl_wait();   // the scores come from the preceding kernel
     const int t = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int32_t *out = a.sel + (size_t)t * a.k_max;
     const int s = find_seq(a.cu_q, a.num_seqs, t);
@@ -79,8 +81,7 @@ int topk_max_blocks() { return 1 << 20; }
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream) {
     if (a.total_q == 0) return cudaSuccess;
     if (a.k_max > 64) return cudaErrorInvalidValue;   // the host rejects these first
-    topk_kernel<<<a.total_q, kTopkThreads, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(topk_kernel, dim3(a.total_q), dim3(kTopkThreads), 0, stream, a);
 }
 
 }  // namespace dsa
