@@ -49,11 +49,18 @@ def init_dist(world: int, backend: str):
         torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
 
 
+def _reduce_device(device):
+    # gloo reduces host tensors, nccl device tensors
+    if torch.distributed.get_backend() == "gloo":
+        return torch.device("cpu")
+    return device
+
+
 def max_over_ranks(x: float, world: int, device) -> float:
     """Max of a per-rank float over all ranks (identity when world == 1)."""
     if world == 1:
         return float(x)
-    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=_reduce_device(device))
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -61,9 +68,15 @@ def max_over_ranks(x: float, world: int, device) -> float:
 def sum_over_ranks(x: float, world: int, device) -> float:
     if world == 1:
         return float(x)
-    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=_reduce_device(device))
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
     return float(t.item())
+
+
+def weak_scaling_throughput(units_per_step_per_rank: int, steps: int, world: int, seconds_max: float) -> float:
+    """Whole-job throughput: every rank processes its own batch each step, and
+    the job takes as long as its slowest rank."""
+    return units_per_step_per_rank * steps * world / seconds_max
 
 
 def barrier(world: int):
@@ -244,7 +257,7 @@ def run_ours(args, world, rank, device):
     total_s = sum(step_ms) / 1e3
     total_s_max = max_over_ranks(total_s, world, device)
     tokens_per_step = spec.total_q
-    value = tokens_per_step * args.steps * world / total_s_max
+    value = weak_scaling_throughput(tokens_per_step, args.steps, world, total_s_max)
     ab = algorithmic_bytes(wl)
     attn_mean_s = sum(attn_ms) / len(attn_ms) / 1e3
     step_mean_s = total_s / args.steps
@@ -285,7 +298,7 @@ def run_ours(args, world, rank, device):
         if i >= 2:
             e2e_ms.append(e_s.elapsed_time(e_e))
     e2e_total = max_over_ranks(sum(e2e_ms) / 1e3, world, device)
-    e2e = {"value": round(tokens_per_step * len(e2e_ms) * world / e2e_total, 1), "unit": UNIT,
+    e2e = {"value": round(weak_scaling_throughput(tokens_per_step, len(e2e_ms), world, e2e_total), 1), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     res = {
@@ -366,14 +379,14 @@ def main(argv=None):
     world, rank, local = dist_env()
     if world != args.gpus and world > 1:
         print(f"warning: WORLD_SIZE={world} but --gpus={args.gpus}", file=sys.stderr)
+    if args.impl == "reference" and rank != 0:
+        return 0   # the oracle arm runs on rank 0 alone
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
 
     if args.impl == "reference":
-        if rank != 0:
-            return 0
         print(json.dumps(run_reference(args, world, rank, device)), flush=True)
         return 0
 

@@ -540,47 +540,69 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 while (cf > 0 && s_rb[cf] > p_lo) --cf;
                 while (cl + 1 < a.num_ctas && s_rb[cl + 1] < p_hi) ++cl;
                 const int n_slots = min(cl - cf + 1, kMaxSplitSlots);
-                // every partial of the row in flight at once, then combine
-                for (int e = tid; e < G * 32; e += kConsumerWarps * 32) {
-                    const int r = e >> 5, d0 = (e & 31) * 4;
-                    float M = -INFINITY, L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-                    for (int k0 = 0; k0 < n_slots; k0 += 4) {
-                        float2 ml[4];
-                        float4 ov[4];
+                // each thread owns kRowsPT (row, 4-column) pieces; the loads of
+                // all of them and of a batch of slots are issued before any is
+                // used, so the merge costs one L2 round trip per batch
+                constexpr int kRowsPT = 2 * NT;                 // 8 * NT rows * 32 pieces / 128 threads
+                constexpr int kBatch = NT == 1 ? 4 : 2;         // slots per round trip
+                float M[kRowsPT], L[kRowsPT], acc[kRowsPT][4];
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
+                for (int i = 0; i < kRowsPT; ++i) {
+                    M[i] = -INFINITY;
+                    L[i] = 0.f;
+                    acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+                }
+                for (int k0 = 0; k0 < n_slots; k0 += kBatch) {
+                    float2 ml[kRowsPT][kBatch];
+                    float4 ov[kRowsPT][kBatch];
+#pragma unroll
+                    for (int i = 0; i < kRowsPT; ++i) {
+                        const int e = tid + i * kConsumerWarps * 32;
+                        const int r = e >> 5, d0 = (e & 31) * 4;
+#pragma unroll
+                        for (int k = 0; k < kBatch; ++k) {
                             const int cc = cf + k0 + k;
-                            if (k0 + k < n_slots) {
+                            if (e < G * 32 && k0 + k < n_slots) {
                                 const int sl = 2 * cc + (s_rb[cc] >= p_lo ? 0 : 1);
                                 const float *src = a.part + ((size_t)sl * G + r) * kAttnPartStride;
-                                ml[k] = __ldcg(reinterpret_cast<const float2 *>(src + 128));
-                                ov[k] = __ldcg(reinterpret_cast<const float4 *>(src + d0));
+                                ml[i][k] = __ldcg(reinterpret_cast<const float2 *>(src + 128));
+                                ov[i][k] = __ldcg(reinterpret_cast<const float4 *>(src + d0));
                             } else {
-                                ml[k] = make_float2(-INFINITY, 0.f);
-                                ov[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                                ml[i][k] = make_float2(-INFINITY, 0.f);
+                                ov[i][k] = make_float4(0.f, 0.f, 0.f, 0.f);
                             }
-                        }
-                        float Mn = M;
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) Mn = fmaxf(Mn, ml[k].x);
-                        if (Mn != -INFINITY) {
-                            const float fo = M == -INFINITY ? 0.f : exp2f(M - Mn);   // rescale what we have
-                            L *= fo;
-                            acc[0] *= fo; acc[1] *= fo; acc[2] *= fo; acc[3] *= fo;
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const float f = ml[k].x == -INFINITY ? 0.f : exp2f(ml[k].x - Mn);
-                                L += ml[k].y * f;
-                                acc[0] += ov[k].x * f; acc[1] += ov[k].y * f;
-                                acc[2] += ov[k].z * f; acc[3] += ov[k].w * f;
-                            }
-                            M = Mn;
                         }
                     }
-                    const float inv = L > 0.f ? 1.f / L : 0.f;
-                    *reinterpret_cast<uint2 *>(a.out + (out_row + r) * kHeadDim + d0) = make_uint2(
-                        pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
-                    if (a.lse && d0 == 0) a.lse[out_row + r] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+#pragma unroll
+                    for (int i = 0; i < kRowsPT; ++i) {
+                        float Mn = M[i];
+#pragma unroll
+                        for (int k = 0; k < kBatch; ++k) Mn = fmaxf(Mn, ml[i][k].x);
+                        if (Mn != -INFINITY) {
+                            const float fo = M[i] == -INFINITY ? 0.f : exp2f(M[i] - Mn);   // rescale what we have
+                            L[i] *= fo;
+                            acc[i][0] *= fo; acc[i][1] *= fo; acc[i][2] *= fo; acc[i][3] *= fo;
+#pragma unroll
+                            for (int k = 0; k < kBatch; ++k) {
+                                const float f = ml[i][k].x == -INFINITY ? 0.f : exp2f(ml[i][k].x - Mn);
+                                L[i] += ml[i][k].y * f;
+                                acc[i][0] += ov[i][k].x * f; acc[i][1] += ov[i][k].y * f;
+                                acc[i][2] += ov[i][k].z * f; acc[i][3] += ov[i][k].w * f;
+                            }
+                            M[i] = Mn;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < kRowsPT; ++i) {
+                    const int e = tid + i * kConsumerWarps * 32;
+                    if (e >= G * 32) break;
+                    const int r = e >> 5, d0 = (e & 31) * 4;
+                    const float inv = L[i] > 0.f ? 1.f / L[i] : 0.f;
+                    *reinterpret_cast<uint2 *>(a.out + (out_row + r) * kHeadDim + d0) =
+                        make_uint2(pack_bf16x2(acc[i][0] * inv, acc[i][1] * inv),
+                                   pack_bf16x2(acc[i][2] * inv, acc[i][3] * inv));
+                    if (a.lse && d0 == 0) a.lse[out_row + r] = L[i] > 0.f ? (M[i] + log2f(L[i])) * kLn2 : -INFINITY;
                 }
                 if (tid == 0) a.counters[pair] = 0;
             }

@@ -128,9 +128,9 @@ int dsa_kv_append(const dsa_kv_cache *cache, const dsa_seqs *seqs, const int32_t
  *   scores int32 [total_q][max_blocks]: entries b <= q_pos[t]/block_size are
  *          written, the rest of the row is left untouched.
  * DSA_ERR_RANGE when num_idx_heads * w_abs_max * idx_dim * 128 * 128 >= 2^31
- * (an int32 result could overflow).  Sequences with at least 16 queries take
- * the tensor-core (tcgen05 int8) path, the others the CUDA-core path; both
- * give the same integers.  Device errors: DSA_DEV_ERR_PAGE, DSA_DEV_ERR_POS.
+ * (an int32 result could overflow).  One CTA scores 256 blocks of one
+ * sequence for all of its queries with dp4a on the CUDA cores.
+ * Device errors: DSA_DEV_ERR_PAGE, DSA_DEV_ERR_POS.
  */
 int dsa_index_score(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
                     const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads,
@@ -188,9 +188,10 @@ int dsa_select_blocks(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa
  * Both entries run one persistent CTA per SM over the list of (query, KV
  * head, selected block) units, split evenly.  The decode entry may split a
  * (query, KV head) pair across CTAs and merge the partial softmax states; it
- * needs a workspace of dsa_sparse_attn_decode_workspace_size() bytes (32
- * bytes per (query, KV head) plus a fixed part), zero-filled before its first
- * use (each call leaves it zeroed again).  The prefill entry keeps every pair
+ * needs a workspace of dsa_sparse_attn_decode_workspace_size() bytes (a
+ * 4-byte counter per (query, KV head) pair plus room for two partial states
+ * per CTA), zero-filled before its first use (each call leaves it zeroed
+ * again).  The prefill entry keeps every pair
  * inside one CTA and needs no workspace.
  * Device errors: DSA_DEV_ERR_SEL, DSA_DEV_ERR_PAGE (that block is skipped).
  */
