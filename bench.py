@@ -33,6 +33,10 @@ if ROOT not in sys.path:
 METRIC = "sparse-attn decode tokens/s @1M ctx; achieved HBM GB/s vs ~8 TB/s peak"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 512 << 20
+# DRAM bytes (read + write) per launch of the roofline kernel, from an ncu
+# capture of the current kernel ((workload, path) -> bytes); absent = not
+# captured since the kernel last changed
+TRAFFIC = {}
 
 
 # ----------------------------------------------------------------------------- distributed plumbing
@@ -177,7 +181,13 @@ def run_ours(args, world, rank, device):
     seqs = dsa.SeqBatch(wl.block_table, wl.seq_lens)
     queries = dsa.QueryBatch(wl.cu_q, wl.q_pos)
     decode = all(n == 1 for n in spec.n_new)
-    fused = decode and spec.k_max <= 64   # score + Top-K in one pass for decode batches
+    path = args.path
+    if path == "auto":   # decode batches: the fused select chain; otherwise the separate calls
+        path = "fused_select" if decode and spec.k_max <= 64 else "score_topk"
+    if path == "fused_decode" and not decode:
+        raise SystemExit("--path fused_decode needs a decode workload")
+    fused = path in ("fused_select", "fused_decode")
+    fused_decode = path == "fused_decode"
     err = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.Stream(device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
@@ -201,10 +211,15 @@ def run_ours(args, world, rank, device):
             dsa.sparse_attn_prefill(cache, seqs, queries, wl.q, b["sel"], b["cnt"], out=b["out"], lse=b["lse"],
                                     dev_err=err)
 
+    def whole_step(b):
+        dsa.decode_fused(cache, seqs, queries, queries.cu_q, wl.k_new, wl.v_new, wl.kc_new, wl.q_idx, wl.w,
+                         wl.k_per_seq, spec.k_max, wl.q, sel=b["sel"], cnt=b["cnt"], out=b["out"], lse=b["lse"],
+                         workspace=b["fused_ws"], dev_err=err)
+
     with torch.cuda.stream(stream):
         bufs = dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
                         q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=spec.k_max, decode=decode,
-                        fused_select=fused, dev_err=err)
+                        fused_select=fused, fused_decode=fused_decode, dev_err=err)
     torch.cuda.synchronize(device)
     if int(err.item()) != 0:
         raise RuntimeError(f"device error bits {int(err.item())} in the first step")
@@ -216,8 +231,11 @@ def run_ours(args, world, rank, device):
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         ev[0].record()
-        front(bufs)
-        attn(bufs)
+        if fused_decode:
+            whole_step(bufs)
+        else:
+            front(bufs)
+            attn(bufs)
         ev[1].record()
     graph_attn = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph_attn, stream=stream):
@@ -262,11 +280,19 @@ def run_ours(args, world, rank, device):
     attn_mean_s = sum(attn_ms) / len(attn_ms) / 1e3
     step_mean_s = total_s / args.steps
     peak, peak_kind = _peaks()
-    achieved = ab["kv"] / attn_mean_s / 1e9
-    roofline = {"bound": "hbm", "kernel": "sparse_attn_kernel (decode entry; timed alone, cold L2)",
-                "achieved": round(achieved, 1),
-                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": peak_kind,
-                "bytes_per_launch": ab["kv"], "traffic": None}
+    if fused_decode:
+        # the step is one kernel: its bytes are the coarse keys plus the selected K/V
+        achieved = ab["total"] / step_mean_s / 1e9
+        roofline = {"bound": "hbm", "kernel": "sparse_attn_kernel<1,true> (single-launch decode step, cold L2)",
+                    "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                    "peak_source": peak_kind, "bytes_per_launch": ab["total"],
+                    "traffic": TRAFFIC.get((spec.name, "fused_decode"))}
+    else:
+        achieved = ab["kv"] / attn_mean_s / 1e9
+        roofline = {"bound": "hbm", "kernel": "sparse_attn_kernel (decode entry; timed alone, cold L2)",
+                    "achieved": round(achieved, 1),
+                    "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": peak_kind,
+                    "bytes_per_launch": ab["kv"], "traffic": TRAFFIC.get((spec.name, "attention"))}
     step_gbs = ab["total"] / step_mean_s / 1e9
     step_roof = {"bytes_per_step": ab["total"], "achieved_gbs": round(step_gbs, 1),
                  "frac_of_measured": round(step_gbs / peak, 4), "frac_of_8tbs": round(step_gbs / 8000.0, 4)}
@@ -290,7 +316,7 @@ def run_ours(args, world, rank, device):
                 dev_in[k].copy_(t, non_blocking=True)
             dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
                      q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=spec.k_max, decode=decode,
-                     fused_select=fused, bufs=bufs, dev_err=err)
+                     fused_select=fused, fused_decode=fused_decode, bufs=bufs, dev_err=err)
             host_out.copy_(bufs["out"], non_blocking=True)
             host_lse.copy_(bufs["lse"], non_blocking=True)
             e_e.record()
@@ -311,14 +337,16 @@ def run_ours(args, world, rank, device):
                    "heads_q_kv_idx": [spec.num_q_heads, spec.num_kv_heads, spec.num_idx_heads],
                    "global_batch": spec.num_seqs * world, "parallelism": f"dp{world} (independent sequences)",
                    "l2": "cold before every timed step: 512 MiB written, then 256 MiB read (no dirty lines)",
-                   "graph": "one CUDA graph per step (PDL between kernels)",
-                   "select": "fused score+top-k" if fused else "index_score then topk_blocks"},
+                   "graph": "one CUDA graph per step" + ("" if fused_decode else " (PDL between kernels)"),
+                   "path": {"fused_decode": "single launch: append + fused score/Top-K + attention",
+                            "fused_select": "kv_append, fused score+Top-K, attention",
+                            "score_topk": "kv_append, index_score, topk_blocks, attention"}[path]},
         "roofline": roofline,
         "step_roofline": step_roof,
         "attn_ms_mean": round(attn_mean_s * 1e3, 5),
         "step_ms_median": round(statistics.median(step_ms), 5),
         "e2e": e2e,
-        "gpu_launches": (3 if fused else 4) * args.steps,
+        "gpu_launches": (1 if fused_decode else 3 if fused else 4) * args.steps,
         "clocks": clk.summary(),
     }
     return res, wl
@@ -372,6 +400,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="decode_1m")
     ap.add_argument("--seed", type=int, default=1003)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", choices=["auto", "fused_decode", "fused_select", "score_topk"], default="auto",
+                    help="decode step as one launch, or as the chain of separate calls")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -254,11 +254,54 @@ def sparse_attn_prefill(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch
     return out, lse
 
 
+def decode_fused_workspace_size(total_q: int, num_q_heads: int, num_kv_heads: int, k_max: int) -> int:
+    return int(load().dsa_decode_fused_workspace_size(total_q, num_q_heads, num_kv_heads, k_max))
+
+
+def decode_fused(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, cu_new: Optional[torch.Tensor],
+                 k_new: Optional[torch.Tensor], v_new: Optional[torch.Tensor], kc_new: Optional[torch.Tensor],
+                 q_idx: torch.Tensor, w: torch.Tensor, k_per_seq: torch.Tensor, k_max: int, q: torch.Tensor,
+                 w_abs_max: int = 16, sm_scale: Optional[float] = None, sel=None, cnt=None, out=None, lse=None,
+                 workspace: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None, stream=None):
+    """One decode step in a single launch (append, select, attention):
+    (sel, cnt, out, lse).  ``cu_new``/``k_new``/``v_new``/``kc_new`` describe
+    the tokens to append (``k_new`` None: nothing appended).  ``workspace`` is
+    a zero-initialised uint8 tensor of decode_fused_workspace_size() bytes
+    (allocated here if None); one workspace serves every later call."""
+    lib = load()
+    _expect(q, torch.bfloat16, "q")
+    _expect(q_idx, torch.int8, "q_idx")
+    _expect(w, torch.int32, "w")
+    T, dev = queries.total_q, q.device
+    if sel is None:
+        sel = torch.empty((T, k_max), dtype=torch.int32, device=dev)
+    if cnt is None:
+        cnt = torch.empty((T,), dtype=torch.int32, device=dev)
+    out, lse = _attn_out(q, out, lse)
+    if workspace is None:
+        workspace = torch.zeros(decode_fused_workspace_size(T, q.shape[1], cache.num_kv_heads, k_max),
+                                dtype=torch.uint8, device=dev)
+    total_new = 0 if k_new is None else k_new.shape[0]
+    if k_new is not None:
+        _expect(k_new, torch.bfloat16, "k_new")
+        _expect(v_new, torch.bfloat16, "v_new")
+    scale = 1.0 / math.sqrt(q.shape[2]) if sm_scale is None else float(sm_scale)
+    c, s, qq = cache.ctype(), seqs.ctype(), queries.ctype()
+    _lib.check("dsa_decode_fused", lib.dsa_decode_fused(
+        ctypes.byref(c), ctypes.byref(s), ctypes.byref(qq), _ptr(cu_new), int(total_new), _ptr(k_new), _ptr(v_new),
+        _ptr(kc_new), _ptr(q_idx), _ptr(w), q_idx.shape[1], int(w_abs_max), _ptr(k_per_seq), int(k_max), _ptr(q),
+        q.shape[1], scale, _ptr(sel), _ptr(cnt), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _ptr(dev_err), _stream(stream)))
+    return sel, cnt, out, lse
+
+
 def step(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, *, k_new, v_new, kc_new, q, q_idx, w,
          k_per_seq, k_max: int, w_abs_max: int = 16, decode: bool = True, fused_select: bool = False,
-         bufs: Optional[dict] = None, dev_err: Optional[torch.Tensor] = None, stream=None):
+         fused_decode: bool = False, bufs: Optional[dict] = None, dev_err: Optional[torch.Tensor] = None,
+         stream=None):
     """One pass of the hot path: append -> index_score -> topk_blocks -> attention
-    (with ``fused_select`` the middle two are the single select_blocks call).
+    (with ``fused_select`` the middle two are the single select_blocks call;
+    with ``fused_decode`` the whole decode step is one decode_fused launch).
 
     ``bufs`` (optional, reused across calls) holds the scores / sel / cnt /
     out / lse / workspace tensors; missing ones are allocated.  Returns bufs.
@@ -274,6 +317,16 @@ def step(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, *, k_new, v_n
         b["workspace"] = torch.zeros(decode_workspace_size(T, q.shape[1], cache.num_kv_heads, k_max),
                                      dtype=torch.uint8, device=dev)
         b["select_ws"] = torch.zeros(select_workspace_size(T), dtype=torch.uint8, device=dev)
+    if fused_decode:
+        if not decode:
+            raise ValueError("fused_decode needs a decode batch")
+        if "fused_ws" not in b:
+            b["fused_ws"] = torch.zeros(decode_fused_workspace_size(T, q.shape[1], cache.num_kv_heads, k_max),
+                                        dtype=torch.uint8, device=dev)
+        decode_fused(cache, seqs, queries, queries.cu_q, k_new, v_new, kc_new, q_idx, w, k_per_seq, k_max, q,
+                     w_abs_max, sel=b["sel"], cnt=b["cnt"], out=b["out"], lse=b["lse"], workspace=b["fused_ws"],
+                     dev_err=dev_err, stream=stream)
+        return b
     kv_append(cache, seqs, queries.cu_q, k_new, v_new, kc_new, dev_err=dev_err, stream=stream)
     if fused_select:
         select_blocks(cache, seqs, queries, q_idx, w, k_per_seq, k_max, w_abs_max, sel=b["sel"], cnt=b["cnt"],

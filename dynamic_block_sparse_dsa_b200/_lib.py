@@ -53,6 +53,10 @@ SIGNATURES = {
                                  ctypes.c_float, c_vp, c_vp, c_vp, c_vp], c_i32),
     "dsa_sparse_attn_decode_noalloc": ([P(KvCacheC), P(SeqsC), P(QueriesC), c_vp, c_i32, c_vp, c_vp, c_i32,
                                         ctypes.c_float, c_vp, c_vp, c_vp, c_vp], c_i32),
+    "dsa_decode_fused_workspace_size": ([c_i32, c_i32, c_i32, c_i32], ctypes.c_size_t),
+    "dsa_decode_fused": ([P(KvCacheC), P(SeqsC), P(QueriesC), c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32,
+                          c_i32, c_vp, c_i32, c_vp, c_i32, ctypes.c_float, c_vp, c_vp, c_vp, c_vp, c_vp,
+                          ctypes.c_size_t, c_vp, c_vp], c_i32),
     "dsa_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "dsa_version": ([], ctypes.c_int),
 }

@@ -70,6 +70,23 @@ SelectLayout select_layout(int total_q) {
     return L;
 }
 
+// single-launch decode workspace: [header 256 B][sel_count T][flags T]
+// [split counters T*Hkv][candidates kAttnMaxCtas*2*(kSelMaxK-1) u64][partials]
+struct FusedLayout {
+    size_t hdr, sel_count, flags, counters, cand, part, total;
+};
+FusedLayout fused_layout(int total_q, int hq, int hkv) {
+    FusedLayout L;
+    L.hdr = 0;
+    L.sel_count = 256;
+    L.flags = align_up(L.sel_count + (size_t)total_q * 4, 256);
+    L.counters = align_up(L.flags + (size_t)total_q * 4, 256);
+    L.cand = align_up(L.counters + (size_t)total_q * hkv * 4, 256);
+    L.part = align_up(L.cand + (size_t)kAttnMaxCtas * 2 * (kSelMaxK - 1) * sizeof(unsigned long long), 256);
+    L.total = align_up(L.part + (size_t)2 * kAttnMaxCtas * (hq / hkv) * kAttnPartStride * sizeof(float), 256);
+    return L;
+}
+
 // grid of the persistent attention kernel: one CTA per SM, never more CTAs
 // than work items so that every CTA owns a non-empty range
 void attn_schedule(AttnArgs &a, bool allow_split) {
@@ -201,6 +218,10 @@ int dsa_index_score(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_q
     a.num_idx_heads = num_idx_heads;
     a.scores = scores;
     a.dev_err = dev_err;
+    // prefill-shaped batches (on average a query tile per sequence) run on the
+    // tensor cores; decode-shaped ones scan with dp4a
+    if ((long long)queries->total_q >= (long long)index_score_tc_min_queries_per_seq() * seqs->num_seqs)
+        return from_cuda(launch_index_score_tc(a, sm_count(), reinterpret_cast<cudaStream_t>(stream)));
     return from_cuda(launch_index_score(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -295,6 +316,61 @@ int dsa_sparse_attn_decode(const dsa_kv_cache *cache, const dsa_seqs *seqs, cons
     a.part = reinterpret_cast<float *>(ws + L.part);
     attn_schedule(a, true);
     return from_cuda(launch_sparse_attn(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t dsa_decode_fused_workspace_size(int32_t total_q, int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t k_max) {
+    if (total_q <= 0 || num_q_heads < 1 || num_kv_heads < 1 || k_max < 1 || num_q_heads % num_kv_heads)
+        return 0;
+    return fused_layout(total_q, num_q_heads, num_kv_heads).total;
+}
+
+int dsa_decode_fused(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                     const int32_t *cu_new, int32_t total_new, const void *k_new, const void *v_new,
+                     const int8_t *kc_new, const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads,
+                     int32_t w_abs_max, const int32_t *k_per_seq, int32_t k_max, const void *q,
+                     int32_t num_q_heads, float sm_scale, int32_t *sel, int32_t *cnt, void *out, float *lse,
+                     void *workspace, size_t workspace_bytes, int32_t *dev_err, dsa_stream_t stream) {
+    AttnArgs a;
+    int rc = attn_common(cache, seqs, queries, q, num_q_heads, sel, cnt, k_max, sm_scale, out, lse, dev_err, a);
+    if (rc) return rc;
+    if (num_idx_heads < 1 || w_abs_max < 0 || total_new < 0) return DSA_ERR_INVALID_ARG;
+    if (num_idx_heads > kMaxIdxHeads || k_max > kSelMaxK || queries->total_q > kFusedMaxQ)
+        return DSA_ERR_UNSUPPORTED;
+    const long long bound = (long long)num_idx_heads * w_abs_max * kIdxDim * 128LL * 128LL;
+    if (bound >= (1LL << 31)) return DSA_ERR_RANGE;
+    if (total_new > 0) {
+        if (!cu_new || !k_new || !v_new) return DSA_ERR_INVALID_ARG;
+        if (!aligned16(k_new) || !aligned16(v_new) || (kc_new && !aligned16(kc_new))) return DSA_ERR_INVALID_ARG;
+    }
+    if (queries->total_q == 0) return DSA_OK;
+    if (!q_idx || !w || !k_per_seq || !aligned16(q_idx)) return DSA_ERR_INVALID_ARG;
+    const FusedLayout L = fused_layout(queries->total_q, num_q_heads, cache->num_kv_heads);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < L.total) return DSA_ERR_WORKSPACE;
+    char *ws = static_cast<char *>(workspace);
+    a.counters = reinterpret_cast<int32_t *>(ws + L.counters);
+    a.part = reinterpret_cast<float *>(ws + L.part);
+    attn_schedule(a, true);
+    FusedArgs f{};
+    f.cu_new = cu_new;
+    f.total_new = total_new;
+    f.k_new = k_new;
+    f.v_new = v_new;
+    f.kc_new = kc_new;
+    f.k_pool = cache->k_pool;
+    f.v_pool = cache->v_pool;
+    f.kc_pool = cache->kc_pool;
+    f.q_idx = q_idx;
+    f.w = w;
+    f.num_idx_heads = num_idx_heads;
+    f.k_per_seq = k_per_seq;
+    f.sel = sel;
+    f.cnt = cnt;
+    f.hdr = reinterpret_cast<int32_t *>(ws + L.hdr);
+    f.sel_count = reinterpret_cast<int32_t *>(ws + L.sel_count);
+    f.flags = reinterpret_cast<int32_t *>(ws + L.flags);
+    f.cand = reinterpret_cast<unsigned long long *>(ws + L.cand);
+    return from_cuda(launch_decode_fused(a, f, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int dsa_sparse_attn_prefill(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,

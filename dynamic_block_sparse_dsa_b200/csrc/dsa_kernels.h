@@ -123,13 +123,43 @@ struct AttnArgs {
     int32_t *dev_err;
 };
 
+// single-launch decode step (append + select + attention in one persistent
+// kernel): the arguments beyond AttnArgs
+constexpr int kFusedMaxQ = 1024;                            // queries per call
+constexpr int kHdrEpoch = 0, kHdrDone = 1, kHdrAppended = 2;  // workspace header words
+struct FusedArgs {
+    // append (total_new == 0: nothing to append)
+    const int32_t *cu_new;
+    int total_new;
+    const void *k_new, *v_new;
+    const int8_t *kc_new;
+    void *k_pool, *v_pool;   // the pools, writable
+    int8_t *kc_pool;
+    // indexer + selection
+    const int8_t *q_idx;     // [T][H][64]
+    const int32_t *w;        // [T][H]
+    int num_idx_heads;
+    const int32_t *k_per_seq;
+    int32_t *sel;            // [T][k_max] (AttnArgs::sel, writable)
+    int32_t *cnt;            // [T]
+    // workspace
+    int32_t *hdr;            // epoch, CTAs done, tokens appended
+    int32_t *sel_count;      // [T] candidate groups merged per query
+    int32_t *flags;          // [T] selection ready: the call's epoch + 1
+    unsigned long long *cand;   // [C][2][kSelMaxK-1] per-CTA Top-(K-1) of split queries
+};
+
 cudaError_t launch_kv_append(const KvAppendArgs &a, cudaStream_t stream);
 cudaError_t launch_index_score(const IndexScoreArgs &a, cudaStream_t stream);
+// tensor-core (tcgen05 int8) scoring for batches with many queries per sequence
+cudaError_t launch_index_score_tc(const IndexScoreArgs &a, int num_sms, cudaStream_t stream);
+int index_score_tc_min_queries_per_seq();
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream);
 cudaError_t launch_select_blocks(const SelectArgs &a, cudaStream_t stream);
 int topk_max_blocks();   // longest block table the standalone Top-K kernel accepts
 // the K/V pool and Q tensor maps are built by the launcher from AttnArgs
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream);
+cudaError_t launch_decode_fused(const AttnArgs &a, const FusedArgs &f, cudaStream_t stream);
 // largest grid the attention kernel uses (sizes the partial-state workspace)
 constexpr int kAttnMaxCtas = 256;
 // floats per partial-state row: o[128], m, l, padded to a 16-byte multiple

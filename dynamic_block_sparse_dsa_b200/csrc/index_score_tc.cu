@@ -1,0 +1,360 @@
+// index_score_tc.cu -- block scores of the int8 indexer on the 5th-generation
+// tensor cores (prefill: many queries per sequence).
+//
+// "Day-0 Adaptation for Massive LLMs: Overcoming Sparse Attention and MXFP4
+// Expert Weights", section 4(1): score the compressed per-block representation
+// against each query in one kernel, writing nothing but the scores;
+// section 4(3): prefill is the compute-heavy phase.  "Day-0 Readiness for
+// Trillion-Parameter Models ...", section "Index Selection Path": low-precision
+// (int8) scoring.  The score is
+//     S[t][b] = sum_h w[t][h] * max(0, q_idx[t][h] . kc[page(s,b)])
+// exactly in int32 (the host checks the range bound).
+//
+// The dot products of a tile of 128 blocks and 16 queries x 16 indexer heads
+// are one int8 contraction D[block][(query, head)] (M = 128, N = 256, K = 64),
+// run with tcgen05.mma kind::i8 into a tensor-memory accumulator; the relu,
+// head weights and head sum then happen in the epilogue, one block row per
+// thread, straight from tensor memory.  One persistent CTA per SM, 6 warps:
+//   warp 0   loader: the tile's 128 coarse keys gathered through the block
+//            table (cp.async, 64-byte swizzle) and the 16 queries' rows
+//            (one 3-D TMA box, heads past H zero-filled), plus the queries'
+//            own blocks and weights, into a 4-stage ring;
+//   warp 1   MMA issuer (one thread): two K=32 MMAs per tile into one of two
+//            256-column accumulators;
+//   warps 2-5 epilogue: tcgen05.ld of the accumulator rows, relu * w summed
+//            over heads, one coalesced 128-byte store per (query, warp).
+// Tiles are (128-block tile, 16-query tile) pairs in block-tile-major order,
+// split evenly over the CTAs; a tile whose queries belong to several
+// sequences is run once per sequence with the other queries masked.  Tiles
+// past every query's own block are skipped.  All waits are bounded.
+#include "dsa_kernels.h"
+#include "dsa_tcgen05.cuh"
+
+namespace dsa {
+
+namespace {
+constexpr int kTcThreads = 192;
+constexpr int kTcStages = 4;
+constexpr int kBT = 128;                 // blocks per tile (MMA M)
+constexpr int kQT = 16;                  // queries per tile (MMA N = 16 x 16 heads)
+constexpr int kN = kQT * kMaxIdxHeads;   // 256
+constexpr int kABytes = kBT * kIdxDim;   // 8 KiB
+constexpr int kBBytes = kN * kIdxDim;    // 16 KiB
+// stage: [A 8 KiB][B 16 KiB][info]
+struct StageInfo {
+    int s, bt, y, end;                   // sequence, block tile, query tile; end marker
+    int own[kQT];                        // own block of each query of the tile in s, else -1
+    uint32_t valid[kBT / 32];            // rows with a usable page
+    int w[kQT][kMaxIdxHeads];            // head weights (0 past H and for masked queries)
+};
+constexpr int kOffB = kABytes;
+constexpr int kOffInfo = kABytes + kBBytes;
+constexpr int kStageBytes = (kOffInfo + (int)sizeof(StageInfo) + 1023) / 1024 * 1024;
+constexpr int kOffBars = kTcStages * kStageBytes;
+// barriers: full[S], empty[S], tfull[2], tempty[2]
+constexpr int kNumBars = 2 * kTcStages + 4;
+constexpr int kOffMisc = kOffBars + kNumBars * 8;   // tmem base, abort flag
+constexpr int kSmemBytes = kOffMisc + 16 + 1024;    // + alignment slack
+constexpr int kFullCount = 33;                       // 32 cp.async arrivals + the info arrival
+constexpr int kEmptyCount = 1 + 4;                   // MMA commit + 4 epilogue warps
+constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+
+struct Bars {
+    uint32_t base;
+    __device__ uint32_t full(int s) const { return base + kOffBars + 8 * s; }
+    __device__ uint32_t empty(int s) const { return base + kOffBars + 8 * (kTcStages + s); }
+    __device__ uint32_t tfull(int b) const { return base + kOffBars + 8 * (2 * kTcStages + b); }
+    __device__ uint32_t tempty(int b) const { return base + kOffBars + 8 * (2 * kTcStages + 2 + b); }
+};
+
+__device__ __forceinline__ int seq_of_query(const IndexScoreArgs &a, int t) { return find_seq(a.cu_q, a.num_seqs, t); }
+}  // namespace
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a, int n_bt, int n_qt) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *g = smem_raw + (base - raw);
+    Bars bars{base};
+    volatile int *misc = reinterpret_cast<volatile int *>(g + kOffMisc);   // [0] tmem base, [1] abort, [2] never
+    volatile int *s_abort = misc + 1;
+    const volatile int *s_never = misc + 2;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(bars.full(s), kFullCount);
+            mbar_init(bars.empty(s), kEmptyCount);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bars.tfull(b), 1);
+            mbar_init(bars.tempty(b), 4);
+        }
+        misc[1] = 0;
+        misc[2] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(smem_u32(g + kOffMisc), kTmemCols);
+        tc::tmem_relinquish();
+    }
+    pdl_trigger();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = (uint32_t)misc[0];
+
+    const long long n_items = (long long)n_bt * n_qt;
+    const long long i0 = n_items * blockIdx.x / gridDim.x, i1 = n_items * (blockIdx.x + 1) / gridDim.x;
+    const int H = a.num_idx_heads;
+
+    if (warp == 0) {
+        // ============================================================ loader
+        if (lane == 0) prefetch_tensormap(&tm_q);
+        pdl_wait();   // coarse keys may come from the preceding append
+        int k = 0;   // sub-items published
+        uint32_t err_bits = 0;
+        for (long long it = i0; it <= i1 && !*s_abort; ++it) {
+            const bool end = it == i1;
+            const int bt = end ? 0 : (int)(it / n_qt), y = end ? 0 : (int)(it % n_qt);
+            const int t0 = kQT * y;
+            // sequences touched by the tile's queries
+            int s_lo = 0, s_hi = -1;
+            if (!end && t0 < a.total_q) {
+                s_lo = seq_of_query(a, t0);
+                s_hi = seq_of_query(a, min(t0 + kQT, a.total_q) - 1);
+            }
+            for (int s = s_lo; end ? (s == s_lo) : (s <= s_hi); ++s) {
+                // own blocks of the tile's queries in s (-1: not in s or invalid)
+                int own = -1;
+                int len = 0;
+                if (!end) {
+                    len = __ldg(a.seq_lens + s);
+                    const int t = t0 + (lane & (kQT - 1));
+                    if (t < a.total_q && __ldg(a.cu_q + s) <= t && t < __ldg(a.cu_q + s + 1)) {
+                        const int p = __ldg(a.q_pos + t);
+                        own = p / kBlockSize;
+                        if (p < 0 || p >= len || own >= a.max_blocks) {
+                            err_bits |= DSA_DEV_ERR_POS;
+                            own = -1;
+                        }
+                    }
+                }
+                const int max_own = __reduce_max_sync(0xffffffffu, own);
+                if (!end && max_own < bt * kBT) continue;   // nothing visible in this tile
+                const int st = k % kTcStages;
+                if (k >= kTcStages && !mbar_wait(bars.empty(st), ((k / kTcStages) - 1) & 1, s_abort)) {
+                    *s_abort = 1;
+                    break;
+                }
+                uint8_t *stage = g + st * kStageBytes;
+                StageInfo *info = reinterpret_cast<StageInfo *>(stage + kOffInfo);
+                const uint32_t sa = base + st * kStageBytes;
+                if (end) {
+                    if (lane == 0) { info->end = 1; info->s = -1; }
+                } else {
+                    if (lane == 0) { info->end = 0; info->s = s; info->bt = bt; info->y = y; }
+                    if (lane < kQT) info->own[lane] = own;
+                    // weights of the tile's queries (0 for masked queries and heads past H)
+                    for (int e = lane; e < kQT * kMaxIdxHeads; e += 32) {
+                        const int qi = e / kMaxIdxHeads, h = e % kMaxIdxHeads;
+                        const int oq = __shfl_sync(0xffffffffu, own, qi);
+                        info->w[qi][h] = (oq >= 0 && h < H) ? __ldg(a.w + (size_t)(t0 + qi) * H + h) : 0;
+                    }
+                    // the 128 coarse keys: 4 rows per lane, 4 x 16 B per row, swizzled
+                    const int n_blocks = (len + kBlockSize - 1) / kBlockSize;
+#pragma unroll
+                    for (int r4 = 0; r4 < kBT / 32; ++r4) {
+                        const int r = r4 * 32 + lane;
+                        const int b = bt * kBT + r;
+                        int page = -1;
+                        if (b < n_blocks && b < a.max_blocks && b <= max_own) {
+                            page = __ldg(a.block_table + (size_t)s * a.max_blocks + b);
+                            if (page < 0 || page >= a.num_pages) {
+                                err_bits |= DSA_DEV_ERR_PAGE;
+                                page = -1;
+                            }
+                        }
+                        const uint32_t bits = __ballot_sync(0xffffffffu, page >= 0);
+                        if (lane == 0) info->valid[r4] = bits;
+                        const int8_t *src = a.kc_pool + (size_t)max(page, 0) * kIdxDim;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const uint32_t dst = sa + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+                            if (page >= 0) cp_async_16(dst, src + 16 * c);
+                            else cp_async_16_zero(dst, a.kc_pool);
+                        }
+                    }
+                    // the queries' rows: box (64 B, 16 heads, 16 queries) at query t0
+                    if (lane == 0) {
+                        tc::mbar_expect_tx(bars.full(st), kBBytes);
+                        tma_load_3d(sa + kOffB, &tm_q, 0, 0, t0, bars.full(st));
+                    }
+                }
+                tc::cp_async_arrive_noinc(bars.full(st));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars.full(st));   // the info words above
+                ++k;
+                if (end) break;
+            }
+        }
+        err_bits = __reduce_or_sync(0xffffffffu, err_bits);
+        if (lane == 0 && err_bits) set_err(a.dev_err, err_bits);
+        // nothing may still be landing when the CTA winds down
+        cp_async_wait<0>();
+        if (*s_abort && lane == 0) {
+            set_err(a.dev_err, DSA_DEV_ERR_WAIT);
+            for (int j = max(0, k - kTcStages); j < k; ++j)
+                mbar_wait(bars.full(j % kTcStages), (j / kTcStages) & 1, s_never);
+        }
+    } else if (warp == 1) {
+        // ============================================================ MMA issuer
+        constexpr uint32_t idesc = tc::idesc_i8(kBT, kN);
+        int k = 0;
+        while (true) {
+            const int st = k % kTcStages, buf = k & 1;
+            bool ok = mbar_wait(bars.full(st), (k / kTcStages) & 1, s_abort);
+            if (ok && k >= 2) ok = mbar_wait(bars.tempty(buf), ((k >> 1) - 1) & 1, s_abort);
+            if (!ok) {
+                if (lane == 0) *s_abort = 1;
+                break;
+            }
+            const StageInfo *info = reinterpret_cast<const StageInfo *>(g + st * kStageBytes + kOffInfo);
+            const bool end = info->end != 0;
+            if (lane == 0) {
+                if (end) {
+                    mbar_arrive(bars.tfull(buf));   // wake the epilogue to see the end marker
+                } else {
+                    tc::fence_proxy_async_smem();   // the cp.async-written keys, for the tensor core
+                    tc::fence_after_sync();
+                    const uint32_t sa = base + st * kStageBytes;
+                    const uint32_t d = tmem + (uint32_t)(buf * kN);
+                    const uint64_t da = tc::smem_desc_k64_sw64(sa), db = tc::smem_desc_k64_sw64(sa + kOffB);
+                    tc::mma_i8(d, da, db, idesc, false);
+                    tc::mma_i8(d, da + (32 >> 4), db + (32 >> 4), idesc, true);   // K bytes 32..63
+                    tc::commit(bars.empty(st));
+                    tc::commit(bars.tfull(buf));
+                }
+            }
+            __syncwarp();
+            ++k;
+            if (end) break;
+        }
+        // the last MMAs have completed before the accumulator is released
+        if (lane == 0 && k > 0) {
+            const int j = k - 1;
+            mbar_wait(bars.tfull(j & 1), (j >> 1) & 1, s_never);
+        }
+    } else {
+        // ============================================================ epilogue
+        const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+        const int row = quarter * 32 + lane;     // block row of the tile
+        int k = 0;
+        while (true) {
+            const int st = k % kTcStages, buf = k & 1;
+            bool ok = mbar_wait(bars.tfull(buf), (k >> 1) & 1, s_abort) &&
+                      mbar_wait(bars.full(st), (k / kTcStages) & 1, s_abort);   // acquire the info words
+            if (!ok) {
+                if (lane == 0) *s_abort = 1;
+                break;
+            }
+            tc::fence_after_sync();
+            const StageInfo *info = reinterpret_cast<const StageInfo *>(g + st * kStageBytes + kOffInfo);
+            if (info->end) break;
+            const int bt = info->bt, y = info->y;
+            const int b = bt * kBT + row;
+            const bool row_ok = (info->valid[row >> 5] >> (row & 31)) & 1u;
+            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kN);
+#pragma unroll 1
+            for (int j = 0; j < kQT / 2; ++j) {
+                uint32_t v[32];
+                tc::ld_32x32b_x32(taddr + 32 * j, v);
+                tc::wait_ld();
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int qi = 2 * j + u;
+                    const int4 *wq = reinterpret_cast<const int4 *>(info->w[qi]);
+                    int sum = 0;
+#pragma unroll
+                    for (int h4 = 0; h4 < 4; ++h4) {
+                        const int4 wv = wq[h4];
+                        sum += wv.x * max((int)v[16 * u + 4 * h4 + 0], 0);
+                        sum += wv.y * max((int)v[16 * u + 4 * h4 + 1], 0);
+                        sum += wv.z * max((int)v[16 * u + 4 * h4 + 2], 0);
+                        sum += wv.w * max((int)v[16 * u + 4 * h4 + 3], 0);
+                    }
+                    if (row_ok && b <= info->own[qi]) a.scores[(size_t)(kQT * y + qi) * a.max_blocks + b] = sum;
+                }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bars.tempty(buf));
+                mbar_arrive(bars.empty(st));
+            }
+            ++k;
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+namespace {
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn tc_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+}  // namespace
+
+int index_score_tc_min_queries_per_seq() { return 16; }
+
+cudaError_t launch_index_score_tc(const IndexScoreArgs &a, int num_sms, cudaStream_t stream) {
+    if (a.total_q == 0 || a.num_seqs == 0) return cudaSuccess;
+    EncodeTiledFn enc = tc_encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    // q_idx as (64 bytes, head, query); boxes of 64 B x 16 heads x 16 queries,
+    // zero-filled past H heads and past the last query
+    CUtensorMap tq;
+    const cuuint64_t dims[3] = {(cuuint64_t)kIdxDim, (cuuint64_t)a.num_idx_heads, (cuuint64_t)a.total_q};
+    const cuuint64_t strides[2] = {(cuuint64_t)kIdxDim, (cuuint64_t)a.num_idx_heads * kIdxDim};
+    const cuuint32_t box[3] = {kIdxDim, kMaxIdxHeads, kQT};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<int8_t *>(a.q_idx), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    static unsigned long long attr_done = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !(attr_done & (1ull << dev))) {
+        e = cudaFuncSetAttribute(index_score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) attr_done |= 1ull << dev;
+    }
+    const int n_bt = (a.max_blocks + kBT - 1) / kBT;
+    const int n_qt = (a.total_q + kQT - 1) / kQT;
+    const long long items = (long long)n_bt * n_qt;
+    const int grid = (int)(items < num_sms ? items : num_sms);
+    return launch_pdl(index_score_tc_kernel, dim3(grid), dim3(kTcThreads), (size_t)kSmemBytes, stream, tq, a, n_bt,
+                      n_qt);
+}
+
+}  // namespace dsa

@@ -32,6 +32,7 @@
 // All waits are bounded (DSA_DEV_ERR_WAIT on timeout, no hang).
 #include "dsa_kernels.h"
 #include "dsa_tma.cuh"
+#include "decode_fused.cuh"
 
 namespace dsa {
 
@@ -46,7 +47,7 @@ constexpr int kSegSlots = 2;                       // query tile + pair facts, d
 constexpr int kMergeStride = 132;                  // floats per merge row (padded against bank conflicts)
 constexpr int kMaxSmemSeqs = 256;                  // cu_q entries cached in shared memory
 // int words after the barriers
-constexpr int kWAbort = 0, kWLast = 1, kWNever = 2;
+constexpr int kWAbort = 0, kWLast = 1, kWNever = 2, kWTag = 3;
 constexpr int kWFill = 4;                           // [kMaxStages] item index the stage was last armed for
 constexpr int kMaxStages = 8;
 constexpr int kWItemBlk = kWFill + kMaxStages;      // [kMaxStages] logical block of that item
@@ -54,7 +55,8 @@ constexpr int kWItemSeg = kWItemBlk + kMaxStages;   // [kMaxStages] segment of t
 constexpr int kWSegEndCnt = kWItemSeg + kMaxStages; // [kSegSlots] items issued when the segment ended
 constexpr int kWSegEndTag = kWSegEndCnt + kSegSlots;  // [kSegSlots] which segment that count belongs to
 constexpr int kWSegInfo = kWSegEndTag + kSegSlots;  // [kSegSlots][4]: t, kvh, p, n_vis
-constexpr int kNumWords = kWSegInfo + 4 * kSegSlots;
+constexpr int kWSelLast = kWSegInfo + 4 * kSegSlots;   // fused select: this CTA merges
+constexpr int kNumWords = kWSelLast + 1;
 constexpr float kLn2 = 0.6931471805599453f;
 // most CTAs whose ranges can cover one pair (the host caps the split at 60)
 constexpr int kMaxSplitSlots = 63;
@@ -75,6 +77,7 @@ struct Plan {
     static constexpr int kOffWords = kOffBars + kNumBars * 8;
     static constexpr int kSmemBytes = kOffWords + kNumWords * 4 + 1024;   // + slack to align the base to 1 KiB
     static_assert(kStages <= kMaxStages, "stage words");
+    static_assert(fused::kScratchBytes <= kStages * kStageBytes, "fused select scratch fits the ring");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 
@@ -110,10 +113,14 @@ __device__ __forceinline__ int seq_of(const AttnArgs &a, const int *s_cuq, int t
 }
 }  // namespace
 
-template <int NT>   // query-head n-tiles of 8: the GQA group is <= 8 * NT
+// NT: query-head n-tiles of 8 (the GQA group is <= 8 * NT).  kFused: the
+// single-launch decode step -- phases A (append) and B (select) of
+// decode_fused.cuh run first, and the producer waits for each query's
+// selection before reading it.
+template <int NT, bool kFused>
 __global__ void __launch_bounds__(kAttnThreads, 1)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_q, AttnArgs a) {
+                   const __grid_constant__ CUtensorMap tm_q, AttnArgs a, FusedArgs f) {
     using P = Plan<NT>;
     constexpr int kStages = P::kStages;
     extern __shared__ uint8_t smem_raw[];
@@ -146,10 +153,18 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         for (int k = 0; k < kNumWords; ++k) W[k] = 0;
         for (int s = 0; s < kStages; ++s) W[kWFill + s] = -1;
         for (int s = 0; s < kSegSlots; ++s) W[kWSegEndTag + s] = -1;
+        if (kFused) W[kWTag] = fused::ld_acquire(f.hdr + kHdrEpoch) + 1;
         fence_barrier_init();
     }
     pdl_trigger();
     __syncthreads();
+    const int tag = W[kWTag];
+    if constexpr (kFused) {
+        fused::append_and_select(a, f, gbase, tag, W + kWSelLast);
+        // the ring's generic-proxy use ends before TMA writes into it
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+    }
 
     if (warp == kConsumerWarps) {
         // ================================================================ producer warp
@@ -167,8 +182,17 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             prefetch_tensormap(&tm_q);
         }
         pdl_wait();   // the selection and the appended tokens come from the kernels before
-        int item = 0, seg = 0;
         uint32_t err_bits = 0;
+        if (kFused && f.total_new > 0 && lane == 0) {
+            // a query's own block holds its new token: every append lands before the first TMA
+            const long long t0 = clock64();
+            while (fused::ld_acquire(f.hdr + kHdrAppended) < f.total_new) {
+                if (clock64() - t0 > kWaitLimitCycles) { err_bits |= DSA_DEV_ERR_WAIT; break; }
+            }
+            fused::fence_proxy_async_global();
+        }
+        __syncwarp();
+        int item = 0, seg = 0;
         bool stop = false;
         for (long long base = u0; base < u1 && !stop; base += 32) {
             const long long uu = base + lane;
@@ -182,8 +206,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 s = seq_of(a, s_cuq, t);
                 p = __ldg(a.q_pos + t);
                 const int len = __ldg(a.seq_lens + s);
-                int n_sel = __ldg(a.cnt + t);
-                const int b = __ldg(a.sel + (size_t)t * a.k_max + j);
+                bool ready = true;
+                if (kFused && !fused::wait_flag(f.flags + t, tag)) {   // this query's selection is published
+                    err_bits |= DSA_DEV_ERR_WAIT;
+                    ready = false;
+                }
+                // the selection may have been written during this launch: read it through L2
+                int n_sel = ready ? __ldcg(a.cnt + t) : 0;
+                const int b = ready ? __ldcg(a.sel + (size_t)t * a.k_max + j) : -1;
                 n_vis = p / kBlockSize + 1;
                 if (p < 0 || p >= len || n_vis > a.max_blocks || n_sel < 0 || n_sel > a.k_max) n_sel = 0;
                 if (j < n_sel) {
@@ -614,6 +644,20 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         ++pair;
         ++seg;
     }
+    if constexpr (kFused) {
+        // the last CTA to finish clears the per-call counters and advances the
+        // epoch, which retires this call's ready flags
+        named_barrier(1, kConsumerWarps * 32);
+        if (tid == 0) {
+            __threadfence();
+            const int old = atomic_add_acq_rel_gpu(f.hdr + kHdrDone, 1);
+            if (old == (int)gridDim.x - 1) {
+                f.hdr[kHdrAppended] = 0;
+                f.hdr[kHdrDone] = 0;
+                fused::st_release(f.hdr + kHdrEpoch, tag);
+            }
+        }
+    }
 }
 
 namespace {
@@ -636,22 +680,25 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream) {
-    if (a.total_q == 0 || a.num_ctas == 0) return cudaSuccess;
+namespace {
+struct AttnMaps {
+    CUtensorMap k, v, q;
+};
+
+cudaError_t make_maps(const AttnArgs &a, AttnMaps &m) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
     // K / V pool: dims (head_dim, kv_head, page*64+token), boxes of 64 dims x 1 head x 64 tokens
-    CUtensorMap tk, tv, tq;
     const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)a.num_kv_heads,
                                 (cuuint64_t)a.num_pages * kBlockSize};
     const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)a.num_kv_heads * kHeadDim * 2};
     const cuuint32_t box[3] = {64, 1, kBlockSize};
     const cuuint32_t estr[3] = {1, 1, 1};
-    if (enc(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(a.k_pool), dims, strides, box,
+    if (enc(&m.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(a.k_pool), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    if (enc(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(a.v_pool), dims, strides, box,
+    if (enc(&m.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(a.v_pool), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
@@ -659,29 +706,74 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream) {
     const cuuint64_t qdims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)a.total_q * a.num_q_heads};
     const cuuint64_t qstr[1] = {(cuuint64_t)kHeadDim * 2};
     const cuuint32_t qbox[2] = {64, 16};
-    if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(a.q), qdims, qstr, qbox, estr,
+    if (enc(&m.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(a.q), qdims, qstr, qbox, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+    return cudaSuccess;
+}
 
-    static unsigned long long attr_done = 0;   // the shared-memory opt-in is per device
+// the shared-memory opt-in of every instantiation, once per device
+cudaError_t set_smem_attrs() {
+    static unsigned long long attr_done = 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !(attr_done & (1ull << dev))) {
-        e = cudaFuncSetAttribute(sparse_attn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (dev < 64 && (attr_done & (1ull << dev))) return cudaSuccess;
+    e = cudaFuncSetAttribute(sparse_attn_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Plan<1>::kSmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sparse_attn_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Plan<2>::kSmemBytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sparse_attn_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Plan<1>::kSmemBytes);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(sparse_attn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     Plan<2>::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        if (dev < 64) attr_done |= 1ull << dev;
-    }
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(sparse_attn_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Plan<2>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) attr_done |= 1ull << dev;
+    return cudaSuccess;
+}
+}  // namespace
+
+cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream) {
+    if (a.total_q == 0 || a.num_ctas == 0) return cudaSuccess;
+    AttnMaps m;
+    cudaError_t e = make_maps(a, m);
+    if (e == cudaSuccess) e = set_smem_attrs();
+    if (e != cudaSuccess) return e;
+    const FusedArgs none{};
     if (a.group <= 8)
-        return launch_pdl(sparse_attn_kernel<1>, dim3(a.num_ctas), dim3(kAttnThreads), Plan<1>::kSmemBytes, stream,
-                          tk, tv, tq, a);
-    return launch_pdl(sparse_attn_kernel<2>, dim3(a.num_ctas), dim3(kAttnThreads), Plan<2>::kSmemBytes, stream, tk,
-                      tv, tq, a);
+        return launch_pdl(sparse_attn_kernel<1, false>, dim3(a.num_ctas), dim3(kAttnThreads), Plan<1>::kSmemBytes,
+                          stream, m.k, m.v, m.q, a, none);
+    return launch_pdl(sparse_attn_kernel<2, false>, dim3(a.num_ctas), dim3(kAttnThreads), Plan<2>::kSmemBytes,
+                      stream, m.k, m.v, m.q, a, none);
+}
+
+cudaError_t launch_decode_fused(const AttnArgs &a, const FusedArgs &f, cudaStream_t stream) {
+    if (a.total_q == 0 || a.num_ctas == 0) return cudaSuccess;
+    AttnMaps m;
+    cudaError_t e = make_maps(a, m);
+    if (e == cudaSuccess) e = set_smem_attrs();
+    if (e != cudaSuccess) return e;
+    // every CTA resident at once: the attention phase waits on selections
+    // that other CTAs publish
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.num_ctas);
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (a.group <= 8) {
+        cfg.dynamicSmemBytes = Plan<1>::kSmemBytes;
+        return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<1, true>, m.k, m.v, m.q, a, f);
+    }
+    cfg.dynamicSmemBytes = Plan<2>::kSmemBytes;
+    return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<2, true>, m.k, m.v, m.q, a, f);
 }
 
 }  // namespace dsa

@@ -210,6 +210,37 @@ int dsa_sparse_attn_prefill(const dsa_kv_cache *cache, const dsa_seqs *seqs,
                             void *out, float *lse, int32_t *dev_err, dsa_stream_t stream);
 
 /*
+ * dsa_decode_fused -- one decode step in a single launch: dsa_kv_append, the
+ * selection of dsa_select_blocks and dsa_sparse_attn_decode run as phases of
+ * one persistent kernel [P5 "Differentiated Adaptation of Prefill and
+ * Decode": in decode, fuse index selection, the gather and attention; P1
+ * 4(1): block-wise scoring with partial selection].  Arguments are those of
+ * the three calls; the results (the pools after the append, sel, cnt, out,
+ * lse) are the same bits.
+ *  - Every appended block of a sequence must lie at or after the own block of
+ *    each of that sequence's queries (decode: one new token per sequence,
+ *    whose query sits at its position).  A query that breaks this gets
+ *    DSA_DEV_ERR_POS and cnt 0.  With total_new == 0 nothing is appended.
+ *  - total_q <= 1024, k_max <= 64, num_idx_heads <= 16.
+ *  - Needs a workspace of dsa_decode_fused_workspace_size() bytes, zero-filled
+ *    before its first use; each call leaves it ready for the next (it keeps a
+ *    call counter, so calls that share one workspace must not overlap).
+ *  - Every CTA of the grid must be resident at once (a cooperative launch):
+ *    the call fails with DSA_ERR_CUDA if the GPU cannot give it one CTA per
+ *    SM.  Waits between phases are bounded (DSA_DEV_ERR_WAIT on timeout).
+ * Device errors: those of the three calls.
+ */
+size_t dsa_decode_fused_workspace_size(int32_t total_q, int32_t num_q_heads, int32_t num_kv_heads,
+                                       int32_t k_max);
+
+int dsa_decode_fused(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                     const int32_t *cu_new, int32_t total_new, const void *k_new, const void *v_new,
+                     const int8_t *kc_new, const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads,
+                     int32_t w_abs_max, const int32_t *k_per_seq, int32_t k_max, const void *q,
+                     int32_t num_q_heads, float sm_scale, int32_t *sel, int32_t *cnt, void *out, float *lse,
+                     void *workspace, size_t workspace_bytes, int32_t *dev_err, dsa_stream_t stream);
+
+/*
  * dsa_sparse_attn_decode_noalloc -- the decode attention above for callers
  * that cannot allocate device memory.  The pages have no counterpart to this
  * call; it exists for callers such as an engine plugin whose enqueue path must

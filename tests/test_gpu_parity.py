@@ -27,12 +27,12 @@ def _handles(wl):
             dsa.QueryBatch(wl.cu_q, wl.q_pos))
 
 
-def gpu_step(wl, decode=True, bufs=None, fused=False):
+def gpu_step(wl, decode=True, bufs=None, fused=False, fused_decode=False):
     cache, seqs, queries = _handles(wl)
     err = torch.zeros(1, dtype=torch.int32, device=wl.device)
     bufs = dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
                     q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=wl.spec.k_max,
-                    decode=decode, fused_select=fused, bufs=bufs, dev_err=err)
+                    decode=decode, fused_select=fused, fused_decode=fused_decode, bufs=bufs, dev_err=err)
     torch.cuda.synchronize()
     return bufs, int(err.item())
 
@@ -78,6 +78,11 @@ SMALL = {
                              k_per_seq=(8,) * 40, k_max=8),
     "prefill_two_chunks": dict(seq_lens=(3000, 2111), n_new=(200, 130), k_per_seq=(12, 7), k_max=12,
                                occupancy=0.6),
+    # query tiles of 16 that straddle sequence boundaries (tensor-core scoring path)
+    "prefill_tiles_straddle": dict(seq_lens=(9000, 300, 5000, 70), n_new=(30, 20, 17, 5), k_per_seq=(9, 3, 6, 2),
+                                   k_max=9),
+    # fewer indexer heads than the 16 of a tensor-core tile
+    "prefill_5_idx_heads": dict(seq_lens=(20000,), n_new=(100,), k_per_seq=(10,), k_max=10, num_idx_heads=5),
 }
 
 
@@ -255,3 +260,111 @@ def test_fused_select_equals_score_then_topk_on_ties(cuda_device):
     own = (wl.q_pos // 64).cpu()
     sel = b1["sel"].cpu()
     assert sel[0, :32].tolist() == list(range(32)) and int(sel[0, 32]) == int(own[0])
+
+
+# ----------------------------------------------------------------------------- single-launch decode
+def _decode_eligible(wl):
+    """Queries whose sequence appends nothing before their own block (the
+    single-launch decode step's precondition)."""
+    spec = wl.spec
+    cu = wl.cu_q.cpu().numpy()
+    pos = wl.q_pos.cpu().numpy()
+    ok = []
+    for s in range(spec.num_seqs):
+        first_new_block = (spec.seq_lens[s] - spec.n_new[s]) // 64
+        for t in range(cu[s], cu[s + 1]):
+            ok.append(spec.n_new[s] == 0 or pos[t] // 64 <= first_new_block)
+    return np.array(ok, dtype=bool)
+
+
+FUSED_DECODE_SMALL = sorted(n for n in SMALL if not n.startswith(("ragged_prefill", "prefill")))
+
+
+@pytest.mark.parametrize("q_scale", [1.0, 12.0], ids=["plain", "sharp"])
+@pytest.mark.parametrize("name", FUSED_DECODE_SMALL)
+def test_fused_decode_small_cases(name, q_scale, cuda_device):
+    wl = wk.make_workload(_small_spec(name, q_scale), seed=100 + len(name), device=cuda_device)
+    assert _decode_eligible(wl).all()
+    ref = oracle_step(wl)
+    bufs, err = gpu_step(wl, fused_decode=True)
+    assert err == 0, f"device error bits {err}"
+    compare(wl, ref, bufs, fused=True)
+
+
+def test_fused_decode_flags_non_decode_queries(cuda_device):
+    # prefill-shaped sequences: queries before the last appended block are
+    # refused (cnt 0, DEV_ERR_POS); every other query is still exact
+    wl = wk.make_workload(_small_spec("ragged_prefill_tail", 8.0), seed=41, device=cuda_device)
+    ok = _decode_eligible(wl)
+    assert ok.any() and not ok.all()
+    good = [int(t) for t in np.flatnonzero(ok)]
+    ref = oracle_step(wl, queries=good)
+    bufs, err = gpu_step(wl, fused_decode=True)
+    assert err & dsa._lib.DEV_ERR_POS
+    compare(wl, ref, bufs, fused=True)
+    cnt = bufs["cnt"].cpu().numpy()
+    assert (cnt[~ok] == 0).all()
+
+
+def test_fused_decode_tiny_workload(cuda_device):
+    wl, ref, bufs = _run(wk.tiny_decode(), 1001, cuda_device, scores=False)
+    b2, err = gpu_step(wl, fused_decode=True)
+    assert err == 0
+    compare(wl, ref, b2, fused=True)
+
+
+@pytest.mark.parametrize("q_scale", [1.0, 12.0])
+def test_fused_decode_batched_gqa_workload(q_scale, cuda_device):
+    spec = wk.scaled(wk.batched_gqa_decode(), q_scale=q_scale)
+    wl = wk.make_workload(spec, seed=1002, device=cuda_device)
+    ref = oracle_step(wl)
+    bufs, err = gpu_step(wl, fused_decode=True)
+    assert err == 0
+    compare(wl, ref, bufs, fused=True)
+
+
+@pytest.mark.slow
+def test_fused_decode_1m_workload(cuda_device):
+    wl = wk.make_workload(wk.decode_1m(), seed=1003, device=cuda_device)
+    ref = oracle_step(wl)
+    bufs, err = gpu_step(wl, fused_decode=True)
+    assert err == 0
+    compare(wl, ref, bufs, fused=True)
+
+
+def test_fused_decode_repeat_calls_and_equals_three_kernel_path(cuda_device):
+    # the workspace keeps an epoch: many calls on one workspace stay exact and
+    # give the same bits as append -> select -> decode attention
+    spec = wk.WorkloadSpec("fused_repeat", seq_lens=(5000, 64, 20000, 130), n_new=(1, 1, 1, 1),
+                           k_per_seq=(9, 4, 33, 2), k_max=33, num_q_heads=16, num_kv_heads=2, q_scale=6.0)
+    wl = wk.make_workload(spec, seed=42, device=cuda_device)
+    b_ref, e_ref = gpu_step(wl, fused=True)
+    assert e_ref == 0
+    b = None
+    for _ in range(5):
+        b, err = gpu_step(wl, bufs=b, fused_decode=True)
+        assert err == 0
+        for k in ("sel", "cnt", "out", "lse"):
+            assert torch.equal(b[k], b_ref[k]), k
+    ref = oracle_step(wl)
+    compare(wl, ref, b, fused=True)
+
+
+@pytest.mark.parametrize("what", ["page", "pos", "k"])
+def test_fused_decode_bad_metadata_sets_flags(what, cuda_device):
+    spec = _small_spec("k_covers_all")
+    wl = wk.make_workload(spec, seed=43, device=cuda_device)
+    if what == "page":
+        wl.block_table[0, 1] = spec.num_pages + 5
+        bit = dsa._lib.DEV_ERR_PAGE
+    elif what == "pos":
+        wl.q_pos[1] = int(wl.seq_lens[1]) + 3
+        bit = dsa._lib.DEV_ERR_POS
+    else:
+        wl.k_per_seq[0] = 0
+        bit = dsa._lib.DEV_ERR_K
+    b, err = gpu_step(wl, fused_decode=True)
+    assert err & bit
+    assert not err & dsa._lib.DEV_ERR_WAIT
+    if what != "page":
+        assert int(b["cnt"][0 if what == "k" else 1]) == 0
