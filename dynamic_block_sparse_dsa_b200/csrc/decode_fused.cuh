@@ -9,9 +9,7 @@
 // block-wise scoring and partial selection instead of a full sort.
 //
 // One persistent CTA per SM runs three phases:
-//   A. append: CTA c copies new tokens c, c + C, ... into their page slots and
-//      releases a count of appended tokens;
-//   B. select: the (query, 64-candidate group) list is split evenly over the
+//   1. select: the (query, 64-candidate group) list is split evenly over the
 //      CTAs.  A CTA stages the page ids, the coarse keys (cp.async into its
 //      idle TMA ring) and the query rows of up to kRoundGroups groups at once,
 //      scores them on the int8 tensor cores and folds each group's 64 keys
@@ -20,11 +18,14 @@
 //      CTA completing its group count (acq_rel atomic, no waiting) merges the
 //      lists.  The finaliser writes the ascending selection and releases the
 //      query's ready flag;
-//   C. attention: the producer warp acquires the ready flag of each query
+//   2. append: CTA c copies new tokens c, c + C, ... into their page slots and
+//      releases a count of appended tokens (after the selection, which never
+//      reads them, so the copies stay off the selection's critical path);
+//   3. attention: the producer warp acquires the ready flag of each query
 //      before reading its selection, and the appended-token count before its
 //      first TMA (a decode query's own block holds the new token).
-// Phases A and B never wait on another CTA, so with every CTA resident (a
-// cooperative launch) the waits of phase C always end; they are bounded all
+// Phases 1 and 2 never wait on another CTA, so with every CTA resident (a
+// cooperative launch) the waits of phase 3 always end; they are bounded all
 // the same.  Flags carry an epoch tag that the last CTA to finish advances,
 // so the workspace needs no clearing between calls.
 //
@@ -34,6 +35,8 @@
 // one new token is the query itself), and the own block is always selected
 // without being scored.
 #pragma once
+
+#include <climits>
 
 #include "dsa_kernels.h"
 #include "dsa_tma.cuh"
@@ -47,7 +50,7 @@ namespace fused {
 constexpr int kThreads = 160;           // the attention kernel's 5 warps
 constexpr int kWarps = kThreads / 32;
 constexpr int kRoundGroups = 24;        // 64-block groups staged per round
-// byte offsets inside the (idle) TMA ring during phases A/B
+// byte offsets inside the (idle) TMA ring during the select phase
 constexpr int kOffKc = 0;                                           // [kRoundGroups*64][64] int8, chunk-swizzled
 constexpr int kOffPages = kOffKc + kRoundGroups * 64 * 64;          // [kRoundGroups*64] int32
 constexpr int kOffGq = kOffPages + kRoundGroups * 64 * 4;           // [kRoundGroups] query of each group
@@ -58,7 +61,9 @@ constexpr int kOffW = kOffQi + kRoundGroups * kMaxIdxHeads * kIdxDim;   // [kRou
 constexpr int kOffLists = (kOffW + kRoundGroups * kMaxIdxHeads * 4 + 15) / 16 * 16;   // [kWarps*64] u64
 constexpr int kOffGstart = kOffLists + kWarps * 64 * 8;             // [kFusedMaxQ+1] int32
 constexpr int kOffFact = (kOffGstart + (kFusedMaxQ + 1) * 4 + 15) / 16 * 16;   // [kFusedMaxQ] int4
-constexpr int kScratchBytes = kOffFact + kFusedMaxQ * 16;
+constexpr int kCuqCache = 1024;                                     // cu_q entries staged
+constexpr int kOffCuq = kOffFact + kFusedMaxQ * 16;                 // [kCuqCache+1] int32
+constexpr int kScratchBytes = kOffCuq + (kCuqCache + 1) * 4;
 
 __device__ __forceinline__ int ld_acquire(const int32_t *p) {
     int v;
@@ -124,15 +129,12 @@ __device__ __forceinline__ void finalize(const AttnArgs &a, const FusedArgs &f, 
     if (lane == 0) st_release(f.flags + t, tag);
 }
 
-// Phases A and B.  Every thread of the CTA calls it; `scratch` is the idle
-// TMA ring (generic pointer, 16-byte aligned, kScratchBytes long).
-__device__ __forceinline__ void append_and_select(const AttnArgs &a, const FusedArgs &f, uint8_t *scratch,
-                                                  int tag, volatile int *s_last) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// Phase 2: CTA c copies new tokens c, c + C, ... into their page slots (K, V
+// and, for the last new token of a block, the coarse key) and adds the count
+// to the workspace.  Run after the selection: no selection reads these rows.
+__device__ __forceinline__ void append_tokens(const AttnArgs &a, const FusedArgs &f) {
+    const int tid = threadIdx.x;
     const int c = blockIdx.x, C = gridDim.x;
-    const int T = a.total_q;
-
-    // ------------------------------------------------------------ A. append
     if (f.total_new > 0) {
         const int row16 = a.num_kv_heads * (kHeadDim * 2 / 16);   // 16-byte vectors per token row
         int done = 0;
@@ -181,6 +183,16 @@ __device__ __forceinline__ void append_and_select(const AttnArgs &a, const Fused
         }
     }
 
+}
+
+// Phase 1.  Every thread of the CTA calls it; `scratch` is the idle TMA ring
+// (generic pointer, 16-byte aligned, kScratchBytes long).
+__device__ __forceinline__ void select_blocks_phase(const AttnArgs &a, const FusedArgs &f, uint8_t *scratch,
+                                                  int tag, volatile int *s_last) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int c = blockIdx.x, C = gridDim.x;
+    const int T = a.total_q;
+
     // ------------------------------------------------------------ B. select
     int *s_gstart = reinterpret_cast<int *>(scratch + kOffGstart);
     Fact *s_fact = reinterpret_cast<Fact *>(scratch + kOffFact);
@@ -194,11 +206,28 @@ __device__ __forceinline__ void append_and_select(const AttnArgs &a, const Fused
     const uint32_t s_kc = smem_u32(scratch + kOffKc);
     int *s_cnt = s_pages;   // group counts of the queries, before the first round
 
-    // facts and candidate-group counts of every query
+    // facts and candidate-group counts of every query: cu_q and the positions
+    // first (one round trip), then the per-sequence facts (a second one)
+    int *s_cuq = reinterpret_cast<int *>(scratch + kOffCuq);
+    const bool cuq_cached = a.num_seqs + 1 <= kCuqCache + 1;
+    if (cuq_cached)
+        for (int i = tid; i <= a.num_seqs; i += kThreads) s_cuq[i] = __ldg(a.cu_q + i);
+    for (int t = tid; t < T; t += kThreads) s_fact[t].p = __ldg(a.q_pos + t);
+    __syncthreads();
     uint32_t err_bits = 0;
     for (int t = tid; t < T; t += kThreads) {
-        const int s = find_seq(a.cu_q, a.num_seqs, t);
-        const int p = __ldg(a.q_pos + t);
+        int s;
+        if (cuq_cached) {
+            int lo = 0, hi = a.num_seqs - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_cuq[mid] <= t) lo = mid; else hi = mid - 1;
+            }
+            s = lo;
+        } else {
+            s = find_seq(a.cu_q, a.num_seqs, t);
+        }
+        const int p = s_fact[t].p;
         const int len = __ldg(a.seq_lens + s);
         int k = __ldg(f.k_per_seq + s);
         const int n_vis = p / kBlockSize + 1;
@@ -279,40 +308,73 @@ __device__ __forceinline__ void append_and_select(const AttnArgs &a, const Fused
         }
         __syncthreads();
         const int nq = s_gqs[ng - 1] + 1;
-        // page ids of the staged candidates (-1: past the candidates or a bad page)
-        for (int e = tid; e < ng * 64; e += kThreads) {
-            const int t = s_gq[e >> 6];
-            const Fact q = s_fact[t];
-            const int b = 64 * (r0 + (e >> 6) - s_gstart[t]) + (e & 63);
-            int page = -1;
-            if (b < q.n_vis - 1) {
-                page = __ldg(a.block_table + (size_t)q.s * a.max_blocks + b);
-                if (page < 0 || page >= a.num_pages) {
-                    err_bits |= DSA_DEV_ERR_PAGE;
-                    page = -1;
-                }
+        // page ids of the staged candidates (-1: past the candidates or a bad
+        // page), the round's query rows and head weights: every load in
+        // registers first, so they all travel in one round trip
+        constexpr int kRowsPT = (kRoundGroups * 64 + kThreads - 1) / kThreads;
+        int pg[kRowsPT];
+#pragma unroll
+        for (int k = 0; k < kRowsPT; ++k) {
+            const int e = tid + k * kThreads;
+            pg[k] = INT_MIN;   // not a candidate
+            if (e < ng * 64) {
+                const int t = s_gq[e >> 6];
+                const Fact q = s_fact[t];
+                const int b = 64 * (r0 + (e >> 6) - s_gstart[t]) + (e & 63);
+                if (b < q.n_vis - 1) pg[k] = __ldg(a.block_table + (size_t)q.s * a.max_blocks + b);
             }
-            s_pages[e] = page;
         }
-        // query rows and head weights of the round's queries (heads past H read as zero)
-        for (int e = tid; e < nq * kMaxIdxHeads * 4; e += kThreads) {
+        int4 qv[kRowsPT];
+#pragma unroll
+        for (int k = 0; k < kRowsPT; ++k) {   // nq * 16 heads * 4 int4 <= kRoundGroups * 64
+            const int e = tid + k * kThreads;
+            qv[k] = make_int4(0, 0, 0, 0);
             const int qq = e / (kMaxIdxHeads * 4), h = (e >> 2) & (kMaxIdxHeads - 1);
-            const int t = s_qlist[qq];
-            s_qi[e] = h < H ? __ldg(reinterpret_cast<const int4 *>(f.q_idx + ((size_t)t * H + h) * kIdxDim) + (e & 3))
-                            : make_int4(0, 0, 0, 0);
+            if (e < nq * kMaxIdxHeads * 4 && h < H)
+                qv[k] = __ldg(reinterpret_cast<const int4 *>(f.q_idx + ((size_t)s_qlist[qq] * H + h) * kIdxDim) +
+                              (e & 3));
         }
-        for (int e = tid; e < nq * kMaxIdxHeads; e += kThreads) {
+        int wv[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {   // nq * 16 <= 384 <= 2 * kThreads + 64: the rest below
+            const int e = tid + k * kThreads;
+            const int qq = e / kMaxIdxHeads, h = e % kMaxIdxHeads;
+            wv[k] = (e < nq * kMaxIdxHeads && h < H) ? __ldg(f.w + (size_t)s_qlist[qq] * H + h) : 0;
+        }
+        for (int e = tid + 2 * kThreads; e < nq * kMaxIdxHeads; e += kThreads) {
             const int qq = e / kMaxIdxHeads, h = e % kMaxIdxHeads;
             s_w[e] = h < H ? __ldg(f.w + (size_t)s_qlist[qq] * H + h) : 0;
         }
-        __syncthreads();
-        // coarse keys, 16-byte chunks swizzled by (row / 2) % 4 against bank conflicts
-        for (int e = tid; e < ng * 64 * 4; e += kThreads) {
-            const int row = e >> 2, part = e & 3;
-            const int page = s_pages[row];
-            const uint32_t dst = s_kc + row * 64 + ((part ^ ((row >> 1) & 3)) << 4);
-            if (page >= 0) cp_async_16(dst, f.kc_pool + (size_t)page * kIdxDim + part * 16);
-            else cp_async_16_zero(dst, f.kc_pool);
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int e = tid + k * kThreads;
+            if (e < nq * kMaxIdxHeads) s_w[e] = wv[k];
+        }
+#pragma unroll
+        for (int k = 0; k < kRowsPT; ++k) {
+            const int e = tid + k * kThreads;
+            if (e < nq * kMaxIdxHeads * 4) s_qi[e] = qv[k];
+        }
+        // coarse keys straight from the page registers: 4 x 16 B per row,
+        // chunks swizzled by (row / 2) % 4 against bank conflicts
+#pragma unroll
+        for (int k = 0; k < kRowsPT; ++k) {
+            const int row = tid + k * kThreads;
+            if (row >= ng * 64) continue;
+            int page = pg[k];
+            if (page == INT_MIN) {
+                page = -1;
+            } else if (page < 0 || page >= a.num_pages) {
+                err_bits |= DSA_DEV_ERR_PAGE;
+                page = -1;
+            }
+            s_pages[row] = page;
+#pragma unroll
+            for (int part = 0; part < 4; ++part) {
+                const uint32_t dst = s_kc + row * 64 + ((part ^ ((row >> 1) & 3)) << 4);
+                if (page >= 0) cp_async_16(dst, f.kc_pool + (size_t)page * kIdxDim + part * 16);
+                else cp_async_16_zero(dst, f.kc_pool);
+            }
         }
         cp_async_commit();
         cp_async_wait<0>();
@@ -366,8 +428,7 @@ __device__ __forceinline__ void append_and_select(const AttnArgs &a, const Fused
                         v[1] = s_pages[r_g8] >= 0 ? make_key64(s_g8, (uint32_t)(b + 8)) : 0ull;
                     }
                 }
-                warp_sort64_desc(v);
-                warp_merge64_desc(acc, v);   // acc starts as zeros: merging into it is a copy
+                warp_fold_topk(acc, v, q.k - 1);
             }
             if (seg_hi <= r0 + ng) {
                 // ---- t's groups in this CTA are done: the CTA's Top-64 of t
@@ -395,14 +456,23 @@ __device__ __forceinline__ void append_and_select(const AttnArgs &a, const Fused
                         // merge the lists of the CTAs covering t (contiguous, non-empty ranges)
                         const int cf = cta_of_group(g_lo, total, C), cl = cta_of_group(g_hi - 1, total, C);
                         key64 m[2] = {0ull, 0ull};
-                        for (int cc = cf + warp; cc <= cl; cc += kWarps) {
-                            const int cb = group_begin(cc, total, C);
-                            if (cb == group_begin(cc + 1, total, C)) continue;   // empty range: no list
-                            const int sl = g_lo < cb ? 0 : 1;
-                            const key64 *src = f.cand + ((size_t)cc * 2 + sl) * (kSelMaxK - 1);
-                            const key64 b2[2] = {lane < kk ? __ldcg(src + lane) : 0ull,
-                                                 32 + lane < kk ? __ldcg(src + 32 + lane) : 0ull};
-                            warp_merge64_desc(m, b2);
+                        constexpr int kBatch = 4;   // lists in flight per warp
+                        for (int c0 = cf + warp; c0 <= cl; c0 += kBatch * kWarps) {
+                            key64 lst[kBatch][2];
+#pragma unroll
+                            for (int j = 0; j < kBatch; ++j) {
+                                const int cc = c0 + j * kWarps;
+                                lst[j][0] = lst[j][1] = 0ull;
+                                if (cc > cl) continue;
+                                const int cb = group_begin(cc, total, C);
+                                if (cb == group_begin(cc + 1, total, C)) continue;   // empty range: no list
+                                const int sl = g_lo < cb ? 0 : 1;
+                                const key64 *src = f.cand + ((size_t)cc * 2 + sl) * (kSelMaxK - 1);
+                                if (lane < kk) lst[j][0] = __ldcg(src + lane);
+                                if (32 + lane < kk) lst[j][1] = __ldcg(src + 32 + lane);
+                            }
+#pragma unroll
+                            for (int j = 0; j < kBatch; ++j) warp_merge64_desc(m, lst[j]);
                         }
                         cta_merge_top64<kWarps>(m, s_lists);
                         if (warp == 0) {

@@ -54,7 +54,12 @@ constexpr int kOffBars = kTcStages * kStageBytes;
 // barriers: full[S], empty[S], tfull[2], tempty[2]
 constexpr int kNumBars = 2 * kTcStages + 4;
 constexpr int kOffMisc = kOffBars + kNumBars * 8;   // tmem base, abort flag
-constexpr int kSmemBytes = kOffMisc + 16 + 1024;    // + alignment slack
+constexpr int kCuqCache = 1024;                      // cu_q entries staged in shared memory
+constexpr int kOffCuq = kOffMisc + 16;
+// + alignment slack; at least 116 KiB so that two CTAs never share an SM (each
+// holds all 512 tensor-memory columns)
+constexpr int kSmemBytes = (kOffCuq + kCuqCache * 4 + 1024) > 116 * 1024 ? (kOffCuq + kCuqCache * 4 + 1024)
+                                                                           : 116 * 1024;
 constexpr int kFullCount = 33;                       // 32 cp.async arrivals + the info arrival
 constexpr int kEmptyCount = 1 + 4;                   // MMA commit + 4 epilogue warps
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
@@ -112,38 +117,69 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
 
     if (warp == 0) {
         // ============================================================ loader
+        // Global loads for tile it+1 (query positions, head weights, the first
+        // sequence's length) are issued while tile it is published, so the
+        // loop never waits on them.  A tile whose (sequence, block tile) is the
+        // previous one's copies the previous stage's coarse keys on chip.
         if (lane == 0) prefetch_tensormap(&tm_q);
-        pdl_wait();   // coarse keys may come from the preceding append
-        int k = 0;   // sub-items published
-        uint32_t err_bits = 0;
-        for (long long it = i0; it <= i1 && !*s_abort; ++it) {
-            const bool end = it == i1;
-            const int bt = end ? 0 : (int)(it / n_qt), y = end ? 0 : (int)(it % n_qt);
-            const int t0 = kQT * y;
-            // sequences touched by the tile's queries
-            int s_lo = 0, s_hi = -1;
-            if (!end && t0 < a.total_q) {
-                s_lo = seq_of_query(a, t0);
-                s_hi = seq_of_query(a, min(t0 + kQT, a.total_q) - 1);
+        int *s_cuq = reinterpret_cast<int *>(g + kOffCuq);
+        const bool cuq_cached = a.num_seqs + 1 <= kCuqCache;
+        if (cuq_cached)
+            for (int i = lane; i <= a.num_seqs; i += 32) s_cuq[i] = __ldg(a.cu_q + i);
+        __syncwarp();
+        auto seq_of = [&](int t) {
+            if (!cuq_cached) return seq_of_query(a, t);
+            int lo = 0, hi = a.num_seqs - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (s_cuq[mid] <= t) lo = mid; else hi = mid - 1;
             }
-            for (int s = s_lo; end ? (s == s_lo) : (s <= s_hi); ++s) {
-                // own blocks of the tile's queries in s (-1: not in s or invalid)
+            return lo;
+        };
+        auto cu = [&](int s) { return cuq_cached ? s_cuq[s] : __ldg(a.cu_q + s); };
+        // per-tile prefetch: lane l holds the position of query t0 + (l % 16)
+        // and weights e = l + 32 j (query e / 16, head e % 16)
+        struct Pre {
+            int pos, len_lo, s_lo, s_hi;
+            int wv[8];
+        };
+        auto prefetch = [&](long long it, Pre &pr) {
+            const int y = (int)(it % n_qt), t0 = kQT * y;
+            const int t = t0 + (lane & (kQT - 1));
+            pr.pos = t < a.total_q ? __ldg(a.q_pos + t) : -1;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int e = lane + 32 * j, qi = e / kMaxIdxHeads, h = e % kMaxIdxHeads;
+                pr.wv[j] = (t0 + qi < a.total_q && h < H) ? __ldg(a.w + (size_t)(t0 + qi) * H + h) : 0;
+            }
+            pr.s_lo = seq_of(t0);
+            pr.s_hi = seq_of(min(t0 + kQT, a.total_q) - 1);
+            pr.len_lo = __ldg(a.seq_lens + pr.s_lo);
+        };
+        pdl_wait();   // coarse keys may come from the preceding append
+        int k = 0;    // stages published
+        int prev_s = -1, prev_bt = -1;
+        uint32_t err_bits = 0;
+        Pre nxt;
+        if (i0 < i1) prefetch(i0, nxt);
+        for (long long it = i0; it < i1 && !*s_abort; ++it) {
+            const Pre cur = nxt;
+            if (it + 1 < i1) prefetch(it + 1, nxt);
+            const int bt = (int)(it / n_qt), y = (int)(it % n_qt);
+            const int t0 = kQT * y;
+            for (int s = cur.s_lo; s <= cur.s_hi; ++s) {
+                const int len = s == cur.s_lo ? cur.len_lo : __ldg(a.seq_lens + s);
+                const int t = t0 + (lane & (kQT - 1));
                 int own = -1;
-                int len = 0;
-                if (!end) {
-                    len = __ldg(a.seq_lens + s);
-                    const int t = t0 + (lane & (kQT - 1));
-                    if (t < a.total_q && __ldg(a.cu_q + s) <= t && t < __ldg(a.cu_q + s + 1)) {
-                        const int p = __ldg(a.q_pos + t);
-                        own = p / kBlockSize;
-                        if (p < 0 || p >= len || own >= a.max_blocks) {
-                            err_bits |= DSA_DEV_ERR_POS;
-                            own = -1;
-                        }
+                if (t < a.total_q && cu(s) <= t && t < cu(s + 1)) {
+                    own = cur.pos / kBlockSize;
+                    if (cur.pos < 0 || cur.pos >= len || own >= a.max_blocks) {
+                        err_bits |= DSA_DEV_ERR_POS;
+                        own = -1;
                     }
                 }
                 const int max_own = __reduce_max_sync(0xffffffffu, own);
-                if (!end && max_own < bt * kBT) continue;   // nothing visible in this tile
+                if (max_own < bt * kBT) continue;   // nothing visible in this tile
                 const int st = k % kTcStages;
                 if (k >= kTcStages && !mbar_wait(bars.empty(st), ((k / kTcStages) - 1) & 1, s_abort)) {
                     *s_abort = 1;
@@ -152,25 +188,30 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
                 uint8_t *stage = g + st * kStageBytes;
                 StageInfo *info = reinterpret_cast<StageInfo *>(stage + kOffInfo);
                 const uint32_t sa = base + st * kStageBytes;
-                if (end) {
-                    if (lane == 0) { info->end = 1; info->s = -1; }
-                } else {
-                    if (lane == 0) { info->end = 0; info->s = s; info->bt = bt; info->y = y; }
-                    if (lane < kQT) info->own[lane] = own;
-                    // weights of the tile's queries (0 for masked queries and heads past H)
-                    for (int e = lane; e < kQT * kMaxIdxHeads; e += 32) {
-                        const int qi = e / kMaxIdxHeads, h = e % kMaxIdxHeads;
-                        const int oq = __shfl_sync(0xffffffffu, own, qi);
-                        info->w[qi][h] = (oq >= 0 && h < H) ? __ldg(a.w + (size_t)(t0 + qi) * H + h) : 0;
+                if (lane == 0) { info->end = 0; info->s = s; info->bt = bt; info->y = y; }
+                if (lane < kQT) info->own[lane] = own;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) (&info->w[0][0])[lane + 32 * j] = cur.wv[j];
+                if (s == prev_s && bt == prev_bt) {
+                    // same coarse keys as the previous stage: copy them on chip
+                    // (that stage's own copies have landed: waited below)
+                    const uint8_t *src = g + ((k - 1) % kTcStages) * kStageBytes;
+                    const StageInfo *pinfo = reinterpret_cast<const StageInfo *>(src + kOffInfo);
+#pragma unroll
+                    for (int j = 0; j < kABytes / 16 / 32; ++j) {
+                        const int e = lane + 32 * j;
+                        reinterpret_cast<int4 *>(stage)[e] = reinterpret_cast<const int4 *>(src)[e];
                     }
-                    // the 128 coarse keys: 4 rows per lane, 4 x 16 B per row, swizzled
+                    if (lane < kBT / 32) info->valid[lane] = pinfo->valid[lane];
+                } else {
+                    // gather the 128 coarse keys: 4 rows per lane, 4 x 16 B per row, swizzled
                     const int n_blocks = (len + kBlockSize - 1) / kBlockSize;
 #pragma unroll
                     for (int r4 = 0; r4 < kBT / 32; ++r4) {
                         const int r = r4 * 32 + lane;
                         const int b = bt * kBT + r;
                         int page = -1;
-                        if (b < n_blocks && b < a.max_blocks && b <= max_own) {
+                        if (b < n_blocks && b < a.max_blocks) {
                             page = __ldg(a.block_table + (size_t)s * a.max_blocks + b);
                             if (page < 0 || page >= a.num_pages) {
                                 err_bits |= DSA_DEV_ERR_PAGE;
@@ -187,22 +228,40 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
                             else cp_async_16_zero(dst, a.kc_pool);
                         }
                     }
-                    // the queries' rows: box (64 B, 16 heads, 16 queries) at query t0
-                    if (lane == 0) {
-                        tc::mbar_expect_tx(bars.full(st), kBBytes);
-                        tma_load_3d(sa + kOffB, &tm_q, 0, 0, t0, bars.full(st));
-                    }
+                    prev_s = s;
+                    prev_bt = bt;
+                }
+                // the queries' rows: box (64 B, 16 heads, 16 queries) at query t0
+                if (lane == 0) {
+                    tc::mbar_expect_tx(bars.full(st), kBBytes);
+                    tma_load_3d(sa + kOffB, &tm_q, 0, 0, t0, bars.full(st));
                 }
                 tc::cp_async_arrive_noinc(bars.full(st));
+                // the next stage may copy this one's keys: let them land first
+                cp_async_commit();
+                cp_async_wait<0>();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bars.full(st));   // the info words above
+                if (lane == 0) mbar_arrive(bars.full(st));   // the info words and copies above
                 ++k;
-                if (end) break;
+            }
+        }
+        // the end marker
+        if (!*s_abort) {
+            const int st = k % kTcStages;
+            if (k >= kTcStages && !mbar_wait(bars.empty(st), ((k / kTcStages) - 1) & 1, s_abort)) {
+                *s_abort = 1;
+            } else {
+                StageInfo *info = reinterpret_cast<StageInfo *>(g + st * kStageBytes + kOffInfo);
+                if (lane == 0) { info->end = 1; info->s = -1; }
+                tc::cp_async_arrive_noinc(bars.full(st));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars.full(st));
+                ++k;
             }
         }
         err_bits = __reduce_or_sync(0xffffffffu, err_bits);
         if (lane == 0 && err_bits) set_err(a.dev_err, err_bits);
-        // nothing may still be landing when the CTA winds down
+        cp_async_commit();
         cp_async_wait<0>();
         if (*s_abort && lane == 0) {
             set_err(a.dev_err, DSA_DEV_ERR_WAIT);
@@ -268,22 +327,24 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
             const bool row_ok = (info->valid[row >> 5] >> (row & 31)) & 1u;
             const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kN);
 #pragma unroll 1
-            for (int j = 0; j < kQT / 2; ++j) {
-                uint32_t v[32];
-                tc::ld_32x32b_x32(taddr + 32 * j, v);
+            for (int j = 0; j < kQT / 4; ++j) {   // four queries (64 columns) per wait
+                uint32_t v[2][32];
+                tc::ld_32x32b_x32(taddr + 64 * j, v[0]);
+                tc::ld_32x32b_x32(taddr + 64 * j + 32, v[1]);
                 tc::wait_ld();
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int qi = 2 * j + u;
+                for (int u = 0; u < 4; ++u) {
+                    const int qi = 4 * j + u;
                     const int4 *wq = reinterpret_cast<const int4 *>(info->w[qi]);
+                    const uint32_t *x = v[u >> 1] + 16 * (u & 1);
                     int sum = 0;
 #pragma unroll
                     for (int h4 = 0; h4 < 4; ++h4) {
                         const int4 wv = wq[h4];
-                        sum += wv.x * max((int)v[16 * u + 4 * h4 + 0], 0);
-                        sum += wv.y * max((int)v[16 * u + 4 * h4 + 1], 0);
-                        sum += wv.z * max((int)v[16 * u + 4 * h4 + 2], 0);
-                        sum += wv.w * max((int)v[16 * u + 4 * h4 + 3], 0);
+                        sum += wv.x * max((int)x[4 * h4 + 0], 0);
+                        sum += wv.y * max((int)x[4 * h4 + 1], 0);
+                        sum += wv.z * max((int)x[4 * h4 + 2], 0);
+                        sum += wv.w * max((int)x[4 * h4 + 3], 0);
                     }
                     if (row_ok && b <= info->own[qi]) a.scores[(size_t)(kQT * y + qi) * a.max_blocks + b] = sum;
                 }

@@ -148,9 +148,7 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
         } else if (gi == 0) {
             pdl_wait();
         }
-        warp_sort64_desc(v);
-        if (gi == 0) { acc[0] = v[0]; acc[1] = v[1]; }
-        else warp_merge64_desc(acc, v);
+        warp_fold_topk(acc, v, kk);
     }
     if (err_bits) set_err(a.dev_err, err_bits);
 

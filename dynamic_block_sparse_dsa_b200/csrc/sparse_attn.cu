@@ -114,7 +114,7 @@ __device__ __forceinline__ int seq_of(const AttnArgs &a, const int *s_cuq, int t
 }  // namespace
 
 // NT: query-head n-tiles of 8 (the GQA group is <= 8 * NT).  kFused: the
-// single-launch decode step -- phases A (append) and B (select) of
+// single-launch decode step -- the select and append phases of
 // decode_fused.cuh run first, and the producer waits for each query's
 // selection before reading it.
 template <int NT, bool kFused>
@@ -160,7 +160,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     __syncthreads();
     const int tag = W[kWTag];
     if constexpr (kFused) {
-        fused::append_and_select(a, f, gbase, tag, W + kWSelLast);
+        fused::select_blocks_phase(a, f, gbase, tag, W + kWSelLast);
+        fused::append_tokens(a, f);
         // the ring's generic-proxy use ends before TMA writes into it
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncthreads();

@@ -85,6 +85,23 @@ __device__ __forceinline__ void warp_merge64_desc(key64 (&a)[2], const key64 (&b
     warp_bitonic_merge64_desc(a);
 }
 
+// Fold a batch of 64 keys (any order, zeros for empty slots) into a running
+// descending list whose first kk (1..63) entries are the kk largest keys seen
+// so far.  Keys not above the current kk-th largest can never reach those kk,
+// so they are dropped first; a batch with none left costs one vote, which is
+// the common case once the list has filled (the entries past kk are then only
+// a partial record and must not be used).
+__device__ __forceinline__ void warp_fold_topk(key64 (&acc)[2], key64 (&v)[2], int kk) {
+    const int i = kk - 1;
+    const key64 thr = __shfl_sync(0xffffffffu, i < 32 ? acc[0] : acc[1], i & 31);
+    const bool p0 = v[0] > thr, p1 = v[1] > thr;
+    if (!__any_sync(0xffffffffu, p0 || p1)) return;
+    v[0] = p0 ? v[0] : 0ull;
+    v[1] = p1 ? v[1] : 0ull;
+    warp_sort64_desc(v);
+    warp_merge64_desc(acc, v);
+}
+
 // sort 64 unsigned 32-bit values ascending (used to order selected block ids)
 __device__ __forceinline__ void warp_sort64_asc_u32(uint32_t (&v)[2]) {
     const int lane = threadIdx.x & 31;
