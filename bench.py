@@ -194,6 +194,11 @@ def run_ours(args, world, rank, device):
     flush_rd = torch.ones(L2_FLUSH_BYTES // 2 // 4, dtype=torch.int32, device=device)
 
     def front(b):
+        if fused and decode:   # a decode batch: the append may overlap the selection
+            dsa.select_blocks_append(cache, seqs, queries, queries.cu_q, wl.k_new, wl.v_new, wl.kc_new, wl.q_idx,
+                                     wl.w, wl.k_per_seq, spec.k_max, 16, sel=b["sel"], cnt=b["cnt"],
+                                     workspace=b["select_ws"], dev_err=err)
+            return
         dsa.kv_append(cache, seqs, queries.cu_q, wl.k_new, wl.v_new, wl.kc_new, dev_err=err)
         if fused:
             dsa.select_blocks(cache, seqs, queries, wl.q_idx, wl.w, wl.k_per_seq, spec.k_max, 16, sel=b["sel"],
@@ -219,7 +224,8 @@ def run_ours(args, world, rank, device):
     with torch.cuda.stream(stream):
         bufs = dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
                         q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=spec.k_max, decode=decode,
-                        fused_select=fused, fused_decode=fused_decode, dev_err=err)
+                        fused_select=fused, overlap_append=fused and decode, fused_decode=fused_decode,
+                        dev_err=err)
     torch.cuda.synchronize(device)
     if int(err.item()) != 0:
         raise RuntimeError(f"device error bits {int(err.item())} in the first step")
@@ -316,7 +322,8 @@ def run_ours(args, world, rank, device):
                 dev_in[k].copy_(t, non_blocking=True)
             dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
                      q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=spec.k_max, decode=decode,
-                     fused_select=fused, fused_decode=fused_decode, bufs=bufs, dev_err=err)
+                     fused_select=fused, overlap_append=fused and decode, fused_decode=fused_decode,
+                     bufs=bufs, dev_err=err)
             host_out.copy_(bufs["out"], non_blocking=True)
             host_lse.copy_(bufs["lse"], non_blocking=True)
             e_e.record()
@@ -339,7 +346,7 @@ def run_ours(args, world, rank, device):
                    "l2": "cold before every timed step: 512 MiB written, then 256 MiB read (no dirty lines)",
                    "graph": "one CUDA graph per step" + ("" if fused_decode else " (PDL between kernels)"),
                    "path": {"fused_decode": "single launch: append + fused score/Top-K + attention",
-                            "fused_select": "kv_append, fused score+Top-K, attention",
+                            "fused_select": "fused score+Top-K with the token append overlapping it, attention",
                             "score_topk": "kv_append, index_score, topk_blocks, attention"}[path]},
         "roofline": roofline,
         "step_roofline": step_roof,
@@ -350,6 +357,53 @@ def run_ours(args, world, rank, device):
         "clocks": clk.summary(),
     }
     return res, wl
+
+
+# ----------------------------------------------------------------------------- prefill indexer
+def prefill_indexer(device, seed=1004, iters=20):
+    """The prefill indexer contraction (dsa_index_score on the 4096-query chunk
+    after a 128K prefix) timed alone with a cold L2, against the int8 tensor
+    roofline: ops = causal (query, block) pairs x 16 heads x 64 x 2."""
+    import dynamic_block_sparse_dsa_b200 as dsa
+    from dynamic_block_sparse_dsa_b200 import workloads as wk
+    spec = wk.chunked_prefill()
+    wl = wk.make_workload(spec, seed=seed, device=device)
+    cache = dsa.PagedKVCache(wl.k_pool, wl.v_pool, wl.kc_pool)
+    seqs = dsa.SeqBatch(wl.block_table, wl.seq_lens)
+    queries = dsa.QueryBatch(wl.cu_q, wl.q_pos)
+    err = torch.zeros(1, dtype=torch.int32, device=device)
+    scores = torch.empty((spec.total_q, wl.block_table.shape[1]), dtype=torch.int32, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 2 // 4, dtype=torch.int32, device=device)
+    stream = torch.cuda.Stream(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pos = wl.q_pos.cpu()
+    pairs = int(((pos // spec.block_size) + 1).sum())
+    ops = pairs * spec.num_idx_heads * spec.idx_dim * 2
+    ms = []
+    with torch.cuda.stream(stream):
+        for i in range(iters + 3):
+            flush.fill_(1)
+            flush_rd.sum(dtype=torch.int32)
+            e0.record()
+            dsa.index_score(cache, seqs, queries, wl.q_idx, wl.w, 16, scores=scores, dev_err=err)
+            e1.record()
+            stream.synchronize()
+            if i >= 3:
+                ms.append(e0.elapsed_time(e1))
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(err.item())} in the prefill indexer")
+    t = statistics.median(ms) * 1e-3
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak = 2.0 * float(json.load(f)["bf16_tflops"])
+        src = "measured bf16 burst x 2 (nominal int8/bf16 ratio)"
+    except Exception:
+        peak, src = 2.0 * 1590.0, "fallback bf16 x 2"
+    tops = ops / t / 1e12
+    return {"workload": spec.name, "kernel": "index_score_tc_kernel (tcgen05 kind::i8)", "us": round(t * 1e6, 2),
+            "int8_ops": ops, "achieved": round(tops, 1), "peak": round(peak, 1), "unit": "TOPS",
+            "frac": round(tops / peak, 4), "peak_source": src, "l2": "cold before every launch"}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) arm
@@ -400,6 +454,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="decode_1m")
     ap.add_argument("--seed", type=int, default=1003)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-indexer measurement")
     ap.add_argument("--path", choices=["auto", "fused_decode", "fused_select", "score_topk"], default="auto",
                     help="decode step as one launch, or as the chain of separate calls")
     args = ap.parse_args(argv)
@@ -422,6 +477,8 @@ def main(argv=None):
 
     init_dist(world, "nccl")
     res, wl = run_ours(args, world, rank, device)
+    if rank == 0 and not args.no_prefill:
+        res["prefill_indexer"] = prefill_indexer(device)
     if rank == 0 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:

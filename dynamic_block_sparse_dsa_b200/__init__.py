@@ -186,6 +186,36 @@ def select_blocks(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, q_id
     return sel, cnt
 
 
+def select_blocks_append(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, cu_new: torch.Tensor,
+                         k_new: torch.Tensor, v_new: torch.Tensor, kc_new: Optional[torch.Tensor],
+                         q_idx: torch.Tensor, w: torch.Tensor, k_per_seq: torch.Tensor, k_max: int,
+                         w_abs_max: int = 16, sel: Optional[torch.Tensor] = None, cnt: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+                         stream=None):
+    """select_blocks then kv_append for a decode batch, the copies overlapping
+    the selection: (sel, cnt).  Queries whose sequence appends a block before
+    their own block are refused (DEV_ERR_POS, cnt 0)."""
+    lib = load()
+    _expect(q_idx, torch.int8, "q_idx")
+    _expect(w, torch.int32, "w")
+    _expect(k_new, torch.bfloat16, "k_new")
+    _expect(v_new, torch.bfloat16, "v_new")
+    dev = q_idx.device
+    T = queries.total_q
+    if sel is None:
+        sel = torch.empty((T, k_max), dtype=torch.int32, device=dev)
+    if cnt is None:
+        cnt = torch.empty((T,), dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = torch.zeros(select_workspace_size(T), dtype=torch.uint8, device=dev)
+    c, s, q = cache.ctype(), seqs.ctype(), queries.ctype()
+    _lib.check("dsa_select_blocks_append", lib.dsa_select_blocks_append(
+        ctypes.byref(c), ctypes.byref(s), ctypes.byref(q), _ptr(cu_new), k_new.shape[0], _ptr(k_new), _ptr(v_new),
+        _ptr(kc_new), _ptr(q_idx), _ptr(w), q_idx.shape[1], int(w_abs_max), _ptr(k_per_seq), int(k_max), _ptr(sel),
+        _ptr(cnt), _ptr(workspace), workspace.numel(), _ptr(dev_err), _stream(stream)))
+    return sel, cnt
+
+
 def decode_workspace_size(total_q: int, num_q_heads: int, num_kv_heads: int, k_max: int) -> int:
     return int(load().dsa_sparse_attn_decode_workspace_size(total_q, num_q_heads, num_kv_heads, k_max))
 
@@ -297,11 +327,13 @@ def decode_fused(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, cu_ne
 
 def step(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, *, k_new, v_new, kc_new, q, q_idx, w,
          k_per_seq, k_max: int, w_abs_max: int = 16, decode: bool = True, fused_select: bool = False,
-         fused_decode: bool = False, bufs: Optional[dict] = None, dev_err: Optional[torch.Tensor] = None,
-         stream=None):
+         overlap_append: bool = False, fused_decode: bool = False, bufs: Optional[dict] = None,
+         dev_err: Optional[torch.Tensor] = None, stream=None):
     """One pass of the hot path: append -> index_score -> topk_blocks -> attention
     (with ``fused_select`` the middle two are the single select_blocks call;
-    with ``fused_decode`` the whole decode step is one decode_fused launch).
+    with ``overlap_append`` as well -- decode batches only -- the append runs
+    as select_blocks_append, overlapping the selection; with ``fused_decode``
+    the whole decode step is one decode_fused launch).
 
     ``bufs`` (optional, reused across calls) holds the scores / sel / cnt /
     out / lse / workspace tensors; missing ones are allocated.  Returns bufs.
@@ -326,6 +358,14 @@ def step(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, *, k_new, v_n
         decode_fused(cache, seqs, queries, queries.cu_q, k_new, v_new, kc_new, q_idx, w, k_per_seq, k_max, q,
                      w_abs_max, sel=b["sel"], cnt=b["cnt"], out=b["out"], lse=b["lse"], workspace=b["fused_ws"],
                      dev_err=dev_err, stream=stream)
+        return b
+    if fused_select and overlap_append:
+        # decode batches: the token copies overlap the selection, which never reads them
+        select_blocks_append(cache, seqs, queries, queries.cu_q, k_new, v_new, kc_new, q_idx, w, k_per_seq, k_max,
+                             w_abs_max, sel=b["sel"], cnt=b["cnt"], workspace=b["select_ws"], dev_err=dev_err,
+                             stream=stream)
+        sparse_attn_decode(cache, seqs, queries, q, b["sel"], b["cnt"], out=b["out"], lse=b["lse"],
+                           workspace=b["workspace"], dev_err=dev_err, stream=stream)
         return b
     kv_append(cache, seqs, queries.cu_q, k_new, v_new, kc_new, dev_err=dev_err, stream=stream)
     if fused_select:

@@ -46,6 +46,8 @@ SIGNATURES = {
     "dsa_select_blocks_workspace_size": ([c_i32], ctypes.c_size_t),
     "dsa_select_blocks": ([P(KvCacheC), P(SeqsC), P(QueriesC), c_vp, c_vp, c_i32, c_i32, c_vp, c_i32, c_vp, c_vp,
                            c_vp, ctypes.c_size_t, c_vp, c_vp], c_i32),
+    "dsa_select_blocks_append": ([P(KvCacheC), P(SeqsC), P(QueriesC), c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                  c_i32, c_i32, c_vp, c_i32, c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp, c_vp], c_i32),
     "dsa_sparse_attn_decode_workspace_size": ([c_i32, c_i32, c_i32, c_i32], ctypes.c_size_t),
     "dsa_sparse_attn_decode": ([P(KvCacheC), P(SeqsC), P(QueriesC), c_vp, c_i32, c_vp, c_vp, c_i32,
                                 ctypes.c_float, c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp, c_vp], c_i32),

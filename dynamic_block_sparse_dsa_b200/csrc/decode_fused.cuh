@@ -78,13 +78,15 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// wait until *p == v (acquire); false on timeout
+// wait until *p == v (acquire); false on timeout.  Polls back off so that a
+// grid of waiters does not crowd out the stores they wait for.
 __device__ __forceinline__ bool wait_flag(const int32_t *p, int v) {
     if (ld_acquire(p) == v) return true;
     const long long t0 = clock64();
 #pragma unroll 1
     while (ld_acquire(p) != v) {
         if (clock64() - t0 > kWaitLimitCycles) return false;
+        __nanosleep(128);
     }
     return true;
 }

@@ -89,11 +89,20 @@ FusedLayout fused_layout(int total_q, int hq, int hkv) {
 
 // grid of the persistent attention kernel: one CTA per SM, never more CTAs
 // than work items so that every CTA owns a non-empty range
-void attn_schedule(AttnArgs &a, bool allow_split) {
+void attn_schedule(AttnArgs &a, bool allow_split, bool allow_cluster = false) {
     const long long pairs = (long long)a.total_q * a.num_kv_heads;
     a.total_units = pairs * a.k_max;
     long long C = sm_count();
     if (C > kAttnMaxCtas) C = kAttnMaxCtas;
+    a.cluster2 = 0;
+    // between a quarter and a half as many pairs as SMs: one 2-CTA cluster per
+    // pair keeps at least half of the SMs streaming and merges on chip
+    if (allow_cluster && allow_split && a.k_max >= 2 && 4 * pairs >= C && 2 * pairs <= C) {
+        a.cluster2 = 1;
+        a.pair_aligned = 0;
+        a.num_ctas = (int)(2 * pairs);
+        return;
+    }
     // whole (query, KV head) pairs per CTA when there are plenty of them (or
     // when no workspace is available); otherwise split pairs across CTAs
     a.pair_aligned = (!allow_split || pairs >= 16 * C) ? 1 : 0;
@@ -144,6 +153,11 @@ int attn_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queri
     a.dev_err = dev_err;
     return DSA_OK;
 }
+
+int select_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                  const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads, int32_t w_abs_max,
+                  const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt, void *workspace,
+                  size_t workspace_bytes, const int32_t *cu_new, int32_t *dev_err, dsa_stream_t stream);
 
 }  // namespace
 
@@ -259,6 +273,53 @@ int dsa_select_blocks(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa
                       const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads, int32_t w_abs_max,
                       const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt, void *workspace,
                       size_t workspace_bytes, int32_t *dev_err, dsa_stream_t stream) {
+    return select_common(cache, seqs, queries, q_idx, w, num_idx_heads, w_abs_max, k_per_seq, k_max, sel, cnt,
+                         workspace, workspace_bytes, nullptr, dev_err, stream);
+}
+
+int dsa_select_blocks_append(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                             const int32_t *cu_new, int32_t total_new, const void *k_new, const void *v_new,
+                             const int8_t *kc_new, const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads,
+                             int32_t w_abs_max, const int32_t *k_per_seq, int32_t k_max, int32_t *sel,
+                             int32_t *cnt, void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                             dsa_stream_t stream) {
+    int rc;
+    if ((rc = check_cache(cache)) || (rc = check_seqs(seqs))) return rc;
+    if (total_new < 0) return DSA_ERR_INVALID_ARG;
+    if (total_new > 0) {
+        if (!cu_new || !k_new || !v_new) return DSA_ERR_INVALID_ARG;
+        if (!aligned16(k_new) || !aligned16(v_new) || (kc_new && !aligned16(kc_new))) return DSA_ERR_INVALID_ARG;
+    }
+    rc = select_common(cache, seqs, queries, q_idx, w, num_idx_heads, w_abs_max, k_per_seq, k_max, sel, cnt,
+                       workspace, workspace_bytes, total_new > 0 ? cu_new : nullptr, dev_err, stream);
+    if (rc || total_new == 0) return rc;
+    KvAppendArgs a{};
+    a.k_pool = cache->k_pool;
+    a.v_pool = cache->v_pool;
+    a.kc_pool = cache->kc_pool;
+    a.num_pages = cache->num_pages;
+    a.num_kv_heads = cache->num_kv_heads;
+    a.block_table = seqs->block_table;
+    a.max_blocks = seqs->max_blocks;
+    a.seq_lens = seqs->seq_lens;
+    a.num_seqs = seqs->num_seqs;
+    a.cu_new = cu_new;
+    a.total_new = total_new;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.kc_new = kc_new;
+    a.dev_err = dev_err;
+    a.overlap_prev = queries->total_q > 0 ? 1 : 0;   // nothing launched before it when there are no queries
+    return from_cuda(launch_kv_append(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
+
+namespace {
+int select_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                  const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads, int32_t w_abs_max,
+                  const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt, void *workspace,
+                  size_t workspace_bytes, const int32_t *cu_new, int32_t *dev_err, dsa_stream_t stream) {
     int rc;
     if ((rc = check_cache(cache)) || (rc = check_seqs(seqs)) || (rc = check_queries(queries))) return rc;
     if (num_idx_heads < 1 || w_abs_max < 0 || k_max < 1) return DSA_ERR_INVALID_ARG;
@@ -291,8 +352,12 @@ int dsa_select_blocks(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa
     a.counters = reinterpret_cast<int32_t *>(ws + L.counters);
     a.cand = reinterpret_cast<unsigned long long *>(ws + L.cand);
     a.dev_err = dev_err;
+    a.cu_new = cu_new;
     return from_cuda(launch_select_blocks(a, reinterpret_cast<cudaStream_t>(stream)));
 }
+}  // namespace
+
+extern "C" {
 
 size_t dsa_sparse_attn_decode_workspace_size(int32_t total_q, int32_t num_q_heads, int32_t num_kv_heads,
                                              int32_t k_max) {
@@ -314,7 +379,7 @@ int dsa_sparse_attn_decode(const dsa_kv_cache *cache, const dsa_seqs *seqs, cons
     char *ws = static_cast<char *>(workspace);
     a.counters = reinterpret_cast<int32_t *>(ws + L.counters);
     a.part = reinterpret_cast<float *>(ws + L.part);
-    attn_schedule(a, true);
+    attn_schedule(a, true, true);
     return from_cuda(launch_sparse_attn(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -34,6 +34,12 @@ struct KvAppendArgs {
     const void *k_new, *v_new;
     const int8_t *kc_new;
     int32_t *dev_err;
+    // 0: an ordinary launch (waits for everything before it).  1: launched
+    // as a programmatic dependent of a selection kernel that reads none of
+    // the rows written here -- the copies overlap it, and the kernel waits
+    // for it only before exiting, so whatever waits for the append also
+    // waits for the selection.
+    int overlap_prev;
 };
 
 struct IndexScoreArgs {
@@ -91,6 +97,11 @@ struct SelectArgs {
     unsigned long long *cand;   // [T][kSelMaxChunks][kSelMaxK-1] 64-bit selection keys, sorted descending
     int32_t *counters;       // [T] chunk CTAs done per query
     int32_t *dev_err;
+    // append ordered after this selection (dsa_select_blocks_append): a
+    // query whose sequence appends a block before its own block is refused
+    // (DSA_DEV_ERR_POS, cnt 0) -- the selection must not read those keys; and
+    // the kernel is launched after everything before it has completed
+    const int32_t *cu_new;   // null: no append follows
 };
 
 struct AttnArgs {
@@ -118,6 +129,10 @@ struct AttnArgs {
     long long total_units;   // U
     int num_ctas;            // C (= gridDim.x)
     int pair_aligned;
+    // 1: pair p is run by the 2-CTA cluster (2p, 2p+1), each CTA taking half
+    // of its units; the halves merge through distributed shared memory and
+    // no workspace is touched
+    int cluster2;
     float *part;             // [2*C][group][kAttnPartStride] partial (o[128], m, l) of split pairs
     int32_t *counters;       // [T*Hkv] units merged so far per split pair
     int32_t *dev_err;

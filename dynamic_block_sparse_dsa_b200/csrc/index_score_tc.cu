@@ -16,24 +16,30 @@
 // head weights and head sum then happen in the epilogue, one block row per
 // thread, straight from tensor memory.  One persistent CTA per SM, 6 warps:
 //   warp 0   loader: the tile's 128 coarse keys gathered through the block
-//            table (cp.async, 64-byte swizzle) and the 16 queries' rows
-//            (one 3-D TMA box, heads past H zero-filled), plus the queries'
-//            own blocks and weights, into a 4-stage ring;
+//            table (cp.async, 64-byte swizzle; the page ids themselves
+//            copied a few tiles ahead) and the 16 queries' rows (one 3-D TMA
+//            box, heads past H zero-filled), plus the queries' own blocks and
+//            weights, into a 4-stage ring;
 //   warp 1   MMA issuer (one thread): two K=32 MMAs per tile into one of two
 //            256-column accumulators;
-//   warps 2-5 epilogue: tcgen05.ld of the accumulator rows, relu * w summed
-//            over heads, one coalesced 128-byte store per (query, warp).
-// Tiles are (128-block tile, 16-query tile) pairs in block-tile-major order,
+//   warps 2-9 epilogue (two per SM sub-partition: a quarter of the rows and
+//            half of the queries each): tcgen05.ld of the accumulator rows,
+//            relu * w summed over heads, one coalesced 128-byte store per
+//            (query, warp).
+// Tiles are (16-query tile, 128-block tile) pairs in query-tile-major order,
 // split evenly over the CTAs; a tile whose queries belong to several
 // sequences is run once per sequence with the other queries masked.  Tiles
 // past every query's own block are skipped.  All waits are bounded.
+#include <cstddef>
+
 #include "dsa_kernels.h"
 #include "dsa_tcgen05.cuh"
 
 namespace dsa {
 
 namespace {
-constexpr int kTcThreads = 192;
+constexpr int kEpiWarps = 8;                       // two per SM sub-partition
+constexpr int kTcThreads = 64 + 32 * kEpiWarps;   // loader, MMA, epilogue
 constexpr int kTcStages = 4;
 constexpr int kBT = 128;                 // blocks per tile (MMA M)
 constexpr int kQT = 16;                  // queries per tile (MMA N = 16 x 16 heads)
@@ -56,12 +62,14 @@ constexpr int kNumBars = 2 * kTcStages + 4;
 constexpr int kOffMisc = kOffBars + kNumBars * 8;   // tmem base, abort flag
 constexpr int kCuqCache = 1024;                      // cu_q entries staged in shared memory
 constexpr int kOffCuq = kOffMisc + 16;
+constexpr int kPidDepth = 4;                         // block tiles of page ids in flight
+constexpr int kOffPid = kOffCuq + kCuqCache * 4;     // [kPidDepth][kBT] int32
 // + alignment slack; at least 116 KiB so that two CTAs never share an SM (each
 // holds all 512 tensor-memory columns)
-constexpr int kSmemBytes = (kOffCuq + kCuqCache * 4 + 1024) > 116 * 1024 ? (kOffCuq + kCuqCache * 4 + 1024)
-                                                                           : 116 * 1024;
+constexpr int kSmemUsed = kOffPid + kPidDepth * kBT * 4 + 1024;
+constexpr int kSmemBytes = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
 constexpr int kFullCount = 33;                       // 32 cp.async arrivals + the info arrival
-constexpr int kEmptyCount = 1 + 4;                   // MMA commit + 4 epilogue warps
+constexpr int kEmptyCount = 1 + kEpiWarps;           // MMA commit + the epilogue warps
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
@@ -95,7 +103,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bars.tfull(b), 1);
-            mbar_init(bars.tempty(b), 4);
+            mbar_init(bars.tempty(b), kEpiWarps);
         }
         misc[1] = 0;
         misc[2] = 0;
@@ -117,12 +125,15 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
 
     if (warp == 0) {
         // ============================================================ loader
-        // Global loads for tile it+1 (query positions, head weights, the first
-        // sequence's length) are issued while tile it is published, so the
-        // loop never waits on them.  A tile whose (sequence, block tile) is the
-        // previous one's copies the previous stage's coarse keys on chip.
+        // Items are (query tile y, block tile bt), y-major: the queries'
+        // positions and weights change once per query tile, the coarse keys
+        // every item.  The page ids of item j are copied into a small ring
+        // kPidDepth items ahead (cp.async), so the gather of item j never
+        // waits on a global load; its keys then land through the stage's
+        // full barrier.
         if (lane == 0) prefetch_tensormap(&tm_q);
         int *s_cuq = reinterpret_cast<int *>(g + kOffCuq);
+        const int *s_pid = reinterpret_cast<const int *>(g + kOffPid);
         const bool cuq_cached = a.num_seqs + 1 <= kCuqCache;
         if (cuq_cached)
             for (int i = lane; i <= a.num_seqs; i += 32) s_cuq[i] = __ldg(a.cu_q + i);
@@ -137,43 +148,64 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
             return lo;
         };
         auto cu = [&](int s) { return cuq_cached ? s_cuq[s] : __ldg(a.cu_q + s); };
-        // per-tile prefetch: lane l holds the position of query t0 + (l % 16)
-        // and weights e = l + 32 j (query e / 16, head e % 16)
-        struct Pre {
-            int pos, len_lo, s_lo, s_hi;
-            int wv[8];
-        };
-        auto prefetch = [&](long long it, Pre &pr) {
-            const int y = (int)(it % n_qt), t0 = kQT * y;
-            const int t = t0 + (lane & (kQT - 1));
-            pr.pos = t < a.total_q ? __ldg(a.q_pos + t) : -1;
+        // page ids of item j's first sequence into ring slot j % kPidDepth
+        // (4 per lane, 4-byte copies: rows of the table need not be 16-byte aligned)
+        auto prefetch_pids = [&](long long j) {
+            const int y = (int)(j / n_bt), bt = (int)(j % n_bt);
+            const int s0 = seq_of(kQT * y);
+            const uint32_t dst = base + kOffPid + (uint32_t)((j % kPidDepth) * kBT * 4);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int e = lane + 32 * j, qi = e / kMaxIdxHeads, h = e % kMaxIdxHeads;
-                pr.wv[j] = (t0 + qi < a.total_q && h < H) ? __ldg(a.w + (size_t)(t0 + qi) * H + h) : 0;
+            for (int r4 = 0; r4 < kBT / 32; ++r4) {
+                const int r = r4 * 32 + lane, b = bt * kBT + r;
+                const int32_t *src = a.block_table + (size_t)s0 * a.max_blocks + min(b, a.max_blocks - 1);
+                if (b < a.max_blocks)
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst + 4 * r), "l"(src));
+                else
+                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, 0;\n" ::"r"(dst + 4 * r), "l"(src));
             }
-            pr.s_lo = seq_of(t0);
-            pr.s_hi = seq_of(min(t0 + kQT, a.total_q) - 1);
-            pr.len_lo = __ldg(a.seq_lens + pr.s_lo);
         };
         pdl_wait();   // coarse keys may come from the preceding append
+        for (int d = 0; d < kPidDepth; ++d) {
+            if (i0 + d < i1) prefetch_pids(i0 + d);
+            cp_async_commit();
+        }
         int k = 0;    // stages published
-        int prev_s = -1, prev_bt = -1;
+        int cur_y = -1;
+        int pos = -1, s_lo = 0, s_hi = -1, len_lo = 0;
+        int wv[8];
         uint32_t err_bits = 0;
-        Pre nxt;
-        if (i0 < i1) prefetch(i0, nxt);
         for (long long it = i0; it < i1 && !*s_abort; ++it) {
-            const Pre cur = nxt;
-            if (it + 1 < i1) prefetch(it + 1, nxt);
-            const int bt = (int)(it / n_qt), y = (int)(it % n_qt);
+            const int y = (int)(it / n_bt), bt = (int)(it % n_bt);
             const int t0 = kQT * y;
-            for (int s = cur.s_lo; s <= cur.s_hi; ++s) {
-                const int len = s == cur.s_lo ? cur.len_lo : __ldg(a.seq_lens + s);
+            if (y != cur_y) {   // a new query tile: positions, weights, sequences
+                cur_y = y;
+                const int t = t0 + (lane & (kQT - 1));
+                pos = t < a.total_q ? __ldg(a.q_pos + t) : -1;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int e = lane + 32 * j, qi = e / kMaxIdxHeads, h = e % kMaxIdxHeads;
+                    wv[j] = (t0 + qi < a.total_q && h < H) ? __ldg(a.w + (size_t)(t0 + qi) * H + h) : 0;
+                }
+                s_lo = seq_of(t0);
+                s_hi = seq_of(min(t0 + kQT, a.total_q) - 1);
+                len_lo = __ldg(a.seq_lens + s_lo);
+            }
+            // this item's page ids have landed (kPidDepth - 1 newer groups may be pending)
+            cp_async_wait<kPidDepth - 1>();
+            __syncwarp();
+            const int *pid = s_pid + (it % kPidDepth) * kBT;
+            int pg_pre[kBT / 32];
+#pragma unroll
+            for (int r4 = 0; r4 < kBT / 32; ++r4) pg_pre[r4] = pid[r4 * 32 + lane];
+            __syncwarp();   // the slot is refilled below
+            if (it + kPidDepth < i1) prefetch_pids(it + kPidDepth);
+            for (int s = s_lo; s <= s_hi && !*s_abort; ++s) {
+                const int len = s == s_lo ? len_lo : __ldg(a.seq_lens + s);
                 const int t = t0 + (lane & (kQT - 1));
                 int own = -1;
                 if (t < a.total_q && cu(s) <= t && t < cu(s + 1)) {
-                    own = cur.pos / kBlockSize;
-                    if (cur.pos < 0 || cur.pos >= len || own >= a.max_blocks) {
+                    own = pos / kBlockSize;
+                    if (pos < 0 || pos >= len || own >= a.max_blocks) {
                         err_bits |= DSA_DEV_ERR_POS;
                         own = -1;
                     }
@@ -191,45 +223,30 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
                 if (lane == 0) { info->end = 0; info->s = s; info->bt = bt; info->y = y; }
                 if (lane < kQT) info->own[lane] = own;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) (&info->w[0][0])[lane + 32 * j] = cur.wv[j];
-                if (s == prev_s && bt == prev_bt) {
-                    // same coarse keys as the previous stage: copy them on chip
-                    // (that stage's own copies have landed: waited below)
-                    const uint8_t *src = g + ((k - 1) % kTcStages) * kStageBytes;
-                    const StageInfo *pinfo = reinterpret_cast<const StageInfo *>(src + kOffInfo);
+                for (int j = 0; j < 8; ++j) (&info->w[0][0])[lane + 32 * j] = wv[j];
+                // the 128 coarse keys: 4 rows per lane, 4 x 16 B per row, swizzled
+                const int n_blocks = (len + kBlockSize - 1) / kBlockSize;
 #pragma unroll
-                    for (int j = 0; j < kABytes / 16 / 32; ++j) {
-                        const int e = lane + 32 * j;
-                        reinterpret_cast<int4 *>(stage)[e] = reinterpret_cast<const int4 *>(src)[e];
-                    }
-                    if (lane < kBT / 32) info->valid[lane] = pinfo->valid[lane];
-                } else {
-                    // gather the 128 coarse keys: 4 rows per lane, 4 x 16 B per row, swizzled
-                    const int n_blocks = (len + kBlockSize - 1) / kBlockSize;
-#pragma unroll
-                    for (int r4 = 0; r4 < kBT / 32; ++r4) {
-                        const int r = r4 * 32 + lane;
-                        const int b = bt * kBT + r;
-                        int page = -1;
-                        if (b < n_blocks && b < a.max_blocks) {
-                            page = __ldg(a.block_table + (size_t)s * a.max_blocks + b);
-                            if (page < 0 || page >= a.num_pages) {
-                                err_bits |= DSA_DEV_ERR_PAGE;
-                                page = -1;
-                            }
-                        }
-                        const uint32_t bits = __ballot_sync(0xffffffffu, page >= 0);
-                        if (lane == 0) info->valid[r4] = bits;
-                        const int8_t *src = a.kc_pool + (size_t)max(page, 0) * kIdxDim;
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            const uint32_t dst = sa + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
-                            if (page >= 0) cp_async_16(dst, src + 16 * c);
-                            else cp_async_16_zero(dst, a.kc_pool);
+                for (int r4 = 0; r4 < kBT / 32; ++r4) {
+                    const int r = r4 * 32 + lane;
+                    const int b = bt * kBT + r;
+                    int page = -1;
+                    if (b < n_blocks && b < a.max_blocks && b <= max_own) {
+                        page = s == s_lo ? pg_pre[r4] : __ldg(a.block_table + (size_t)s * a.max_blocks + b);
+                        if (page < 0 || page >= a.num_pages) {
+                            err_bits |= DSA_DEV_ERR_PAGE;
+                            page = -1;
                         }
                     }
-                    prev_s = s;
-                    prev_bt = bt;
+                    const uint32_t bits = __ballot_sync(0xffffffffu, page >= 0);
+                    if (lane == 0) info->valid[r4] = bits;
+                    const int8_t *src = a.kc_pool + (size_t)max(page, 0) * kIdxDim;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t dst = sa + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+                        if (page >= 0) cp_async_16(dst, src + 16 * c);
+                        else cp_async_16_zero(dst, a.kc_pool);
+                    }
                 }
                 // the queries' rows: box (64 B, 16 heads, 16 queries) at query t0
                 if (lane == 0) {
@@ -237,13 +254,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
                     tma_load_3d(sa + kOffB, &tm_q, 0, 0, t0, bars.full(st));
                 }
                 tc::cp_async_arrive_noinc(bars.full(st));
-                // the next stage may copy this one's keys: let them land first
-                cp_async_commit();
-                cp_async_wait<0>();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bars.full(st));   // the info words and copies above
+                if (lane == 0) mbar_arrive(bars.full(st));   // the info words above
                 ++k;
             }
+            cp_async_commit();   // this item's group: its gathers and the page ids kPidDepth ahead
         }
         // the end marker
         if (!*s_abort) {
@@ -308,7 +323,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
         }
     } else {
         // ============================================================ epilogue
+        const int ew = warp - 2;
         const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+        const int half = ew >> 2;                // queries 8*half .. +7 (columns 128*half ..)
         const int row = quarter * 32 + lane;     // block row of the tile
         int k = 0;
         while (true) {
@@ -325,29 +342,38 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
             const int bt = info->bt, y = info->y;
             const int b = bt * kBT + row;
             const bool row_ok = (info->valid[row >> 5] >> (row & 31)) & 1u;
-            const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kN);
-#pragma unroll 1
-            for (int j = 0; j < kQT / 4; ++j) {   // four queries (64 columns) per wait
-                uint32_t v[2][32];
-                tc::ld_32x32b_x32(taddr + 64 * j, v[0]);
-                tc::ld_32x32b_x32(taddr + 64 * j + 32, v[1]);
-                tc::wait_ld();
+            const uint32_t taddr =
+                tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kN + half * (kN / 2));
+            // weights and own blocks of this warp's 8 queries, read as shared-space vectors
+            const uint32_t s_info = base + st * kStageBytes + kOffInfo;
+            const uint32_t s_w = s_info + (uint32_t)offsetof(StageInfo, w) + (uint32_t)(8 * half * kMaxIdxHeads * 4);
+            int own8[8];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int qi = 4 * j + u;
-                    const int4 *wq = reinterpret_cast<const int4 *>(info->w[qi]);
-                    const uint32_t *x = v[u >> 1] + 16 * (u & 1);
-                    int sum = 0;
+            for (int u = 0; u < 8; ++u) own8[u] = info->own[8 * half + u];
+            // both 64-column loads in flight before the first wait; the second
+            // half's math overlaps nothing, the first's hides the second's load
+            uint32_t v[4][32];
+            tc::ld_32x32b_x32(taddr, v[0]);
+            tc::ld_32x32b_x32(taddr + 32, v[1]);
+            tc::ld_32x32b_x32(taddr + 64, v[2]);
+            tc::ld_32x32b_x32(taddr + 96, v[3]);
+            tc::wait_ld();
 #pragma unroll
-                    for (int h4 = 0; h4 < 4; ++h4) {
-                        const int4 wv = wq[h4];
-                        sum += wv.x * max((int)x[4 * h4 + 0], 0);
-                        sum += wv.y * max((int)x[4 * h4 + 1], 0);
-                        sum += wv.z * max((int)x[4 * h4 + 2], 0);
-                        sum += wv.w * max((int)x[4 * h4 + 3], 0);
-                    }
-                    if (row_ok && b <= info->own[qi]) a.scores[(size_t)(kQT * y + qi) * a.max_blocks + b] = sum;
+            for (int u = 0; u < 8; ++u) {   // query 8*half + u: columns 16u .. 16u+15
+                const uint32_t *x = v[u >> 1] + 16 * (u & 1);
+                int part[4];
+#pragma unroll
+                for (int h4 = 0; h4 < 4; ++h4) {   // four independent chains
+                    int4 wv;
+                    asm volatile("ld.shared.v4.s32 {%0,%1,%2,%3}, [%4];"
+                                 : "=r"(wv.x), "=r"(wv.y), "=r"(wv.z), "=r"(wv.w)
+                                 : "r"(s_w + (uint32_t)((u * kMaxIdxHeads + 4 * h4) * 4)));
+                    part[h4] = wv.x * max((int)x[4 * h4 + 0], 0) + wv.y * max((int)x[4 * h4 + 1], 0) +
+                               wv.z * max((int)x[4 * h4 + 2], 0) + wv.w * max((int)x[4 * h4 + 3], 0);
                 }
+                const int sum = (part[0] + part[1]) + (part[2] + part[3]);
+                if (row_ok && b <= own8[u])
+                    a.scores[(size_t)(kQT * y + 8 * half + u) * a.max_blocks + b] = sum;
             }
             tc::fence_before_sync();
             __syncwarp();
@@ -411,7 +437,7 @@ cudaError_t launch_index_score_tc(const IndexScoreArgs &a, int num_sms, cudaStre
         if (dev < 64) attr_done |= 1ull << dev;
     }
     const int n_bt = (a.max_blocks + kBT - 1) / kBT;
-    const int n_qt = (a.total_q + kQT - 1) / kQT;
+    const int n_qt = (a.total_q + kQT - 1) / kQT;   // items (y, bt), y-major
     const long long items = (long long)n_bt * n_qt;
     const int grid = (int)(items < num_sms ? items : num_sms);
     return launch_pdl(index_score_tc_kernel, dim3(grid), dim3(kTcThreads), (size_t)kSmemBytes, stream, tq, a, n_bt,

@@ -11,8 +11,16 @@
 
 namespace dsa {
 
+__device__ __forceinline__ void append_one(const KvAppendArgs &a);
+
 __global__ void __launch_bounds__(128) kv_append_kernel(KvAppendArgs a) {
     pdl_trigger();   // the next kernel may start its prologue; it waits for us before reading
+    append_one(a);
+    // overlapping a selection: finish only once it has (see KvAppendArgs)
+    if (a.overlap_prev) pdl_wait();
+}
+
+__device__ __forceinline__ void append_one(const KvAppendArgs &a) {
     const int i = blockIdx.x;
     const int s = find_seq(a.cu_new, a.num_seqs, i);
     const int first = __ldg(a.cu_new + s), last = __ldg(a.cu_new + s + 1);
@@ -54,6 +62,7 @@ __global__ void __launch_bounds__(128) kv_append_kernel(KvAppendArgs a) {
 
 cudaError_t launch_kv_append(const KvAppendArgs &a, cudaStream_t stream) {
     if (a.total_new == 0) return cudaSuccess;
+    if (a.overlap_prev) return launch_pdl(kv_append_kernel, dim3(a.total_new), dim3(128), 0, stream, a);
     kv_append_kernel<<<a.total_new, 128, 0, stream>>>(a);
     return cudaGetLastError();
 }

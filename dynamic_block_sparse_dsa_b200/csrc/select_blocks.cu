@@ -69,7 +69,12 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     const int K = __ldg(a.k_per_seq + s);
     const int n_vis = p / kBlockSize + 1;
     int32_t *out = a.sel + (size_t)t * a.k_max;
-    const bool bad_pos = p < 0 || p >= len || n_vis > a.max_blocks;
+    bool bad_pos = p < 0 || p >= len || n_vis > a.max_blocks;
+    if (a.cu_new && !bad_pos) {
+        // an append follows and overlaps this kernel: no candidate block may be appended to
+        const int n_new = __ldg(a.cu_new + s + 1) - __ldg(a.cu_new + s);
+        if (n_new > len || (n_new > 0 && n_vis - 1 > (len - n_new) / kBlockSize)) bad_pos = true;
+    }
     const bool bad_k = K < 1 || K > a.k_max;
     if (bad_pos || bad_k) {
         pdl_wait();
@@ -210,6 +215,10 @@ cudaError_t launch_select_blocks(const SelectArgs &a, cudaStream_t stream) {
     const int gr = (need + kSelWarps * 64 - 1) / (kSelWarps * 64);
     auto go = [&](auto kern, int G) {
         const int chunks = (a.max_blocks + kSelWarps * 64 * G - 1) / (kSelWarps * 64 * G);
+        if (a.cu_new) {   // the overlapping append relies on nothing earlier still running
+            kern<<<dim3(a.total_q, chunks), dim3(kSelThreads), 0, stream>>>(a);
+            return cudaGetLastError();
+        }
         return launch_pdl(kern, dim3(a.total_q, chunks), dim3(kSelThreads), 0, stream, a);
     };
     if (gr <= 1) return go(select_blocks_kernel<1>, 1);

@@ -73,9 +73,11 @@ struct Plan {
     static constexpr int kOffCuq = kOffMergeML + kConsumerWarps * 16 * 2 * 4;
     static constexpr int kOffRb = (kOffCuq + (kMaxSmemSeqs + 1) * 4 + 4 + 7) / 8 * 8;
     static constexpr int kOffBars = kOffRb + (kAttnMaxCtas + 1) * 8;
-    static constexpr int kNumBars = 2 * kStages + 2 * kSegSlots;
+    static constexpr int kNumBars = 2 * kStages + 2 * kSegSlots + 1;   // + the cluster inbox
     static constexpr int kOffWords = kOffBars + kNumBars * 8;
-    static constexpr int kSmemBytes = kOffWords + kNumWords * 4 + 1024;   // + slack to align the base to 1 KiB
+    // 2-CTA cluster mode: the partner's merged state (kMergeRows x (o[128], m, l))
+    static constexpr int kOffInbox = (kOffWords + kNumWords * 4 + 15) / 16 * 16;
+    static constexpr int kSmemBytes = kOffInbox + kMergeRows * kAttnPartStride * 4 + 1024;   // + base alignment slack
     static_assert(kStages <= kMaxStages, "stage words");
     static_assert(fused::kScratchBytes <= kStages * kStageBytes, "fused select scratch fits the ring");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -91,6 +93,8 @@ struct Smem {
     __device__ uint32_t empty(int s) const { return base + P::kOffBars + 8 * (P::kStages + s); }
     __device__ uint32_t qfull(int s) const { return base + P::kOffBars + 8 * (2 * P::kStages + s); }
     __device__ uint32_t qempty(int s) const { return base + P::kOffBars + 8 * (2 * P::kStages + kSegSlots + s); }
+    __device__ uint32_t inbox_full() const { return base + P::kOffBars + 8 * (2 * P::kStages + 2 * kSegSlots); }
+    __device__ uint32_t inbox() const { return base + P::kOffInbox; }
 };
 
 __device__ __forceinline__ long long range_begin(const AttnArgs &a, int c) {
@@ -137,7 +141,16 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     // every CTA's range start, once (64-bit divisions are slow; lookups are not)
     long long *s_rb = reinterpret_cast<long long *>(gbase + P::kOffRb);
     for (int i = tid; i <= a.num_ctas; i += kAttnThreads) s_rb[i] = range_begin(a, i);
-    const long long u0 = range_begin(a, c), u1 = range_begin(a, c + 1);
+    long long u0, u1;
+    if (a.cluster2) {   // half of pair c/2: units [0, h0) for rank 0, [h0, K) for rank 1
+        const long long p0 = (long long)(c >> 1) * a.k_max;
+        const int h0 = (a.k_max + 1) / 2;
+        u0 = p0 + ((c & 1) ? h0 : 0);
+        u1 = p0 + ((c & 1) ? a.k_max : h0);
+    } else {
+        u0 = range_begin(a, c);
+        u1 = range_begin(a, c + 1);
+    }
     const int G = a.group;
     const long long K = a.k_max;
 
@@ -150,6 +163,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             mbar_init(sm.qfull(s), 1);
             mbar_init(sm.qempty(s), 1);
         }
+        mbar_init(sm.inbox_full(), 1);
         for (int k = 0; k < kNumWords; ++k) W[k] = 0;
         for (int s = 0; s < kStages; ++s) W[kWFill + s] = -1;
         for (int s = 0; s < kSegSlots; ++s) W[kWSegEndTag + s] = -1;
@@ -158,6 +172,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     }
     pdl_trigger();
     __syncthreads();
+    if (a.cluster2) cluster_sync_all();   // the partner's inbox barrier is initialised before any remote arrive
     const int tag = W[kWTag];
     if constexpr (kFused) {
         fused::select_blocks_phase(a, f, gbase, tag, W + kWSelLast);
@@ -182,17 +197,28 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             prefetch_tensormap(&tm_v);
             prefetch_tensormap(&tm_q);
         }
-        pdl_wait();   // the selection and the appended tokens come from the kernels before
+        // the selection and the appended tokens come from the kernels before:
+        // pdl_wait() below, once the positions (inputs of the whole step) are
+        // already on their way
         uint32_t err_bits = 0;
-        if (kFused && f.total_new > 0 && lane == 0) {
-            // a query's own block holds its new token: every append lands before the first TMA
-            const long long t0 = clock64();
-            while (fused::ld_acquire(f.hdr + kHdrAppended) < f.total_new) {
-                if (clock64() - t0 > kWaitLimitCycles) { err_bits |= DSA_DEV_ERR_WAIT; break; }
+        bool sel_ready = true;
+        if (kFused && lane == 0 && u0 < u1) {
+            // the selections of the queries this CTA attends to (one poller
+            // per CTA), then every append: a query's own block holds its new
+            // token and the first TMA may read it
+            const int t_first = (int)((u0 / K) / a.num_kv_heads), t_last = (int)(((u1 - 1) / K) / a.num_kv_heads);
+            for (int t = t_first; t <= t_last && sel_ready; ++t) sel_ready = fused::wait_flag(f.flags + t, tag);
+            if (f.total_new > 0) {
+                const long long t0 = clock64();
+                while (fused::ld_acquire(f.hdr + kHdrAppended) < f.total_new) {
+                    if (clock64() - t0 > kWaitLimitCycles) { sel_ready = false; break; }
+                    __nanosleep(128);
+                }
+                fused::fence_proxy_async_global();
             }
-            fused::fence_proxy_async_global();
+            if (!sel_ready) err_bits |= DSA_DEV_ERR_WAIT;
         }
-        __syncwarp();
+        sel_ready = __shfl_sync(0xffffffffu, (int)sel_ready, 0) != 0;
         int item = 0, seg = 0;
         bool stop = false;
         for (long long base = u0; base < u1 && !stop; base += 32) {
@@ -207,14 +233,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 s = seq_of(a, s_cuq, t);
                 p = __ldg(a.q_pos + t);
                 const int len = __ldg(a.seq_lens + s);
-                bool ready = true;
-                if (kFused && !fused::wait_flag(f.flags + t, tag)) {   // this query's selection is published
-                    err_bits |= DSA_DEV_ERR_WAIT;
-                    ready = false;
-                }
+                pdl_wait();   // returns at once after the first time
                 // the selection may have been written during this launch: read it through L2
-                int n_sel = ready ? __ldcg(a.cnt + t) : 0;
-                const int b = ready ? __ldcg(a.sel + (size_t)t * a.k_max + j) : -1;
+                int n_sel = sel_ready ? __ldcg(a.cnt + t) : 0;
+                const int b = sel_ready ? __ldcg(a.sel + (size_t)t * a.k_max + j) : -1;
                 n_vis = p / kBlockSize + 1;
                 if (p < 0 || p >= len || n_vis > a.max_blocks || n_sel < 0 || n_sel > a.k_max) n_sel = 0;
                 if (j < n_sel) {
@@ -523,6 +545,92 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         const bool whole = seg_begin == pair * K && seg_end == (pair + 1) * K;
         const size_t out_row = (size_t)pt * a.num_q_heads + (size_t)pkvh * G;
         const int slot = 2 * c + (seg == 0 ? 0 : 1);
+        if (a.cluster2) {
+            // the two halves of the pair meet in rank 0's shared memory: rank 1
+            // stores its merged state there and arrives on rank 0's inbox
+            // barrier; rank 0 combines it with its own and writes the output
+            constexpr int kRowsPT = 2 * NT;
+            float Mo[kRowsPT], Lo[kRowsPT], Ao[kRowsPT][4];
+#pragma unroll
+            for (int i = 0; i < kRowsPT; ++i) {
+                const int e = tid + i * kConsumerWarps * 32;
+                const int r = (e >> 5) < G ? (e >> 5) : 0, d0 = (e & 31) * 4;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, s_ml[(w * 16 + r) * 2]);
+                float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+                if (M != -INFINITY) {
+#pragma unroll
+                    for (int w = 0; w < kConsumerWarps; ++w) {
+                        const float f = exp2f(s_ml[(w * 16 + r) * 2] - M);
+                        L += s_ml[(w * 16 + r) * 2 + 1] * f;
+                        const float4 v =
+                            *reinterpret_cast<const float4 *>(s_mo + (w * P::kMergeRows + r) * kMergeStride + d0);
+                        acc[0] += v.x * f; acc[1] += v.y * f; acc[2] += v.z * f; acc[3] += v.w * f;
+                    }
+                }
+                Mo[i] = M; Lo[i] = L;
+                Ao[i][0] = acc[0]; Ao[i][1] = acc[1]; Ao[i][2] = acc[2]; Ao[i][3] = acc[3];
+            }
+            if (c & 1) {
+                const uint32_t remote = mapa_shared(sm.inbox(), 0);
+#pragma unroll
+                for (int i = 0; i < kRowsPT; ++i) {
+                    const int e = tid + i * kConsumerWarps * 32;
+                    if (e >= G * 32) break;
+                    const int r = e >> 5, d0 = (e & 31) * 4;
+                    const uint32_t row = remote + (uint32_t)(r * kAttnPartStride * 4);
+                    st_cluster_f32x4(row + d0 * 4, Ao[i][0], Ao[i][1], Ao[i][2], Ao[i][3]);
+                    if (d0 == 0) st_cluster_f32x2(row + 128 * 4, Mo[i], Lo[i]);
+                }
+                __syncwarp();
+                named_barrier(1, kConsumerWarps * 32);
+                if (tid == 0) mbar_arrive_remote(mapa_shared(sm.inbox_full(), 0));
+            } else {
+                // the partner's state; the wait outlasts any bounded stall of the partner
+                bool got = mbar_try_wait_cluster(sm.inbox_full(), 0);
+                const long long t0 = clock64();
+                while (!got && clock64() - t0 < 4 * kWaitLimitCycles) got = mbar_try_wait_cluster(sm.inbox_full(), 0);
+                if (!got && tid == 0) {
+                    *s_abort = 1;
+                    set_err(a.dev_err, DSA_DEV_ERR_WAIT);
+                }
+                const float *inbox = reinterpret_cast<const float *>(gbase + P::kOffInbox);
+#pragma unroll
+                for (int i = 0; i < kRowsPT; ++i) {
+                    const int e = tid + i * kConsumerWarps * 32;
+                    if (e >= G * 32) break;
+                    const int r = e >> 5, d0 = (e & 31) * 4;
+                    float Mp = -INFINITY, Lp = 0.f;
+                    float4 ap = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (got) {
+                        Mp = inbox[r * kAttnPartStride + 128];
+                        Lp = inbox[r * kAttnPartStride + 129];
+                        ap = *reinterpret_cast<const float4 *>(inbox + r * kAttnPartStride + d0);
+                    }
+                    const float Mn = fmaxf(Mo[i], Mp);
+                    float L = 0.f, o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+                    if (Mn != -INFINITY) {
+                        const float f0 = Mo[i] == -INFINITY ? 0.f : exp2f(Mo[i] - Mn);
+                        const float f1 = Mp == -INFINITY ? 0.f : exp2f(Mp - Mn);
+                        L = Lo[i] * f0 + Lp * f1;
+                        o0 = Ao[i][0] * f0 + ap.x * f1; o1 = Ao[i][1] * f0 + ap.y * f1;
+                        o2 = Ao[i][2] * f0 + ap.z * f1; o3 = Ao[i][3] * f0 + ap.w * f1;
+                    }
+                    const float inv = L > 0.f ? 1.f / L : 0.f;
+                    *reinterpret_cast<uint2 *>(a.out + (out_row + r) * kHeadDim + d0) =
+                        make_uint2(pack_bf16x2(o0 * inv, o1 * inv), pack_bf16x2(o2 * inv, o3 * inv));
+                    if (a.lse && d0 == 0) a.lse[out_row + r] = L > 0.f ? (Mn + log2f(L)) * kLn2 : -INFINITY;
+                }
+            }
+            __syncwarp();
+            named_barrier(1, kConsumerWarps * 32);   // merge buffers free again
+            cursor = next_cursor;
+            u = seg_end;
+            ++pair;
+            ++seg;
+            continue;
+        }
         for (int e = tid; e < G * 32; e += kConsumerWarps * 32) {
             const int r = e >> 5, d0 = (e & 31) * 4;
             float M = -INFINITY;
@@ -745,6 +853,27 @@ cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream) {
     if (e == cudaSuccess) e = set_smem_attrs();
     if (e != cudaSuccess) return e;
     const FusedArgs none{};
+    if (a.cluster2) {   // pairs of CTAs on one GPC, merging through distributed shared memory
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(a.num_ctas);
+        cfg.blockDim = dim3(kAttnThreads);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = 2;
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        if (a.group <= 8) {
+            cfg.dynamicSmemBytes = Plan<1>::kSmemBytes;
+            return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<1, false>, m.k, m.v, m.q, a, none);
+        }
+        cfg.dynamicSmemBytes = Plan<2>::kSmemBytes;
+        return cudaLaunchKernelEx(&cfg, sparse_attn_kernel<2, false>, m.k, m.v, m.q, a, none);
+    }
     if (a.group <= 8)
         return launch_pdl(sparse_attn_kernel<1, false>, dim3(a.num_ctas), dim3(kAttnThreads), Plan<1>::kSmemBytes,
                           stream, m.k, m.v, m.q, a, none);

@@ -174,6 +174,25 @@ int dsa_select_blocks(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa
                       void *workspace, size_t workspace_bytes, int32_t *dev_err, dsa_stream_t stream);
 
 /*
+ * dsa_select_blocks_append -- dsa_select_blocks, then dsa_kv_append, for a
+ * decode batch: the two are ordered so that the token copies overlap the
+ * selection (the selection never reads them), and whatever is launched
+ * after this call on `stream` sees both finished.  Same arguments and
+ * results as the two calls; the selection kernel waits for all earlier work
+ * on the stream before it starts.
+ *  - Every appended block of a sequence must lie at or after the own block of
+ *    each of that sequence's queries; a query that breaks this gets
+ *    DSA_DEV_ERR_POS and cnt 0 (its selection would read keys being written).
+ * Device errors: those of the two calls.
+ */
+int dsa_select_blocks_append(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                             const int32_t *cu_new, int32_t total_new, const void *k_new, const void *v_new,
+                             const int8_t *kc_new, const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads,
+                             int32_t w_abs_max, const int32_t *k_per_seq, int32_t k_max, int32_t *sel,
+                             int32_t *cnt, void *workspace, size_t workspace_bytes, int32_t *dev_err,
+                             dsa_stream_t stream);
+
+/*
  * Exact attention over the selected blocks [P1 4(3) decode schematic; P3 4:
  * exact attention on the selected part; P4 "Day-0 Adaptation for Large
  * Language Models: From Architecture Analysis to Inference Serving", table:

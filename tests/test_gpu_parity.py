@@ -27,12 +27,13 @@ def _handles(wl):
             dsa.QueryBatch(wl.cu_q, wl.q_pos))
 
 
-def gpu_step(wl, decode=True, bufs=None, fused=False, fused_decode=False):
+def gpu_step(wl, decode=True, bufs=None, fused=False, fused_decode=False, overlap=False):
     cache, seqs, queries = _handles(wl)
     err = torch.zeros(1, dtype=torch.int32, device=wl.device)
     bufs = dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
                     q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=wl.spec.k_max,
-                    decode=decode, fused_select=fused, fused_decode=fused_decode, bufs=bufs, dev_err=err)
+                    decode=decode, fused_select=fused or overlap, overlap_append=overlap,
+                    fused_decode=fused_decode, bufs=bufs, dev_err=err)
     torch.cuda.synchronize()
     return bufs, int(err.item())
 
@@ -81,6 +82,10 @@ SMALL = {
     # query tiles of 16 that straddle sequence boundaries (tensor-core scoring path)
     "prefill_tiles_straddle": dict(seq_lens=(9000, 300, 5000, 70), n_new=(30, 20, 17, 5), k_per_seq=(9, 3, 6, 2),
                                    k_max=9),
+    # 48 (query, KV head) pairs: the decode entry runs one 2-CTA cluster per pair
+    # (odd Top-K: unequal halves; short sequences: one half without usable blocks)
+    "cluster_pairs": dict(seq_lens=tuple(range(70, 70 + 24 * 431, 431)), n_new=(1,) * 24, k_per_seq=(7,) * 24,
+                          k_max=7),
     # fewer indexer heads than the 16 of a tensor-core tile
     "prefill_5_idx_heads": dict(seq_lens=(20000,), n_new=(100,), k_per_seq=(10,), k_max=10, num_idx_heads=5),
 }
@@ -368,3 +373,44 @@ def test_fused_decode_bad_metadata_sets_flags(what, cuda_device):
     assert not err & dsa._lib.DEV_ERR_WAIT
     if what != "page":
         assert int(b["cnt"][0 if what == "k" else 1]) == 0
+
+
+# ----------------------------------------------------------------------------- append overlapping the selection
+@pytest.mark.parametrize("q_scale", [1.0, 12.0], ids=["plain", "sharp"])
+@pytest.mark.parametrize("name", FUSED_DECODE_SMALL)
+def test_select_append_small_cases(name, q_scale, cuda_device):
+    wl = wk.make_workload(_small_spec(name, q_scale), seed=200 + len(name), device=cuda_device)
+    ref = oracle_step(wl)
+    bufs, err = gpu_step(wl, overlap=True)
+    assert err == 0, f"device error bits {err}"
+    compare(wl, ref, bufs, fused=True)
+
+
+def test_select_append_flags_non_decode_queries(cuda_device):
+    wl = wk.make_workload(_small_spec("ragged_prefill_tail", 8.0), seed=44, device=cuda_device)
+    ok = _decode_eligible(wl)
+    good = [int(t) for t in np.flatnonzero(ok)]
+    ref = oracle_step(wl, queries=good)
+    bufs, err = gpu_step(wl, overlap=True)
+    assert err & dsa._lib.DEV_ERR_POS
+    compare(wl, ref, bufs, fused=True)
+    assert (bufs["cnt"].cpu().numpy()[~ok] == 0).all()
+
+
+@pytest.mark.parametrize("q_scale", [1.0, 12.0])
+def test_select_append_batched_gqa_workload(q_scale, cuda_device):
+    spec = wk.scaled(wk.batched_gqa_decode(), q_scale=q_scale)
+    wl = wk.make_workload(spec, seed=1002, device=cuda_device)
+    ref = oracle_step(wl)
+    bufs, err = gpu_step(wl, overlap=True)
+    assert err == 0
+    compare(wl, ref, bufs, fused=True)
+
+
+@pytest.mark.slow
+def test_select_append_1m_workload(cuda_device):
+    wl = wk.make_workload(wk.decode_1m(), seed=1003, device=cuda_device)
+    ref = oracle_step(wl)
+    bufs, err = gpu_step(wl, overlap=True)
+    assert err == 0
+    compare(wl, ref, bufs, fused=True)
