@@ -78,26 +78,36 @@ __device__ __forceinline__ void fence_proxy_async_global() {
     asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// wait until *p == v (acquire); false on timeout.  Polls back off so that a
-// grid of waiters does not crowd out the stores they wait for.
+__device__ __forceinline__ int ld_relaxed(const int32_t *p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// wait until *p == v; false on timeout.  Polls are relaxed loads with a back
+// off (a grid of acquire loads would crowd out the stores they wait for);
+// the acquire is one fence once the value is seen.
 __device__ __forceinline__ bool wait_flag(const int32_t *p, int v) {
-    if (ld_acquire(p) == v) return true;
     const long long t0 = clock64();
 #pragma unroll 1
-    while (ld_acquire(p) != v) {
+    while (ld_relaxed(p) != v) {
         if (clock64() - t0 > kWaitLimitCycles) return false;
         __nanosleep(128);
     }
+    fence_acquire_gpu();
     return true;
 }
 
-// first group of CTA c in the even split of `total` groups over C CTAs
+// first group of CTA c in the even split of `total` groups over C CTAs (32-bit
+// arithmetic: c <= 256 and total <= kFusedMaxQ * 2048 keep c * total < 2^31;
+// 64-bit divisions are long dependent chains on the GPU)
 __device__ __forceinline__ int group_begin(int c, int total, int C) {
-    return (int)((long long)c * total / C);
+    return (int)((unsigned)c * (unsigned)total / (unsigned)C);
 }
 // the CTA whose range holds group x (ranges are contiguous and ascending)
 __device__ __forceinline__ int cta_of_group(int x, int total, int C) {
-    int c = (int)(((long long)x * C) / total);
+    int c = (int)((unsigned)x * (unsigned)C / (unsigned)total);
     while (c + 1 < C && group_begin(c + 1, total, C) <= x) ++c;
     while (c > 0 && group_begin(c, total, C) > x) --c;
     return c;
@@ -126,7 +136,8 @@ __device__ __forceinline__ void finalize(const AttnArgs &a, const FusedArgs &f, 
         f.cnt[t] = km + 1;
     }
     for (int i = km + 1 + lane; i < a.k_max; i += 32) out[i] = -1;
-    __threadfence();
+    // the warp barrier orders every lane's stores before lane 0's release,
+    // which carries them to whoever acquires the flag
     __syncwarp();
     if (lane == 0) st_release(f.flags + t, tag);
 }
@@ -179,8 +190,7 @@ __device__ __forceinline__ void append_tokens(const AttnArgs &a, const FusedArgs
         }
         if (done > 0) {
             fence_proxy_async_global();   // the attention phase reads these rows with TMA
-            __threadfence();
-            __syncthreads();
+            __syncthreads();               // ordered before tid 0's release (cumulative)
             if (tid == 0) atomic_add_acq_rel_gpu(f.hdr + kHdrAppended, done);
         }
     }
@@ -280,7 +290,6 @@ __device__ __forceinline__ void select_blocks_phase(const AttnArgs &a, const Fus
         if (q.k > 0) n = q.n_vis <= q.k ? q.n_vis : 1;
         for (int i = lane; i < a.k_max; i += 32) out[i] = i < n ? (n == 1 ? q.n_vis - 1 : i) : -1;
         if (lane == 0) f.cnt[t] = n;
-        __threadfence();
         __syncwarp();
         if (lane == 0) st_release(f.flags + t, tag);
     }
@@ -445,8 +454,7 @@ __device__ __forceinline__ void select_blocks_phase(const AttnArgs &a, const Fus
                     if (warp == 0) {
                         if (lane < kk) cand[lane] = acc[0];
                         if (32 + lane < kk) cand[32 + lane] = acc[1];
-                        __threadfence();
-                        __syncwarp();
+                        __syncwarp();   // ordered before lane 0's acq_rel add (cumulative)
                         if (lane == 0) {
                             const int covered = min(g_hi, ge) - max(g_lo, gb);
                             const int old = atomic_add_acq_rel_gpu(f.sel_count + t, covered);

@@ -125,9 +125,11 @@ int attn_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queri
     const int group = num_q_heads / cache->num_kv_heads;
     if (group > kMaxGroup) return DSA_ERR_UNSUPPORTED;
     if (!(sm_scale > 0.f)) return DSA_ERR_INVALID_ARG;
-    // TMA coordinates are int32: pool rows (page*64+token) and query rows (t*Hq+h)
+    // TMA coordinates are int32: pool rows (page*64+token) and query rows (t*Hq+h);
+    // work units (query, KV head, selection slot) are counted in 32 bits
     if ((long long)cache->num_pages * kBlockSize >= (1LL << 31) ||
-        (long long)queries->total_q * num_q_heads >= (1LL << 31))
+        (long long)queries->total_q * num_q_heads >= (1LL << 31) ||
+        (long long)queries->total_q * cache->num_kv_heads * k_max >= (1LL << 31))
         return DSA_ERR_UNSUPPORTED;
     a = AttnArgs{};
     a.k_pool = static_cast<const __nv_bfloat16 *>(cache->k_pool);

@@ -22,8 +22,8 @@
 //            weights, into a 4-stage ring;
 //   warp 1   MMA issuer (one thread): two K=32 MMAs per tile into one of two
 //            256-column accumulators;
-//   warps 2-9 epilogue (two per SM sub-partition: a quarter of the rows and
-//            half of the queries each): tcgen05.ld of the accumulator rows,
+//   warps 2-17 epilogue (four per SM sub-partition: a quarter of the rows and
+//            a quarter of the queries each): tcgen05.ld of the accumulator rows,
 //            relu * w summed over heads, one coalesced 128-byte store per
 //            (query, warp).
 // Tiles are (16-query tile, 128-block tile) pairs in query-tile-major order,
@@ -38,8 +38,11 @@
 namespace dsa {
 
 namespace {
-constexpr int kEpiWarps = 8;                       // two per SM sub-partition
-constexpr int kTcThreads = 64 + 32 * kEpiWarps;   // loader, MMA, epilogue
+constexpr int kEpiWarps = 16;                      // four per SM sub-partition
+constexpr int kLoadWarps = 4;                      // one gathered row per lane
+constexpr int kMmaWarp = kLoadWarps;
+constexpr int kEpiWarp0 = kLoadWarps + 1;
+constexpr int kTcThreads = 32 * (kLoadWarps + 1 + kEpiWarps);   // loaders, MMA, epilogue
 constexpr int kTcStages = 4;
 constexpr int kBT = 128;                 // blocks per tile (MMA M)
 constexpr int kQT = 16;                  // queries per tile (MMA N = 16 x 16 heads)
@@ -63,12 +66,11 @@ constexpr int kOffMisc = kOffBars + kNumBars * 8;   // tmem base, abort flag
 constexpr int kCuqCache = 1024;                      // cu_q entries staged in shared memory
 constexpr int kOffCuq = kOffMisc + 16;
 constexpr int kPidDepth = 4;                         // block tiles of page ids in flight
-constexpr int kOffPid = kOffCuq + kCuqCache * 4;     // [kPidDepth][kBT] int32
 // + alignment slack; at least 116 KiB so that two CTAs never share an SM (each
 // holds all 512 tensor-memory columns)
-constexpr int kSmemUsed = kOffPid + kPidDepth * kBT * 4 + 1024;
+constexpr int kSmemUsed = kOffCuq + kCuqCache * 4 + 1024;
 constexpr int kSmemBytes = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
-constexpr int kFullCount = 33;                       // 32 cp.async arrivals + the info arrival
+constexpr int kFullCount = kLoadWarps * 33;          // per loader warp: 32 cp.async arrivals + its info arrival
 constexpr int kEmptyCount = 1 + kEpiWarps;           // MMA commit + the epilogue warps
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -109,7 +111,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
         misc[2] = 0;
         fence_barrier_init();
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc::tmem_alloc(smem_u32(g + kOffMisc), kTmemCols);
         tc::tmem_relinquish();
     }
@@ -119,25 +121,26 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
     tc::fence_after_sync();
     const uint32_t tmem = (uint32_t)misc[0];
 
-    const long long n_items = (long long)n_bt * n_qt;
-    const long long i0 = n_items * blockIdx.x / gridDim.x, i1 = n_items * (blockIdx.x + 1) / gridDim.x;
+    // item indices fit 32 bits (the host checks); only this split uses 64-bit products
+    const unsigned n_items = (unsigned)n_bt * (unsigned)n_qt;
+    const unsigned i0 = (unsigned)((unsigned long long)n_items * blockIdx.x / gridDim.x);
+    const unsigned i1 = (unsigned)((unsigned long long)n_items * (blockIdx.x + 1) / gridDim.x);
     const int H = a.num_idx_heads;
 
-    if (warp == 0) {
-        // ============================================================ loader
+    if (warp < kLoadWarps) {
+        // ============================================================ loaders
+        const int lw = warp;   // rows 32*lw .. 32*lw+31 of every tile
         // Items are (query tile y, block tile bt), y-major: the queries'
         // positions and weights change once per query tile, the coarse keys
-        // every item.  The page ids of item j are copied into a small ring
-        // kPidDepth items ahead (cp.async), so the gather of item j never
-        // waits on a global load; its keys then land through the stage's
-        // full barrier.
-        if (lane == 0) prefetch_tensormap(&tm_q);
+        // every item.  The page ids of item j are loaded into a register ring
+        // kPidDepth items ahead, so the gather of item j never waits on a
+        // global load; its keys then land through the stage's full barrier.
+        if (lw == 0 && lane == 0) prefetch_tensormap(&tm_q);
         int *s_cuq = reinterpret_cast<int *>(g + kOffCuq);
-        const int *s_pid = reinterpret_cast<const int *>(g + kOffPid);
         const bool cuq_cached = a.num_seqs + 1 <= kCuqCache;
         if (cuq_cached)
-            for (int i = lane; i <= a.num_seqs; i += 32) s_cuq[i] = __ldg(a.cu_q + i);
-        __syncwarp();
+            for (int i = lane + 32 * lw; i <= a.num_seqs; i += 32 * kLoadWarps) s_cuq[i] = __ldg(a.cu_q + i);
+        named_barrier(1, 32 * kLoadWarps);
         auto seq_of = [&](int t) {
             if (!cuq_cached) return seq_of_query(a, t);
             int lo = 0, hi = a.num_seqs - 1;
@@ -148,34 +151,25 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
             return lo;
         };
         auto cu = [&](int s) { return cuq_cached ? s_cuq[s] : __ldg(a.cu_q + s); };
-        // page ids of item j's first sequence into ring slot j % kPidDepth
-        // (4 per lane, 4-byte copies: rows of the table need not be 16-byte aligned)
-        auto prefetch_pids = [&](long long j) {
-            const int y = (int)(j / n_bt), bt = (int)(j % n_bt);
+        // page id of this lane's row of item j (first sequence of its tile)
+        auto load_pid = [&](unsigned j) {
+            const int y = (int)(j / (unsigned)n_bt), bt = (int)(j - (unsigned)y * (unsigned)n_bt);
             const int s0 = seq_of(kQT * y);
-            const uint32_t dst = base + kOffPid + (uint32_t)((j % kPidDepth) * kBT * 4);
-#pragma unroll
-            for (int r4 = 0; r4 < kBT / 32; ++r4) {
-                const int r = r4 * 32 + lane, b = bt * kBT + r;
-                const int32_t *src = a.block_table + (size_t)s0 * a.max_blocks + min(b, a.max_blocks - 1);
-                if (b < a.max_blocks)
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst + 4 * r), "l"(src));
-                else
-                    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, 0;\n" ::"r"(dst + 4 * r), "l"(src));
-            }
+            const int b = bt * kBT + 32 * lw + lane;
+            return b < a.max_blocks ? __ldg(a.block_table + (size_t)s0 * a.max_blocks + b) : -1;
         };
         pdl_wait();   // coarse keys may come from the preceding append
-        for (int d = 0; d < kPidDepth; ++d) {
-            if (i0 + d < i1) prefetch_pids(i0 + d);
-            cp_async_commit();
-        }
+        int ring[kPidDepth];
+#pragma unroll
+        for (int d = 0; d < kPidDepth; ++d) ring[d] = i0 + d < i1 ? load_pid(i0 + d) : -1;
         int k = 0;    // stages published
         int cur_y = -1;
         int pos = -1, s_lo = 0, s_hi = -1, len_lo = 0;
         int wv[8];
         uint32_t err_bits = 0;
-        for (long long it = i0; it < i1 && !*s_abort; ++it) {
-            const int y = (int)(it / n_bt), bt = (int)(it % n_bt);
+        // one item: its sub-items (one per sequence of the query tile) into the ring
+        auto process = [&](unsigned it, int pg_pre) {
+            const int y = (int)(it / (unsigned)n_bt), bt = (int)(it - (unsigned)y * (unsigned)n_bt);
             const int t0 = kQT * y;
             if (y != cur_y) {   // a new query tile: positions, weights, sequences
                 cur_y = y;
@@ -190,15 +184,6 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
                 s_hi = seq_of(min(t0 + kQT, a.total_q) - 1);
                 len_lo = __ldg(a.seq_lens + s_lo);
             }
-            // this item's page ids have landed (kPidDepth - 1 newer groups may be pending)
-            cp_async_wait<kPidDepth - 1>();
-            __syncwarp();
-            const int *pid = s_pid + (it % kPidDepth) * kBT;
-            int pg_pre[kBT / 32];
-#pragma unroll
-            for (int r4 = 0; r4 < kBT / 32; ++r4) pg_pre[r4] = pid[r4 * 32 + lane];
-            __syncwarp();   // the slot is refilled below
-            if (it + kPidDepth < i1) prefetch_pids(it + kPidDepth);
             for (int s = s_lo; s <= s_hi && !*s_abort; ++s) {
                 const int len = s == s_lo ? len_lo : __ldg(a.seq_lens + s);
                 const int t = t0 + (lane & (kQT - 1));
@@ -220,26 +205,27 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
                 uint8_t *stage = g + st * kStageBytes;
                 StageInfo *info = reinterpret_cast<StageInfo *>(stage + kOffInfo);
                 const uint32_t sa = base + st * kStageBytes;
-                if (lane == 0) { info->end = 0; info->s = s; info->bt = bt; info->y = y; }
-                if (lane < kQT) info->own[lane] = own;
+                if (lw == 0) {
+                    if (lane == 0) { info->end = 0; info->s = s; info->bt = bt; info->y = y; }
+                    if (lane < kQT) info->own[lane] = own;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) (&info->w[0][0])[lane + 32 * j] = wv[j];
-                // the 128 coarse keys: 4 rows per lane, 4 x 16 B per row, swizzled
-                const int n_blocks = (len + kBlockSize - 1) / kBlockSize;
-#pragma unroll
-                for (int r4 = 0; r4 < kBT / 32; ++r4) {
-                    const int r = r4 * 32 + lane;
+                    for (int j = 0; j < 8; ++j) (&info->w[0][0])[lane + 32 * j] = wv[j];
+                }
+                // this lane's coarse key: 4 x 16 B, swizzled
+                {
+                    const int n_blocks = (len + kBlockSize - 1) / kBlockSize;
+                    const int r = 32 * lw + lane;
                     const int b = bt * kBT + r;
                     int page = -1;
                     if (b < n_blocks && b < a.max_blocks && b <= max_own) {
-                        page = s == s_lo ? pg_pre[r4] : __ldg(a.block_table + (size_t)s * a.max_blocks + b);
+                        page = s == s_lo ? pg_pre : __ldg(a.block_table + (size_t)s * a.max_blocks + b);
                         if (page < 0 || page >= a.num_pages) {
                             err_bits |= DSA_DEV_ERR_PAGE;
                             page = -1;
                         }
                     }
                     const uint32_t bits = __ballot_sync(0xffffffffu, page >= 0);
-                    if (lane == 0) info->valid[r4] = bits;
+                    if (lane == 0) info->valid[lw] = bits;
                     const int8_t *src = a.kc_pool + (size_t)max(page, 0) * kIdxDim;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
@@ -249,7 +235,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
                     }
                 }
                 // the queries' rows: box (64 B, 16 heads, 16 queries) at query t0
-                if (lane == 0) {
+                if (lw == 0 && lane == 0) {
                     tc::mbar_expect_tx(bars.full(st), kBBytes);
                     tma_load_3d(sa + kOffB, &tm_q, 0, 0, t0, bars.full(st));
                 }
@@ -258,7 +244,21 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
                 if (lane == 0) mbar_arrive(bars.full(st));   // the info words above
                 ++k;
             }
-            cp_async_commit();   // this item's group: its gathers and the page ids kPidDepth ahead
+        };
+        // the item loop, unrolled by the ring depth so that every ring slot is a
+        // fixed register: slot d is read for item base + d and refilled with
+        // the page id of item base + d + kPidDepth, which is read kPidDepth
+        // items later -- no register copy ever waits on a load in flight
+        for (unsigned base0 = i0; base0 < i1 && !*s_abort; base0 += kPidDepth) {
+#pragma unroll
+            for (int d = 0; d < kPidDepth; ++d) {
+                const unsigned it = base0 + d;
+                if (it < i1 && !*s_abort) {
+                    const int pg_pre = ring[d];
+                    ring[d] = it + kPidDepth < i1 ? load_pid(it + kPidDepth) : -1;
+                    process(it, pg_pre);
+                }
+            }
         }
         // the end marker
         if (!*s_abort) {
@@ -267,7 +267,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
                 *s_abort = 1;
             } else {
                 StageInfo *info = reinterpret_cast<StageInfo *>(g + st * kStageBytes + kOffInfo);
-                if (lane == 0) { info->end = 1; info->s = -1; }
+                if (lw == 0 && lane == 0) { info->end = 1; info->s = -1; }
                 tc::cp_async_arrive_noinc(bars.full(st));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bars.full(st));
@@ -278,12 +278,12 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
         if (lane == 0 && err_bits) set_err(a.dev_err, err_bits);
         cp_async_commit();
         cp_async_wait<0>();
-        if (*s_abort && lane == 0) {
+        if (*s_abort && lw == 0 && lane == 0) {
             set_err(a.dev_err, DSA_DEV_ERR_WAIT);
             for (int j = max(0, k - kTcStages); j < k; ++j)
                 mbar_wait(bars.full(j % kTcStages), (j / kTcStages) & 1, s_never);
         }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
         constexpr uint32_t idesc = tc::idesc_i8(kBT, kN);
         int k = 0;
@@ -323,9 +323,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
         }
     } else {
         // ============================================================ epilogue
-        const int ew = warp - 2;
+        const int ew = warp - kEpiWarp0;
         const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
-        const int half = ew >> 2;                // queries 8*half .. +7 (columns 128*half ..)
+        const int qgrp = ew >> 2;                // queries 4*qgrp .. +3 (columns 64*qgrp ..)
         const int row = quarter * 32 + lane;     // block row of the tile
         int k = 0;
         while (true) {
@@ -343,23 +343,19 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
             const int b = bt * kBT + row;
             const bool row_ok = (info->valid[row >> 5] >> (row & 31)) & 1u;
             const uint32_t taddr =
-                tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kN + half * (kN / 2));
-            // weights and own blocks of this warp's 8 queries, read as shared-space vectors
+                tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kN + qgrp * 64);
+            // weights and own blocks of this warp's 4 queries, read as shared-space vectors
             const uint32_t s_info = base + st * kStageBytes + kOffInfo;
-            const uint32_t s_w = s_info + (uint32_t)offsetof(StageInfo, w) + (uint32_t)(8 * half * kMaxIdxHeads * 4);
-            int own8[8];
+            const uint32_t s_w = s_info + (uint32_t)offsetof(StageInfo, w) + (uint32_t)(4 * qgrp * kMaxIdxHeads * 4);
+            int own4[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) own8[u] = info->own[8 * half + u];
-            // both 64-column loads in flight before the first wait; the second
-            // half's math overlaps nothing, the first's hides the second's load
-            uint32_t v[4][32];
+            for (int u = 0; u < 4; ++u) own4[u] = info->own[4 * qgrp + u];
+            uint32_t v[2][32];
             tc::ld_32x32b_x32(taddr, v[0]);
             tc::ld_32x32b_x32(taddr + 32, v[1]);
-            tc::ld_32x32b_x32(taddr + 64, v[2]);
-            tc::ld_32x32b_x32(taddr + 96, v[3]);
             tc::wait_ld();
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {   // query 8*half + u: columns 16u .. 16u+15
+            for (int u = 0; u < 4; ++u) {   // query 4*qgrp + u: columns 16u .. 16u+15 of this warp's 64
                 const uint32_t *x = v[u >> 1] + 16 * (u & 1);
                 int part[4];
 #pragma unroll
@@ -372,8 +368,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
                                wv.z * max((int)x[4 * h4 + 2], 0) + wv.w * max((int)x[4 * h4 + 3], 0);
                 }
                 const int sum = (part[0] + part[1]) + (part[2] + part[3]);
-                if (row_ok && b <= own8[u])
-                    a.scores[(size_t)(kQT * y + 8 * half + u) * a.max_blocks + b] = sum;
+                if (row_ok && b <= own4[u])
+                    a.scores[(size_t)(kQT * y + 4 * qgrp + u) * a.max_blocks + b] = sum;
             }
             tc::fence_before_sync();
             __syncwarp();
@@ -387,7 +383,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
 
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
     }
@@ -439,6 +435,7 @@ cudaError_t launch_index_score_tc(const IndexScoreArgs &a, int num_sms, cudaStre
     const int n_bt = (a.max_blocks + kBT - 1) / kBT;
     const int n_qt = (a.total_q + kQT - 1) / kQT;   // items (y, bt), y-major
     const long long items = (long long)n_bt * n_qt;
+    if (items >= (1LL << 31)) return cudaErrorInvalidValue;   // item indices are 32-bit in the kernel
     const int grid = (int)(items < num_sms ? items : num_sms);
     return launch_pdl(index_score_tc_kernel, dim3(grid), dim3(kTcThreads), (size_t)kSmemBytes, stream, tq, a, n_bt,
                       n_qt);

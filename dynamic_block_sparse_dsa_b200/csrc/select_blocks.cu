@@ -165,16 +165,17 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
         if (32 + lane < kk) cand[32 + lane] = acc[1];
     }
 
-    // ---- the last chunk CTA of this query merges the chunks' lists
-    __threadfence();
+    // ---- the last chunk CTA of this query merges the chunks' lists: the
+    // barrier orders warp 0's list stores before tid 0's release-add, and the
+    // last adder's acquire (then the barrier) orders every list before the
+    // loads below
     __syncthreads();
     if (tid == 0) {
-        const int old = atomicAdd(a.counters + t, 1);
+        const int old = atomic_add_acq_rel_gpu(a.counters + t, 1);
         s_last = (old == n_chunks - 1);
     }
     __syncthreads();
     if (!s_last) return;
-    __threadfence();
     constexpr int kPer = (kSelMaxChunks + kSelWarps - 1) / kSelWarps;   // lists per warp
     key64 lists[kPer][2];
 #pragma unroll

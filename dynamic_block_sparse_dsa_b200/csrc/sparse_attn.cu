@@ -97,12 +97,18 @@ struct Smem {
     __device__ uint32_t inbox() const { return base + P::kOffInbox; }
 };
 
-__device__ __forceinline__ long long range_begin(const AttnArgs &a, int c) {
+// Unit indices are 32-bit (the host keeps total_units below 2^31): the hot
+// loops divide them by the Top-K and the KV-head count, and 64-bit integer
+// division is a long dependent instruction chain on the GPU.
+using unit_t = uint32_t;
+
+// first unit of CTA c (64-bit products; computed once per CTA)
+__device__ __forceinline__ unit_t range_begin(const AttnArgs &a, int c) {
     if (a.pair_aligned) {
-        const long long pairs = a.total_units / a.k_max;
-        return (long long)c * pairs / a.num_ctas * a.k_max;
+        const unsigned long long pairs = (unsigned long long)a.total_units / (unsigned)a.k_max;
+        return (unit_t)((unsigned long long)c * pairs / (unsigned)a.num_ctas * (unsigned)a.k_max);
     }
-    return (long long)c * a.total_units / a.num_ctas;
+    return (unit_t)((unsigned long long)c * (unsigned long long)a.total_units / (unsigned)a.num_ctas);
 }
 
 // sequence of query t: last s with cu_q[s] <= t, from the shared-memory copy when it fits
@@ -139,11 +145,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x;
     // every CTA's range start, once (64-bit divisions are slow; lookups are not)
-    long long *s_rb = reinterpret_cast<long long *>(gbase + P::kOffRb);
+    unit_t *s_rb = reinterpret_cast<unit_t *>(gbase + P::kOffRb);
     for (int i = tid; i <= a.num_ctas; i += kAttnThreads) s_rb[i] = range_begin(a, i);
-    long long u0, u1;
+    unit_t u0, u1;
     if (a.cluster2) {   // half of pair c/2: units [0, h0) for rank 0, [h0, K) for rank 1
-        const long long p0 = (long long)(c >> 1) * a.k_max;
+        const unit_t p0 = (unit_t)(c >> 1) * (unit_t)a.k_max;
         const int h0 = (a.k_max + 1) / 2;
         u0 = p0 + ((c & 1) ? h0 : 0);
         u1 = p0 + ((c & 1) ? a.k_max : h0);
@@ -152,7 +158,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         u1 = range_begin(a, c + 1);
     }
     const int G = a.group;
-    const long long K = a.k_max;
+    const unit_t K = (unit_t)a.k_max;
+    const unit_t Hkv = (unit_t)a.num_kv_heads;
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -206,14 +213,15 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             // the selections of the queries this CTA attends to (one poller
             // per CTA), then every append: a query's own block holds its new
             // token and the first TMA may read it
-            const int t_first = (int)((u0 / K) / a.num_kv_heads), t_last = (int)(((u1 - 1) / K) / a.num_kv_heads);
+            const int t_first = (int)((u0 / K) / Hkv), t_last = (int)(((u1 - 1) / K) / Hkv);
             for (int t = t_first; t <= t_last && sel_ready; ++t) sel_ready = fused::wait_flag(f.flags + t, tag);
             if (f.total_new > 0) {
                 const long long t0 = clock64();
-                while (fused::ld_acquire(f.hdr + kHdrAppended) < f.total_new) {
+                while (fused::ld_relaxed(f.hdr + kHdrAppended) < f.total_new) {
                     if (clock64() - t0 > kWaitLimitCycles) { sel_ready = false; break; }
                     __nanosleep(128);
                 }
+                fused::fence_acquire_gpu();
                 fused::fence_proxy_async_global();
             }
             if (!sel_ready) err_bits |= DSA_DEV_ERR_WAIT;
@@ -221,15 +229,15 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         sel_ready = __shfl_sync(0xffffffffu, (int)sel_ready, 0) != 0;
         int item = 0, seg = 0;
         bool stop = false;
-        for (long long base = u0; base < u1 && !stop; base += 32) {
-            const long long uu = base + lane;
+        for (unit_t base = u0; base < u1 && !stop; base += 32) {
+            const unit_t uu = base + lane;
             const bool in = uu < u1;
             int t = 0, kvh = 0, s = 0, p = 0, n_vis = 0, blk = -1, page = -1;
             if (in) {
-                const long long pair = uu / K;
+                const unit_t pair = uu / K;
                 const int j = (int)(uu - pair * K);
-                t = (int)(pair / a.num_kv_heads);
-                kvh = (int)(pair % a.num_kv_heads);
+                t = (int)(pair / Hkv);
+                kvh = (int)(pair - (unit_t)t * Hkv);
                 s = seq_of(a, s_cuq, t);
                 p = __ldg(a.q_pos + t);
                 const int len = __ldg(a.seq_lens + s);
@@ -249,13 +257,13 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     }
                 }
             }
-            const long long chunk_end = min(u1, base + 32);
-            long long v = base;
+            const unit_t chunk_end = min(u1, base + 32);
+            unit_t v = base;
             while (v < chunk_end) {
                 const int lf = (int)(v - base);
-                const long long pair = v / K;
-                const long long seg_stop = min(u1, (pair + 1) * K);
-                const long long run_end = min(chunk_end, seg_stop);
+                const unit_t pair = v / K;
+                const unit_t seg_stop = min(u1, (pair + 1) * K);
+                const unit_t run_end = min(chunk_end, seg_stop);
                 const int ll = (int)(run_end - 1 - base);
                 const int pt = __shfl_sync(0xffffffffu, t, lf);
                 const int pkvh = __shfl_sync(0xffffffffu, kvh, lf);
@@ -347,12 +355,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     float *s_mo = reinterpret_cast<float *>(gbase + P::kOffMergeO);   // [4][kMergeRows][kMergeStride]
     float *s_ml = reinterpret_cast<float *>(gbase + P::kOffMergeML);  // [4][16][2]
 
-    long long u = u0;
-    long long pair = u0 / K;
+    unit_t u = u0;
+    unit_t pair = u0 / K;
     int cursor = 0, seg = 0;
     while (u < u1) {
-        const long long seg_begin = u;
-        const long long seg_end = min(u1, (pair + 1) * K);
+        const unit_t seg_begin = u;
+        const unit_t seg_end = min(u1, (pair + 1) * K);
         const int qs = seg % kSegSlots;
         bool ok = !*s_abort && mbar_wait(sm.qfull(qs), (seg / kSegSlots) & 1, s_abort);
         if (!ok) *s_abort = 1;
@@ -674,7 +682,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 // CTAs covering the pair: closed form from the split, then a
                 // fix-up step in case of rounding
                 // the pair's CTAs are this CTA's neighbours (ranges are contiguous)
-                const long long p_lo = pair * K, p_hi = p_lo + K;
+                const unit_t p_lo = pair * K, p_hi = p_lo + K;
                 int cf = c, cl = c;
                 while (cf > 0 && s_rb[cf] > p_lo) --cf;
                 while (cl + 1 < a.num_ctas && s_rb[cl + 1] < p_hi) ++cl;
@@ -758,7 +766,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         // epoch, which retires this call's ready flags
         named_barrier(1, kConsumerWarps * 32);
         if (tid == 0) {
-            __threadfence();
             const int old = atomic_add_acq_rel_gpu(f.hdr + kHdrDone, 1);
             if (old == (int)gridDim.x - 1) {
                 f.hdr[kHdrAppended] = 0;
