@@ -35,8 +35,10 @@ UNIT = "tokens/s"
 L2_FLUSH_BYTES = 512 << 20
 # DRAM bytes (read + write) per launch of the roofline kernel, from an ncu
 # capture of the current kernel ((workload, path) -> bytes); absent = not
-# captured since the kernel last changed
-TRAFFIC = {}
+# captured since the kernel last changed.  The decode attention figure comes
+# from the 128K-context case, which processes the same units (8 queries x 8 KV
+# heads x 32 selected blocks) and so the same selected bytes per launch.
+TRAFFIC = {("decode_1m", "attention"): 68_428_544}
 
 
 # ----------------------------------------------------------------------------- distributed plumbing

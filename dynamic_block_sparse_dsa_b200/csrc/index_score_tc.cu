@@ -51,11 +51,16 @@ constexpr int kABytes = kBT * kIdxDim;   // 8 KiB
 constexpr int kBBytes = kN * kIdxDim;    // 16 KiB
 // stage: [A 8 KiB][B 16 KiB][info]
 struct StageInfo {
-    int s, bt, y, end;                   // sequence, block tile, query tile; end marker
-    int own[kQT];                        // own block of each query of the tile in s, else -1
+    int bt, y, qslot, end;               // block tile, query tile, its facts slot; end marker
     uint32_t valid[kBT / 32];            // rows with a usable page
-    int w[kQT][kMaxIdxHeads];            // head weights (0 past H and for masked queries)
 };
+// facts of a (query tile, sequence): written once per change into a ring of
+// kQSlots (a slot is rewritten only after every tile using it has finished)
+struct QueryFacts {
+    int own[kQT];                        // own block of each query of the tile in the sequence, else -1
+    int w[kQT][kMaxIdxHeads];            // head weights (0 past H)
+};
+constexpr int kQSlots = 5;               // > kTcStages: see the loader
 constexpr int kOffB = kABytes;
 constexpr int kOffInfo = kABytes + kBBytes;
 constexpr int kStageBytes = (kOffInfo + (int)sizeof(StageInfo) + 1023) / 1024 * 1024;
@@ -65,10 +70,11 @@ constexpr int kNumBars = 2 * kTcStages + 4;
 constexpr int kOffMisc = kOffBars + kNumBars * 8;   // tmem base, abort flag
 constexpr int kCuqCache = 1024;                      // cu_q entries staged in shared memory
 constexpr int kOffCuq = kOffMisc + 16;
+constexpr int kOffFacts = kOffCuq + kCuqCache * 4;   // [kQSlots] QueryFacts (16-byte aligned)
 constexpr int kPidDepth = 4;                         // block tiles of page ids in flight
 // + alignment slack; at least 116 KiB so that two CTAs never share an SM (each
 // holds all 512 tensor-memory columns)
-constexpr int kSmemUsed = kOffCuq + kCuqCache * 4 + 1024;
+constexpr int kSmemUsed = kOffFacts + kQSlots * (int)sizeof(QueryFacts) + 1024;
 constexpr int kSmemBytes = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
 constexpr int kFullCount = kLoadWarps * 33;          // per loader warp: 32 cp.async arrivals + its info arrival
 constexpr int kEmptyCount = 1 + kEpiWarps;           // MMA commit + the epilogue warps
@@ -166,6 +172,10 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
         int cur_y = -1;
         int pos = -1, s_lo = 0, s_hi = -1, len_lo = 0;
         int wv[8];
+        // facts of the current (query tile, sequence): own block of query
+        // lane % 16, the largest of them, and their slot
+        int fy = -1, fs = -1, f_own = -1, f_max = -1, f_len = 0, n_slots = 0, qslot = 0;
+        bool slot_due = false;
         uint32_t err_bits = 0;
         // one item: its sub-items (one per sequence of the query tile) into the ring
         auto process = [&](unsigned it, int pg_pre) {
@@ -185,39 +195,53 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
                 len_lo = __ldg(a.seq_lens + s_lo);
             }
             for (int s = s_lo; s <= s_hi && !*s_abort; ++s) {
-                const int len = s == s_lo ? len_lo : __ldg(a.seq_lens + s);
-                const int t = t0 + (lane & (kQT - 1));
-                int own = -1;
-                if (t < a.total_q && cu(s) <= t && t < cu(s + 1)) {
-                    own = pos / kBlockSize;
-                    if (pos < 0 || pos >= len || own >= a.max_blocks) {
-                        err_bits |= DSA_DEV_ERR_POS;
-                        own = -1;
+                if (y != fy || s != fs) {   // facts of this (query tile, sequence)
+                    fy = y;
+                    fs = s;
+                    f_len = s == s_lo ? len_lo : __ldg(a.seq_lens + s);
+                    const int t = t0 + (lane & (kQT - 1));
+                    f_own = -1;
+                    if (t < a.total_q && cu(s) <= t && t < cu(s + 1)) {
+                        f_own = pos / kBlockSize;
+                        if (pos < 0 || pos >= f_len || f_own >= a.max_blocks) {
+                            err_bits |= DSA_DEV_ERR_POS;
+                            f_own = -1;
+                        }
                     }
+                    f_max = __reduce_max_sync(0xffffffffu, f_own);
+                    slot_due = true;
                 }
-                const int max_own = __reduce_max_sync(0xffffffffu, own);
-                if (max_own < bt * kBT) continue;   // nothing visible in this tile
+                if (f_max < bt * kBT) continue;   // nothing visible in this tile
                 const int st = k % kTcStages;
                 if (k >= kTcStages && !mbar_wait(bars.empty(st), ((k / kTcStages) - 1) & 1, s_abort)) {
                     *s_abort = 1;
                     break;
                 }
+                if (slot_due) {
+                    // slot n_slots % kQSlots was last used by a tile published at
+                    // least kQSlots tiles ago; the empty wait above completed every
+                    // tile up to kTcStages < kQSlots before this one
+                    qslot = n_slots % kQSlots;
+                    ++n_slots;
+                    slot_due = false;
+                    if (lw == 0) {
+                        QueryFacts *qf = reinterpret_cast<QueryFacts *>(g + kOffFacts) + qslot;
+                        if (lane < kQT) qf->own[lane] = f_own;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) (&qf->w[0][0])[lane + 32 * j] = wv[j];
+                    }
+                }
                 uint8_t *stage = g + st * kStageBytes;
                 StageInfo *info = reinterpret_cast<StageInfo *>(stage + kOffInfo);
                 const uint32_t sa = base + st * kStageBytes;
-                if (lw == 0) {
-                    if (lane == 0) { info->end = 0; info->s = s; info->bt = bt; info->y = y; }
-                    if (lane < kQT) info->own[lane] = own;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) (&info->w[0][0])[lane + 32 * j] = wv[j];
-                }
+                if (lw == 0 && lane == 0) { info->end = 0; info->bt = bt; info->y = y; info->qslot = qslot; }
                 // this lane's coarse key: 4 x 16 B, swizzled
                 {
-                    const int n_blocks = (len + kBlockSize - 1) / kBlockSize;
+                    const int n_blocks = (f_len + kBlockSize - 1) / kBlockSize;
                     const int r = 32 * lw + lane;
                     const int b = bt * kBT + r;
                     int page = -1;
-                    if (b < n_blocks && b < a.max_blocks && b <= max_own) {
+                    if (b < n_blocks && b < a.max_blocks && b <= f_max) {
                         page = s == s_lo ? pg_pre : __ldg(a.block_table + (size_t)s * a.max_blocks + b);
                         if (page < 0 || page >= a.num_pages) {
                             err_bits |= DSA_DEV_ERR_PAGE;
@@ -267,7 +291,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
                 *s_abort = 1;
             } else {
                 StageInfo *info = reinterpret_cast<StageInfo *>(g + st * kStageBytes + kOffInfo);
-                if (lw == 0 && lane == 0) { info->end = 1; info->s = -1; }
+                if (lw == 0 && lane == 0) info->end = 1;
                 tc::cp_async_arrive_noinc(bars.full(st));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bars.full(st));
@@ -340,16 +364,17 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
             const StageInfo *info = reinterpret_cast<const StageInfo *>(g + st * kStageBytes + kOffInfo);
             if (info->end) break;
             const int bt = info->bt, y = info->y;
+            const QueryFacts *qf = reinterpret_cast<const QueryFacts *>(g + kOffFacts) + info->qslot;
             const int b = bt * kBT + row;
             const bool row_ok = (info->valid[row >> 5] >> (row & 31)) & 1u;
             const uint32_t taddr =
                 tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kN + qgrp * 64);
             // weights and own blocks of this warp's 4 queries, read as shared-space vectors
-            const uint32_t s_info = base + st * kStageBytes + kOffInfo;
-            const uint32_t s_w = s_info + (uint32_t)offsetof(StageInfo, w) + (uint32_t)(4 * qgrp * kMaxIdxHeads * 4);
+            const uint32_t s_w = base + kOffFacts + (uint32_t)(info->qslot * (int)sizeof(QueryFacts)) +
+                                 (uint32_t)offsetof(QueryFacts, w) + (uint32_t)(4 * qgrp * kMaxIdxHeads * 4);
             int own4[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) own4[u] = info->own[4 * qgrp + u];
+            for (int u = 0; u < 4; ++u) own4[u] = qf->own[4 * qgrp + u];
             uint32_t v[2][32];
             tc::ld_32x32b_x32(taddr, v[0]);
             tc::ld_32x32b_x32(taddr + 32, v[1]);

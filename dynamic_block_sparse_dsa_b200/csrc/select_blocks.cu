@@ -44,7 +44,10 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     const int H = a.num_idx_heads;
 
     pdl_trigger();
-    // ---- query facts: the sequence from a shared-memory copy of cu_q
+    // ---- query facts.  The position and cu_q travel together; then, once the
+    // sequence is known, its length, Top-K and the first group's page ids
+    // travel together: two round trips before the coarse keys
+    const int p = __ldg(a.q_pos + t);
     const bool cached = a.num_seqs + 1 <= kCuqCache;
     if (cached)
         for (int i = tid; i <= a.num_seqs; i += kSelThreads) s_cuq[i] = __ldg(a.cu_q + i);
@@ -64,10 +67,24 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     } else {
         s = find_seq(a.cu_q, a.num_seqs, t);
     }
-    const int p = __ldg(a.q_pos + t);
     const int len = __ldg(a.seq_lens + s);
     const int K = __ldg(a.k_per_seq + s);
     const int n_vis = p / kBlockSize + 1;
+    const int32_t *table = a.block_table + (size_t)s * a.max_blocks;
+    // page ids of this warp's first group, before the facts are checked (the
+    // bound min(own, max_blocks) keeps every load inside the table row)
+    int pg0[4][2];
+    {
+        const int lim = min(n_vis - 1, a.max_blocks);
+        const int base = c * CH + (warp * G) * 64;
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int b = base + 16 * mt + g + 8 * h;
+                pg0[mt][h] = b < lim ? __ldg(table + b) : -1;
+            }
+    }
     int32_t *out = a.sel + (size_t)t * a.k_max;
     bool bad_pos = p < 0 || p >= len || n_vis > a.max_blocks;
     if (a.cu_new && !bad_pos) {
@@ -116,7 +133,6 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
             wl[nt][1] = s_w[8 * nt + 2 * cq + 1];
         }
     }
-    const int32_t *table = a.block_table + (size_t)s * a.max_blocks;
     key64 acc[2] = {0ull, 0ull};
     uint32_t err_bits = 0;
 #pragma unroll 1
@@ -132,7 +148,7 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int b = base + 16 * mt + g + 8 * h;
-                    int page = b < own ? __ldg(table + b) : -1;
+                    int page = b < own ? (gi == 0 ? pg0[mt][h] : __ldg(table + b)) : -1;
                     if (b < own && (page < 0 || page >= a.num_pages)) { err_bits |= DSA_DEV_ERR_PAGE; page = -1; }
                     pg[mt][h] = page;
                 }
