@@ -305,36 +305,58 @@ def run_ours(args, world, rank, device):
     step_roof = {"bytes_per_step": ab["total"], "achieved_gbs": round(step_gbs, 1),
                  "frac_of_measured": round(step_gbs / peak, 4), "frac_of_8tbs": round(step_gbs / 8000.0, 4)}
 
-    # end to end through the public API with host buffers: inputs H2D from
-    # pinned memory, the four calls launched from Python, output D2H
+    # end to end through the public API with host buffers: every step copies
+    # its inputs H2D from pinned memory, runs dsa.step (the four C-ABI calls,
+    # launched from Python) and copies out/lse back D2H; the timed region holds
+    # all of it.  The same step captured once in a CUDA graph (how a serving
+    # loop would launch it) is timed as well and reported beside it.
     host_in = {k: getattr(wl, k).cpu().pin_memory() for k in ("k_new", "v_new", "kc_new", "q", "q_idx", "w")}
     dev_in = {k: getattr(wl, k) for k in host_in}
     host_out = torch.empty(bufs["out"].shape, dtype=bufs["out"].dtype).pin_memory()
     host_lse = torch.empty(bufs["lse"].shape, dtype=bufs["lse"].dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = host_out.numel() * host_out.element_size() + host_lse.numel() * host_lse.element_size()
+
+    def e2e_step():
+        for k, t in host_in.items():
+            dev_in[k].copy_(t, non_blocking=True)
+        dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
+                 q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=spec.k_max, decode=decode,
+                 fused_select=fused, overlap_append=fused and decode, fused_decode=fused_decode,
+                 bufs=bufs, dev_err=err)
+        host_out.copy_(bufs["out"], non_blocking=True)
+        host_lse.copy_(bufs["lse"], non_blocking=True)
+
+    graph_e2e = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_e2e, stream=stream):
+        e2e_step()
+    torch.cuda.synchronize(device)
     e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e2e_ms = []
     n_e2e = max(3, min(args.steps, 50))
-    for i in range(n_e2e + 2):
-        with torch.cuda.stream(stream):
-            cold_l2()
-            e_s.record()
-            for k, t in host_in.items():
-                dev_in[k].copy_(t, non_blocking=True)
-            dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
-                     q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=spec.k_max, decode=decode,
-                     fused_select=fused, overlap_append=fused and decode, fused_decode=fused_decode,
-                     bufs=bufs, dev_err=err)
-            host_out.copy_(bufs["out"], non_blocking=True)
-            host_lse.copy_(bufs["lse"], non_blocking=True)
-            e_e.record()
-        stream.synchronize()
-        if i >= 2:
-            e2e_ms.append(e_s.elapsed_time(e_e))
-    e2e_total = max_over_ranks(sum(e2e_ms) / 1e3, world, device)
-    e2e = {"value": round(weak_scaling_throughput(tokens_per_step, len(e2e_ms), world, e2e_total), 1), "unit": UNIT,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    def time_e2e(run):
+        ms = []
+        for i in range(n_e2e + 2):
+            with torch.cuda.stream(stream):
+                cold_l2()
+                e_s.record()
+                run()
+                e_e.record()
+            stream.synchronize()
+            if i >= 2:
+                ms.append(e_s.elapsed_time(e_e))
+        total = max_over_ranks(sum(ms) / 1e3, world, device)
+        return round(weak_scaling_throughput(tokens_per_step, len(ms), world, total), 1)
+
+    e2e_eager = time_e2e(e2e_step)
+    e2e_graph = time_e2e(graph_e2e.replay)
+    if int(err.item()) != 0:
+        raise RuntimeError(f"device error bits {int(err.item())} in the end-to-end loop")
+    e2e = {"value": e2e_eager, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "how": "dsa.step called from Python every step, H2D input copies and D2H output copies inside the timed region",
+           "graph_value": e2e_graph,
+           "graph_how": "the same copies and calls captured once in a CUDA graph, replayed every step"}
+    del graph_e2e
 
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -235,8 +235,11 @@ int dsa_index_score(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_q
     a.scores = scores;
     a.dev_err = dev_err;
     // prefill-shaped batches (on average a query tile per sequence) run on the
-    // tensor cores; decode-shaped ones scan with dp4a
-    if ((long long)queries->total_q >= (long long)index_score_tc_min_queries_per_seq() * seqs->num_seqs)
+    // tensor cores; decode-shaped ones scan with dp4a (as do batches whose
+    // positions array is not 16-byte aligned: the tensor-core kernel copies it
+    // in 16-byte pieces)
+    if ((long long)queries->total_q >= (long long)index_score_tc_min_queries_per_seq() * seqs->num_seqs &&
+        aligned16(queries->q_pos))
         return from_cuda(launch_index_score_tc(a, sm_count(), reinterpret_cast<cudaStream_t>(stream)));
     return from_cuda(launch_index_score(a, reinterpret_cast<cudaStream_t>(stream)));
 }

@@ -14,23 +14,32 @@
 // are one int8 contraction D[block][(query, head)] (M = 128, N = 256, K = 64),
 // run with tcgen05.mma kind::i8 into a tensor-memory accumulator; the relu,
 // head weights and head sum then happen in the epilogue, one block row per
-// thread, straight from tensor memory.  One persistent CTA per SM, 6 warps:
-//   warp 0   loader: the tile's 128 coarse keys gathered through the block
-//            table (cp.async, 64-byte swizzle; the page ids themselves
-//            copied a few tiles ahead) and the 16 queries' rows (one 3-D TMA
-//            box, heads past H zero-filled), plus the queries' own blocks and
-//            weights, into a 4-stage ring;
-//   warp 1   MMA issuer (one thread): two K=32 MMAs per tile into one of two
-//            256-column accumulators;
-//   warps 2-17 epilogue (four per SM sub-partition: a quarter of the rows and
-//            a quarter of the queries each): tcgen05.ld of the accumulator rows,
-//            relu * w summed over heads, one coalesced 128-byte store per
-//            (query, warp).
-// Tiles are (16-query tile, 128-block tile) pairs in query-tile-major order,
-// split evenly over the CTAs; a tile whose queries belong to several
-// sequences is run once per sequence with the other queries masked.  Tiles
-// past every query's own block are skipped.  All waits are bounded.
+// thread, straight from tensor memory.
+//
+// Work items are (128-block tile, 16-query tile) pairs in block-tile-major
+// order, split evenly over one persistent CTA per SM, so a CTA keeps the same
+// 128 coarse keys (the MMA's A operand, gathered through the block table) for
+// many query tiles.  Per item only asynchronous copies remain: one 3-D TMA box
+// of the 16 queries' rows (heads past H zero-filled) and one 2-D box of their
+// head weights.  Warps:
+//   0     loader.  It works through its items 32 at a time: the batch's query
+//         positions arrive in shared memory a batch ahead (cp.async), every
+//         lane then decides one item (its sequences, whether any of its blocks
+//         is visible), and a short loop publishes the visible items into a
+//         4-stage ring.  When the (sequence, block tile) changes it gathers the
+//         new tile (64-byte swizzle) into one of two A buffers, once the items
+//         still reading that buffer have finished;
+//   1     MMA issuer (one thread): two K = 32 MMAs per item into one of two
+//         256-column accumulators;
+//   2-17  epilogue (four per SM sub-partition: a quarter of the rows and a
+//         quarter of the queries each): tcgen05.ld, relu * w summed over heads,
+//         one coalesced 128-byte store per (query, warp).
+// A query tile spanning several sequences runs once per sequence with the
+// other queries masked; items past every query's own block are skipped.  All
+// waits are bounded.
+#include <climits>
 #include <cstddef>
+#include <cstdint>
 
 #include "dsa_kernels.h"
 #include "dsa_tcgen05.cuh"
@@ -39,47 +48,51 @@ namespace dsa {
 
 namespace {
 constexpr int kEpiWarps = 16;                      // four per SM sub-partition
-constexpr int kLoadWarps = 4;                      // one gathered row per lane
-constexpr int kMmaWarp = kLoadWarps;
-constexpr int kEpiWarp0 = kLoadWarps + 1;
-constexpr int kTcThreads = 32 * (kLoadWarps + 1 + kEpiWarps);   // loaders, MMA, epilogue
+constexpr int kLoadWarp = 0;
+constexpr int kMmaWarp = 1;
+constexpr int kEpiWarp0 = 2;
+constexpr int kTcThreads = 32 * (2 + kEpiWarps);   // loader, MMA, epilogue
 constexpr int kTcStages = 4;
 constexpr int kBT = 128;                 // blocks per tile (MMA M)
 constexpr int kQT = 16;                  // queries per tile (MMA N = 16 x 16 heads)
 constexpr int kN = kQT * kMaxIdxHeads;   // 256
 constexpr int kABytes = kBT * kIdxDim;   // 8 KiB
 constexpr int kBBytes = kN * kIdxDim;    // 16 KiB
-// stage: [A 8 KiB][B 16 KiB][info]
+// stage: [B 16 KiB][weights 16 x 16 int32][info]
 struct StageInfo {
-    int bt, y, qslot, end;               // block tile, query tile, its facts slot; end marker
-    uint32_t valid[kBT / 32];            // rows with a usable page
+    int bt, y, abuf, agen;               // block tile, query tile, A buffer and its fill number
+    int end, pad[3];                     // end marker
+    int own[kQT];                        // own block of each query of the tile in this sequence, else -1
 };
-// facts of a (query tile, sequence): written once per change into a ring of
-// kQSlots (a slot is rewritten only after every tile using it has finished)
-struct QueryFacts {
-    int own[kQT];                        // own block of each query of the tile in the sequence, else -1
-    int w[kQT][kMaxIdxHeads];            // head weights (0 past H)
-};
-constexpr int kQSlots = 5;               // > kTcStages: see the loader
-constexpr int kOffB = kABytes;
-constexpr int kOffInfo = kABytes + kBBytes;
+constexpr int kOffW = kBBytes;
+constexpr int kOffInfo = kOffW + kQT * kMaxIdxHeads * 4;
 constexpr int kStageBytes = (kOffInfo + (int)sizeof(StageInfo) + 1023) / 1024 * 1024;
-constexpr int kOffBars = kTcStages * kStageBytes;
-// barriers: full[S], empty[S], tfull[2], tempty[2]
-constexpr int kNumBars = 2 * kTcStages + 4;
-constexpr int kOffMisc = kOffBars + kNumBars * 8;   // tmem base, abort flag
-constexpr int kCuqCache = 1024;                      // cu_q entries staged in shared memory
-constexpr int kOffCuq = kOffMisc + 16;
-constexpr int kOffFacts = kOffCuq + kCuqCache * 4;   // [kQSlots] QueryFacts (16-byte aligned)
-constexpr int kPidDepth = 4;                         // block tiles of page ids in flight
+constexpr int kOffA = kTcStages * kStageBytes;           // [2][kABytes], 1 KiB aligned
+constexpr int kOffAValid = kOffA + 2 * kABytes;          // [2][kBT / 32] rows with a usable page
+constexpr int kOffBars = kOffAValid + 2 * (kBT / 32) * 4;
+// barriers: full[S], empty[S], tfull[2], tempty[2], afull[2]
+constexpr int kNumBars = 2 * kTcStages + 6;
+constexpr int kOffMisc = kOffBars + kNumBars * 8;   // tmem base, abort, never
+constexpr int kOffDone = kOffMisc + 16;              // items finished, per epilogue warp
+constexpr int kSeqCache = 1024;                      // cu_q and seq_lens entries staged in shared memory
+constexpr int kOffCuq = kOffDone + 4 * kEpiWarps;    // [kSeqCache] cu_q, then [kSeqCache] seq_lens
+constexpr int kBatch = 32;                           // items decided together, one per lane
+constexpr int kOffPos = kOffCuq + 2 * kSeqCache * 4; // [2][kBatch][kQT] int32 query positions
+constexpr int kWBytes = kQT * kMaxIdxHeads * 4;      // one tile's head weights
 // + alignment slack; at least 116 KiB so that two CTAs never share an SM (each
 // holds all 512 tensor-memory columns)
-constexpr int kSmemUsed = kOffFacts + kQSlots * (int)sizeof(QueryFacts) + 1024;
+constexpr int kSmemUsed = kOffPos + 2 * kBatch * kQT * 4 + 1024;
 constexpr int kSmemBytes = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
-constexpr int kFullCount = kLoadWarps * 33;          // per loader warp: 32 cp.async arrivals + its info arrival
+// full barrier: the loader's arrival with the TMA bytes, plus 32 cp.async
+// arrivals when the weights are copied by cp.async (H not a multiple of 4)
+constexpr int kFullCountTma = 1;
+constexpr int kFullCountCpAsync = 33;
+constexpr int kAFullCount = 33;                      // the loader: 32 cp.async arrivals + one
 constexpr int kEmptyCount = 1 + kEpiWarps;           // MMA commit + the epilogue warps
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kOffA % 1024 == 0, "A buffers keep the 64-byte swizzle's 512-byte alignment");
+static_assert(kOffPos % 16 == 0, "positions are copied and read in 16-byte pieces");
 
 struct Bars {
     uint32_t base;
@@ -87,34 +100,50 @@ struct Bars {
     __device__ uint32_t empty(int s) const { return base + kOffBars + 8 * (kTcStages + s); }
     __device__ uint32_t tfull(int b) const { return base + kOffBars + 8 * (2 * kTcStages + b); }
     __device__ uint32_t tempty(int b) const { return base + kOffBars + 8 * (2 * kTcStages + 2 + b); }
+    __device__ uint32_t afull(int b) const { return base + kOffBars + 8 * (2 * kTcStages + 4 + b); }
 };
 
 __device__ __forceinline__ int seq_of_query(const IndexScoreArgs &a, int t) { return find_seq(a.cu_q, a.num_seqs, t); }
+
+// 4-byte asynchronous copy global -> shared (zero-filled when !valid)
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src, bool valid) {
+    if (valid) asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(dst), "l"(src) : "memory");
+    else asm volatile("cp.async.ca.shared.global [%0], [%1], 4, 0;\n" ::"r"(dst), "l"(src) : "memory");
+}
+// 16-byte asynchronous copy of which the first `nbytes` are read, the rest zero-filled
+__device__ __forceinline__ void cp_async_16_n(uint32_t dst, const void *src, int nbytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(nbytes) : "memory");
+}
 }  // namespace
 
 __global__ void __launch_bounds__(kTcThreads, 1)
-index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a, int n_bt, int n_qt) {
+index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_w,
+                      IndexScoreArgs a, int n_bt, int n_qt, int w_tma) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *g = smem_raw + (base - raw);
     Bars bars{base};
-    volatile int *misc = reinterpret_cast<volatile int *>(g + kOffMisc);   // [0] tmem base, [1] abort, [2] never
+    // [0] tmem base, [1] abort, [2] never set
+    volatile int *misc = reinterpret_cast<volatile int *>(g + kOffMisc);
+    volatile int *s_done = reinterpret_cast<volatile int *>(g + kOffDone);
     volatile int *s_abort = misc + 1;
     const volatile int *s_never = misc + 2;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
         for (int s = 0; s < kTcStages; ++s) {
-            mbar_init(bars.full(s), kFullCount);
+            mbar_init(bars.full(s), w_tma ? kFullCountTma : kFullCountCpAsync);
             mbar_init(bars.empty(s), kEmptyCount);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bars.tfull(b), 1);
             mbar_init(bars.tempty(b), kEpiWarps);
+            mbar_init(bars.afull(b), kAFullCount);
         }
         misc[1] = 0;
         misc[2] = 0;
+        for (int e = 0; e < kEpiWarps; ++e) s_done[e] = 0;
         fence_barrier_init();
     }
     if (warp == kMmaWarp) {
@@ -133,22 +162,22 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
     const unsigned i1 = (unsigned)((unsigned long long)n_items * (blockIdx.x + 1) / gridDim.x);
     const int H = a.num_idx_heads;
 
-    if (warp < kLoadWarps) {
-        // ============================================================ loaders
-        const int lw = warp;   // rows 32*lw .. 32*lw+31 of every tile
-        // Items are (query tile y, block tile bt), y-major: the queries'
-        // positions and weights change once per query tile, the coarse keys
-        // every item.  The page ids of item j are loaded into a register ring
-        // kPidDepth items ahead, so the gather of item j never waits on a
-        // global load; its keys then land through the stage's full barrier.
-        if (lw == 0 && lane == 0) prefetch_tensormap(&tm_q);
+    if (warp == kLoadWarp) {
+        // ============================================================ loader
+        if (lane == 0) {
+            prefetch_tensormap(&tm_q);
+            if (w_tma) prefetch_tensormap(&tm_w);
+        }
         int *s_cuq = reinterpret_cast<int *>(g + kOffCuq);
-        const bool cuq_cached = a.num_seqs + 1 <= kCuqCache;
-        if (cuq_cached)
-            for (int i = lane + 32 * lw; i <= a.num_seqs; i += 32 * kLoadWarps) s_cuq[i] = __ldg(a.cu_q + i);
-        named_barrier(1, 32 * kLoadWarps);
+        int *s_len = s_cuq + kSeqCache;
+        const bool cached = a.num_seqs + 1 <= kSeqCache;
+        if (cached) {
+            for (int i = lane; i <= a.num_seqs; i += 32) s_cuq[i] = __ldg(a.cu_q + i);
+            for (int i = lane; i < a.num_seqs; i += 32) s_len[i] = __ldg(a.seq_lens + i);
+        }
+        __syncwarp();
         auto seq_of = [&](int t) {
-            if (!cuq_cached) return seq_of_query(a, t);
+            if (!cached) return seq_of_query(a, t);
             int lo = 0, hi = a.num_seqs - 1;
             while (lo < hi) {
                 const int mid = (lo + hi + 1) >> 1;
@@ -156,143 +185,206 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
             }
             return lo;
         };
-        auto cu = [&](int s) { return cuq_cached ? s_cuq[s] : __ldg(a.cu_q + s); };
-        // page id of this lane's row of item j (first sequence of its tile)
-        auto load_pid = [&](unsigned j) {
-            const int y = (int)(j / (unsigned)n_bt), bt = (int)(j - (unsigned)y * (unsigned)n_bt);
-            const int s0 = seq_of(kQT * y);
-            const int b = bt * kBT + 32 * lw + lane;
-            return b < a.max_blocks ? __ldg(a.block_table + (size_t)s0 * a.max_blocks + b) : -1;
+        auto cu = [&](int s) { return cached ? s_cuq[s] : __ldg(a.cu_q + s); };
+        auto seq_len = [&](int s) { return cached ? s_len[s] : __ldg(a.seq_lens + s); };
+        // the query positions of items b0 .. b0+31 into buffer `buf` (16 bytes
+        // per copy, zero past the last query); one commit group per batch
+        int *s_posb = reinterpret_cast<int *>(g + kOffPos);
+        const uint32_t s_posb_u32 = smem_u32(s_posb);
+        auto fetch_batch = [&](unsigned b0, int buf) {
+#pragma unroll
+            for (int c = lane; c < kBatch * 4; c += 32) {
+                const unsigned j = b0 + (unsigned)(c >> 2);
+                if (j < i1) {
+                    const unsigned bt = j / (unsigned)n_qt;
+                    const int t = kQT * (int)(j - bt * (unsigned)n_qt) + 4 * (c & 3);
+                    const int n = min(max(a.total_q - t, 0), 4);
+                    cp_async_16_n(s_posb_u32 + (uint32_t)(((buf * kBatch + (c >> 2)) * kQT + 4 * (c & 3)) * 4),
+                                  a.q_pos + (n > 0 ? t : 0), 4 * n);
+                }
+            }
+            cp_async_commit();
         };
         pdl_wait();   // coarse keys may come from the preceding append
-        int ring[kPidDepth];
-#pragma unroll
-        for (int d = 0; d < kPidDepth; ++d) ring[d] = i0 + d < i1 ? load_pid(i0 + d) : -1;
-        int k = 0;    // stages published
-        int cur_y = -1;
-        int pos = -1, s_lo = 0, s_hi = -1, len_lo = 0;
-        int wv[8];
-        // facts of the current (query tile, sequence): own block of query
-        // lane % 16, the largest of them, and their slot
-        int fy = -1, fs = -1, f_own = -1, f_max = -1, f_len = 0, n_slots = 0, qslot = 0;
-        bool slot_due = false;
+        fetch_batch(i0, 0);
+        fetch_batch(i0 + kBatch, 1);
+        int k = 0;          // items published
+        int a_s = -1, a_bt = -1, ab = 1;
+        int agen0 = 0, agen1 = 0, alast0 = -1, alast1 = -1;   // per A buffer: fill number, last item
         uint32_t err_bits = 0;
-        // one item: its sub-items (one per sequence of the query tile) into the ring
-        auto process = [&](unsigned it, int pg_pre) {
-            const int y = (int)(it / (unsigned)n_bt), bt = (int)(it - (unsigned)y * (unsigned)n_bt);
-            const int t0 = kQT * y;
-            if (y != cur_y) {   // a new query tile: positions, weights, sequences
-                cur_y = y;
+        bool stop = false;
+        int pbuf = 0;
+        for (unsigned b0 = i0; b0 < i1 && !stop; b0 += kBatch, pbuf ^= 1) {
+            cp_async_wait<1>();   // this batch's positions (the next batch may still be in flight)
+            __syncwarp();
+            const int *posb = s_posb + pbuf * kBatch * kQT;
+            // ---- decisions: lane L takes item b0 + L
+            int d_bt = 0, d_y = 0, d_slo = 0, d_shi = -1, d_len = 0, d_vis = 0;
+            {
+                const unsigned my = b0 + (unsigned)lane;
+                if (my < i1) {
+                    d_bt = (int)(my / (unsigned)n_qt);
+                    d_y = (int)(my - (unsigned)d_bt * (unsigned)n_qt);
+                    const int t0 = kQT * d_y, tn = min(t0 + kQT, a.total_q);
+                    d_slo = seq_of(t0);
+                    d_shi = seq_of(tn - 1);
+                    if (d_slo == d_shi) {
+                        // one sequence: visible when a member's own block reaches the tile
+                        d_len = seq_len(d_slo);
+                        const int4 *pp = reinterpret_cast<const int4 *>(posb + lane * kQT);
+                        int mx = -1;
+                        bool bad = false;
+                        auto take = [&](int pos, int t) {
+                            if (t < tn) {
+                                const int own = pos / kBlockSize;
+                                if (pos < 0 || pos >= d_len || own >= a.max_blocks) bad = true;
+                                else mx = max(mx, own);
+                            }
+                        };
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const int4 p = pp[v];
+                            take(p.x, t0 + 4 * v);
+                            take(p.y, t0 + 4 * v + 1);
+                            take(p.z, t0 + 4 * v + 2);
+                            take(p.w, t0 + 4 * v + 3);
+                        }
+                        if (bad) err_bits |= DSA_DEV_ERR_POS;
+                        d_vis = mx >= d_bt * kBT;
+                    } else {
+                        d_vis = 1;   // several sequences: decided per sequence below
+                    }
+                }
+            }
+            // ---- publish the batch's visible items in order
+            const int n_here = (int)min((unsigned)kBatch, i1 - b0);
+            for (int i = 0; i < n_here && !stop; ++i) {
+                if (!__shfl_sync(0xffffffffu, d_vis, i)) continue;
+                const int bt = __shfl_sync(0xffffffffu, d_bt, i);
+                const int y = __shfl_sync(0xffffffffu, d_y, i);
+                const int s_lo = __shfl_sync(0xffffffffu, d_slo, i);
+                const int s_hi = __shfl_sync(0xffffffffu, d_shi, i);
+                const int len_lo = __shfl_sync(0xffffffffu, d_len, i);
+                const bool single = s_lo == s_hi;
+                const int t0 = kQT * y;
                 const int t = t0 + (lane & (kQT - 1));
-                pos = t < a.total_q ? __ldg(a.q_pos + t) : -1;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int e = lane + 32 * j, qi = e / kMaxIdxHeads, h = e % kMaxIdxHeads;
-                    wv[j] = (t0 + qi < a.total_q && h < H) ? __ldg(a.w + (size_t)(t0 + qi) * H + h) : 0;
-                }
-                s_lo = seq_of(t0);
-                s_hi = seq_of(min(t0 + kQT, a.total_q) - 1);
-                len_lo = __ldg(a.seq_lens + s_lo);
-            }
-            for (int s = s_lo; s <= s_hi && !*s_abort; ++s) {
-                if (y != fy || s != fs) {   // facts of this (query tile, sequence)
-                    fy = y;
-                    fs = s;
-                    f_len = s == s_lo ? len_lo : __ldg(a.seq_lens + s);
-                    const int t = t0 + (lane & (kQT - 1));
-                    f_own = -1;
-                    if (t < a.total_q && cu(s) <= t && t < cu(s + 1)) {
-                        f_own = pos / kBlockSize;
-                        if (pos < 0 || pos >= f_len || f_own >= a.max_blocks) {
+                const int pos = posb[i * kQT + (lane & (kQT - 1))];
+                for (int s = s_lo; s <= s_hi; ++s) {
+                    const int len = single ? len_lo : seq_len(s);
+                    int own = -1;
+                    if (t < a.total_q && (single || (cu(s) <= t && t < cu(s + 1)))) {
+                        own = pos / kBlockSize;
+                        if (pos < 0 || pos >= len || own >= a.max_blocks) {
                             err_bits |= DSA_DEV_ERR_POS;
-                            f_own = -1;
+                            own = -1;
                         }
                     }
-                    f_max = __reduce_max_sync(0xffffffffu, f_own);
-                    slot_due = true;
-                }
-                if (f_max < bt * kBT) continue;   // nothing visible in this tile
-                const int st = k % kTcStages;
-                if (k >= kTcStages && !mbar_wait(bars.empty(st), ((k / kTcStages) - 1) & 1, s_abort)) {
-                    *s_abort = 1;
-                    break;
-                }
-                if (slot_due) {
-                    // slot n_slots % kQSlots was last used by a tile published at
-                    // least kQSlots tiles ago; the empty wait above completed every
-                    // tile up to kTcStages < kQSlots before this one
-                    qslot = n_slots % kQSlots;
-                    ++n_slots;
-                    slot_due = false;
-                    if (lw == 0) {
-                        QueryFacts *qf = reinterpret_cast<QueryFacts *>(g + kOffFacts) + qslot;
-                        if (lane < kQT) qf->own[lane] = f_own;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) (&qf->w[0][0])[lane + 32 * j] = wv[j];
-                    }
-                }
-                uint8_t *stage = g + st * kStageBytes;
-                StageInfo *info = reinterpret_cast<StageInfo *>(stage + kOffInfo);
-                const uint32_t sa = base + st * kStageBytes;
-                if (lw == 0 && lane == 0) { info->end = 0; info->bt = bt; info->y = y; info->qslot = qslot; }
-                // this lane's coarse key: 4 x 16 B, swizzled
-                {
-                    const int n_blocks = (f_len + kBlockSize - 1) / kBlockSize;
-                    const int r = 32 * lw + lane;
-                    const int b = bt * kBT + r;
-                    int page = -1;
-                    if (b < n_blocks && b < a.max_blocks && b <= f_max) {
-                        page = s == s_lo ? pg_pre : __ldg(a.block_table + (size_t)s * a.max_blocks + b);
-                        if (page < 0 || page >= a.num_pages) {
-                            err_bits |= DSA_DEV_ERR_PAGE;
-                            page = -1;
+                    if (!single && __reduce_max_sync(0xffffffffu, own) < bt * kBT) continue;   // nothing visible
+                    if (s != a_s || bt != a_bt) {
+                        // a new block tile: into the other A buffer once the items
+                        // still reading it have all finished
+                        a_s = s;
+                        a_bt = bt;
+                        ab ^= 1;
+                        const int last = ab ? alast1 : alast0;
+                        if (last >= 0) {
+                            const long long t_start = clock64();
+                            while (__reduce_min_sync(0xffffffffu, lane < kEpiWarps ? s_done[lane] : INT_MAX) <=
+                                   last) {
+                                if (*s_abort || clock64() - t_start > kWaitLimitCycles) {
+                                    *s_abort = 1;
+                                    stop = true;
+                                    break;
+                                }
+                                __nanosleep(64);
+                            }
+                            if (stop) break;
                         }
-                    }
-                    const uint32_t bits = __ballot_sync(0xffffffffu, page >= 0);
-                    if (lane == 0) info->valid[lw] = bits;
-                    const int8_t *src = a.kc_pool + (size_t)max(page, 0) * kIdxDim;
+                        if (ab) ++agen1; else ++agen0;
+                        const int n_blocks = (len + kBlockSize - 1) / kBlockSize;
+                        const int32_t *row = a.block_table + (size_t)s * a.max_blocks;
+                        int page[kBT / 32];
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint32_t dst = sa + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
-                        if (page >= 0) cp_async_16(dst, src + 16 * c);
-                        else cp_async_16_zero(dst, a.kc_pool);
-                    }
-                }
-                // the queries' rows: box (64 B, 16 heads, 16 queries) at query t0
-                if (lw == 0 && lane == 0) {
-                    tc::mbar_expect_tx(bars.full(st), kBBytes);
-                    tma_load_3d(sa + kOffB, &tm_q, 0, 0, t0, bars.full(st));
-                }
-                tc::cp_async_arrive_noinc(bars.full(st));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bars.full(st));   // the info words above
-                ++k;
-            }
-        };
-        // the item loop, unrolled by the ring depth so that every ring slot is a
-        // fixed register: slot d is read for item base + d and refilled with
-        // the page id of item base + d + kPidDepth, which is read kPidDepth
-        // items later -- no register copy ever waits on a load in flight
-        for (unsigned base0 = i0; base0 < i1 && !*s_abort; base0 += kPidDepth) {
+                        for (int j = 0; j < kBT / 32; ++j) {   // rows 32 j + lane
+                            const int b = bt * kBT + 32 * j + lane;
+                            page[j] = b < n_blocks && b < a.max_blocks ? __ldg(row + b) : -1;
+                        }
+                        const uint32_t sa = base + kOffA + ab * kABytes;
+                        uint32_t *vbits = reinterpret_cast<uint32_t *>(g + kOffAValid) + ab * (kBT / 32);
 #pragma unroll
-            for (int d = 0; d < kPidDepth; ++d) {
-                const unsigned it = base0 + d;
-                if (it < i1 && !*s_abort) {
-                    const int pg_pre = ring[d];
-                    ring[d] = it + kPidDepth < i1 ? load_pid(it + kPidDepth) : -1;
-                    process(it, pg_pre);
+                        for (int j = 0; j < kBT / 32; ++j) {
+                            const int b = bt * kBT + 32 * j + lane;
+                            if (b < n_blocks && b < a.max_blocks && (page[j] < 0 || page[j] >= a.num_pages)) {
+                                err_bits |= DSA_DEV_ERR_PAGE;
+                                page[j] = -1;
+                            }
+                            const uint32_t bits = __ballot_sync(0xffffffffu, page[j] >= 0);
+                            if (lane == 0) vbits[j] = bits;
+                            const int r = 32 * j + lane;
+                            const int8_t *src = a.kc_pool + (size_t)max(page[j], 0) * kIdxDim;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const uint32_t dst = sa + r * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+                                if (page[j] >= 0) cp_async_16(dst, src + 16 * c);
+                                else cp_async_16_zero(dst, a.kc_pool);
+                            }
+                        }
+                        tc::cp_async_arrive_noinc(bars.afull(ab));
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bars.afull(ab));
+                    }
+                    if (ab) alast1 = k; else alast0 = k;
+                    const int st = k & (kTcStages - 1);
+                    if (k >= kTcStages && !mbar_wait(bars.empty(st), ((k / kTcStages) - 1) & 1, s_abort)) {
+                        *s_abort = 1;
+                        stop = true;
+                        break;
+                    }
+                    StageInfo *info = reinterpret_cast<StageInfo *>(g + st * kStageBytes + kOffInfo);
+                    const uint32_t sb = base + st * kStageBytes;
+                    if (lane == 0) {
+                        info->end = 0;
+                        info->bt = bt;
+                        info->y = y;
+                        info->abuf = ab;
+                        info->agen = ab ? agen1 : agen0;
+                    }
+                    if (lane < kQT) info->own[lane] = own;
+                    if (!w_tma) {
+                        // the tile's head weights (16 queries x 16 heads, zero past H and the last query)
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const int e = lane + 32 * j, qi = e / kMaxIdxHeads, h = e % kMaxIdxHeads;
+                            const bool ok = t0 + qi < a.total_q && h < H;
+                            cp_async_4(sb + kOffW + 4 * e, a.w + (ok ? (size_t)(t0 + qi) * H + h : 0), ok);
+                        }
+                        tc::cp_async_arrive_noinc(bars.full(st));
+                    }
+                    __syncwarp();   // the info words above, before the release arrival
+                    if (lane == 0) {
+                        // the queries' rows: box (64 B, 16 heads, 16 queries) at query t0, and
+                        // their weights: box (16 heads, 16 queries), zero past H and the last query
+                        mbar_arrive_expect_tx(bars.full(st), kBBytes + (w_tma ? kWBytes : 0));
+                        tma_load_3d(sb, &tm_q, 0, 0, t0, bars.full(st));
+                        if (w_tma) tma_load_2d(sb + kOffW, &tm_w, 0, t0, bars.full(st));
+                    }
+                    ++k;
                 }
             }
+            // every lane is done with this batch's positions: refill the buffer
+            __syncwarp();
+            fetch_batch(b0 + 2 * kBatch, pbuf);
+            if (*s_abort) stop = true;
         }
         // the end marker
-        if (!*s_abort) {
-            const int st = k % kTcStages;
+        if (!stop && !*s_abort) {
+            const int st = k & (kTcStages - 1);
             if (k >= kTcStages && !mbar_wait(bars.empty(st), ((k / kTcStages) - 1) & 1, s_abort)) {
                 *s_abort = 1;
             } else {
                 StageInfo *info = reinterpret_cast<StageInfo *>(g + st * kStageBytes + kOffInfo);
-                if (lw == 0 && lane == 0) info->end = 1;
-                tc::cp_async_arrive_noinc(bars.full(st));
+                if (lane == 0) info->end = 1;
+                if (!w_tma) tc::cp_async_arrive_noinc(bars.full(st));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bars.full(st));
                 ++k;
@@ -302,7 +394,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
         if (lane == 0 && err_bits) set_err(a.dev_err, err_bits);
         cp_async_commit();
         cp_async_wait<0>();
-        if (*s_abort && lw == 0 && lane == 0) {
+        if (*s_abort && lane == 0) {
             set_err(a.dev_err, DSA_DEV_ERR_WAIT);
             for (int j = max(0, k - kTcStages); j < k; ++j)
                 mbar_wait(bars.full(j % kTcStages), (j / kTcStages) & 1, s_never);
@@ -314,22 +406,26 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
         while (true) {
             const int st = k % kTcStages, buf = k & 1;
             bool ok = mbar_wait(bars.full(st), (k / kTcStages) & 1, s_abort);
+            const StageInfo *info = reinterpret_cast<const StageInfo *>(g + st * kStageBytes + kOffInfo);
+            const bool end = ok && info->end != 0;
+            if (ok && !end) ok = mbar_wait(bars.afull(info->abuf), (info->agen - 1) & 1, s_abort);
+            // the accumulator's previous item has been read (the end marker's
+            // arrival on tfull must not run two phases ahead of the epilogue)
             if (ok && k >= 2) ok = mbar_wait(bars.tempty(buf), ((k >> 1) - 1) & 1, s_abort);
             if (!ok) {
                 if (lane == 0) *s_abort = 1;
                 break;
             }
-            const StageInfo *info = reinterpret_cast<const StageInfo *>(g + st * kStageBytes + kOffInfo);
-            const bool end = info->end != 0;
             if (lane == 0) {
                 if (end) {
                     mbar_arrive(bars.tfull(buf));   // wake the epilogue to see the end marker
                 } else {
                     tc::fence_proxy_async_smem();   // the cp.async-written keys, for the tensor core
                     tc::fence_after_sync();
-                    const uint32_t sa = base + st * kStageBytes;
+                    const uint32_t sa = base + kOffA + info->abuf * kABytes;
+                    const uint32_t sb = base + st * kStageBytes;
                     const uint32_t d = tmem + (uint32_t)(buf * kN);
-                    const uint64_t da = tc::smem_desc_k64_sw64(sa), db = tc::smem_desc_k64_sw64(sa + kOffB);
+                    const uint64_t da = tc::smem_desc_k64_sw64(sa), db = tc::smem_desc_k64_sw64(sb);
                     tc::mma_i8(d, da, db, idesc, false);
                     tc::mma_i8(d, da + (32 >> 4), db + (32 >> 4), idesc, true);   // K bytes 32..63
                     tc::commit(bars.empty(st));
@@ -363,18 +459,22 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
             tc::fence_after_sync();
             const StageInfo *info = reinterpret_cast<const StageInfo *>(g + st * kStageBytes + kOffInfo);
             if (info->end) break;
+            // acquire the A buffer's valid bits (cannot be refilled before this warp finishes the item)
+            if (!mbar_wait(bars.afull(info->abuf), (info->agen - 1) & 1, s_abort)) {
+                if (lane == 0) *s_abort = 1;
+                break;
+            }
             const int bt = info->bt, y = info->y;
-            const QueryFacts *qf = reinterpret_cast<const QueryFacts *>(g + kOffFacts) + info->qslot;
             const int b = bt * kBT + row;
-            const bool row_ok = (info->valid[row >> 5] >> (row & 31)) & 1u;
+            const uint32_t vbits = reinterpret_cast<const uint32_t *>(g + kOffAValid)[info->abuf * (kBT / 32) + (row >> 5)];
+            const bool row_ok = (vbits >> (row & 31)) & 1u;
             const uint32_t taddr =
                 tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kN + qgrp * 64);
-            // weights and own blocks of this warp's 4 queries, read as shared-space vectors
-            const uint32_t s_w = base + kOffFacts + (uint32_t)(info->qslot * (int)sizeof(QueryFacts)) +
-                                 (uint32_t)offsetof(QueryFacts, w) + (uint32_t)(4 * qgrp * kMaxIdxHeads * 4);
+            // weights (shared-space vector loads) and own blocks of this warp's 4 queries
+            const uint32_t s_w = base + st * kStageBytes + kOffW + (uint32_t)(4 * qgrp * kMaxIdxHeads * 4);
             int own4[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) own4[u] = qf->own[4 * qgrp + u];
+            for (int u = 0; u < 4; ++u) own4[u] = info->own[4 * qgrp + u];
             uint32_t v[2][32];
             tc::ld_32x32b_x32(taddr, v[0]);
             tc::ld_32x32b_x32(taddr + 32, v[1]);
@@ -401,6 +501,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, IndexScoreArgs a
             if (lane == 0) {
                 mbar_arrive(bars.tempty(buf));
                 mbar_arrive(bars.empty(st));
+                __threadfence_block();
+                s_done[ew] = k + 1;   // lets the loaders refill the A buffer
             }
             ++k;
         }
@@ -448,6 +550,21 @@ cudaError_t launch_index_score_tc(const IndexScoreArgs &a, int num_sms, cudaStre
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+    // head weights as (head, query) int32 boxes of 16 x 16 when a row is a whole
+    // number of 16-byte units (H % 4 == 0) and the base is 16-byte aligned;
+    // otherwise the kernel copies them with cp.async
+    CUtensorMap tw = tq;
+    int w_tma = 0;
+    if (a.num_idx_heads % 4 == 0 && (reinterpret_cast<uintptr_t>(a.w) & 15) == 0) {
+        const cuuint64_t wdims[2] = {(cuuint64_t)a.num_idx_heads, (cuuint64_t)a.total_q};
+        const cuuint64_t wstrides[1] = {(cuuint64_t)a.num_idx_heads * 4};
+        const cuuint32_t wbox[2] = {kMaxIdxHeads, kQT};
+        const cuuint32_t westr[2] = {1, 1};
+        if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, const_cast<int32_t *>(a.w), wdims, wstrides, wbox, westr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            w_tma = 1;
+    }
     static unsigned long long attr_done = 0;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -458,12 +575,12 @@ cudaError_t launch_index_score_tc(const IndexScoreArgs &a, int num_sms, cudaStre
         if (dev < 64) attr_done |= 1ull << dev;
     }
     const int n_bt = (a.max_blocks + kBT - 1) / kBT;
-    const int n_qt = (a.total_q + kQT - 1) / kQT;   // items (y, bt), y-major
+    const int n_qt = (a.total_q + kQT - 1) / kQT;   // items (bt, y), block-tile-major
     const long long items = (long long)n_bt * n_qt;
     if (items >= (1LL << 31)) return cudaErrorInvalidValue;   // item indices are 32-bit in the kernel
     const int grid = (int)(items < num_sms ? items : num_sms);
-    return launch_pdl(index_score_tc_kernel, dim3(grid), dim3(kTcThreads), (size_t)kSmemBytes, stream, tq, a, n_bt,
-                      n_qt);
+    return launch_pdl(index_score_tc_kernel, dim3(grid), dim3(kTcThreads), (size_t)kSmemBytes, stream, tq, tw, a, n_bt,
+                      n_qt, w_tma);
 }
 
 }  // namespace dsa

@@ -128,8 +128,11 @@ int dsa_kv_append(const dsa_kv_cache *cache, const dsa_seqs *seqs, const int32_t
  *   scores int32 [total_q][max_blocks]: entries b <= q_pos[t]/block_size are
  *          written, the rest of the row is left untouched.
  * DSA_ERR_RANGE when num_idx_heads * w_abs_max * idx_dim * 128 * 128 >= 2^31
- * (an int32 result could overflow).  One CTA scores 256 blocks of one
- * sequence for all of its queries with dp4a on the CUDA cores.
+ * (an int32 result could overflow).  Batches with at least 16 queries per
+ * sequence on average (prefill) run as int8 tensor-core tiles of 128 blocks x
+ * 16 queries (tcgen05, one persistent CTA per SM) when q_pos is 16-byte
+ * aligned; the others (decode) scan 256 blocks of one sequence per CTA with
+ * dp4a on the CUDA cores.  Both write identical scores.
  * Device errors: DSA_DEV_ERR_PAGE, DSA_DEV_ERR_POS.
  */
 int dsa_index_score(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,

@@ -86,8 +86,9 @@ SMALL = {
     # (odd Top-K: unequal halves; short sequences: one half without usable blocks)
     "cluster_pairs": dict(seq_lens=tuple(range(70, 70 + 24 * 431, 431)), n_new=(1,) * 24, k_per_seq=(7,) * 24,
                           k_max=7),
-    # fewer indexer heads than the 16 of a tensor-core tile
+    # fewer indexer heads than the 16 of a tensor-core tile (5: weights by cp.async, 8: by TMA)
     "prefill_5_idx_heads": dict(seq_lens=(20000,), n_new=(100,), k_per_seq=(10,), k_max=10, num_idx_heads=5),
+    "prefill_8_idx_heads": dict(seq_lens=(5000, 3000), n_new=(40, 25), k_per_seq=(6, 5), k_max=6, num_idx_heads=8),
 }
 
 
@@ -104,6 +105,20 @@ def _small_spec(name, q_scale=1.0):
 def test_small_cases_all_outputs(name, q_scale, decode, fused, cuda_device):
     wl, ref, bufs = _run(_small_spec(name, q_scale), 100 + len(name), cuda_device, decode=decode, fused=fused)
     compare(wl, ref, bufs, fused=fused)
+
+
+def test_tensor_core_indexer_many_tile_switches(cuda_device):
+    """Many short prefill chunks of long sequences: every 16-query tile straddles
+    sequences, so each CTA of the tensor-core indexer switches block tiles many
+    times and refills both of its coarse-key buffers (all scores compared)."""
+    rng = np.random.default_rng(77)
+    n = 120
+    lens = tuple(int(x) for x in rng.integers(2000, 18000, size=n))
+    n_new = tuple(int(x) for x in rng.integers(5, 31, size=n))
+    spec = wk.WorkloadSpec("tc_tile_switches", seq_lens=lens, n_new=n_new, k_per_seq=(4,) * n, k_max=4,
+                           num_q_heads=8, num_kv_heads=1, num_idx_heads=16)
+    wl, ref, bufs = _run(spec, 2024, cuda_device, decode=False)
+    compare(wl, ref, bufs)
 
 
 @pytest.mark.parametrize("fused", [False, True], ids=["score_topk", "fused_select"])
