@@ -37,7 +37,6 @@
 // A query tile spanning several sequences runs once per sequence with the
 // other queries masked; items past every query's own block are skipped.  All
 // waits are bounded.
-#include <climits>
 #include <cstddef>
 #include <cstdint>
 
@@ -60,28 +59,29 @@ constexpr int kABytes = kBT * kIdxDim;   // 8 KiB
 constexpr int kBBytes = kN * kIdxDim;    // 16 KiB
 // stage: [B 16 KiB][weights 16 x 16 int32][info]
 struct StageInfo {
-    int bt, y, abuf, agen;               // block tile, query tile, A buffer and its fill number
-    int end, pad[3];                     // end marker
-    int own[kQT];                        // own block of each query of the tile in this sequence, else -1
+    int bt, y;                           // block tile (-1: the end marker), query tile
+    int abw;                             // A buffer | its fill number << 1
+    int mask;                            // queries of the tile in this item's sequence (bit q)
+    uint32_t vbits[kBT / 32];            // rows of the A tile with a usable page, per 32-row quarter
+    int own_off, pad[3];                 // the queries' own blocks: int offset into the batch own buffer
 };
 constexpr int kOffW = kBBytes;
 constexpr int kOffInfo = kOffW + kQT * kMaxIdxHeads * 4;
 constexpr int kStageBytes = (kOffInfo + (int)sizeof(StageInfo) + 1023) / 1024 * 1024;
 constexpr int kOffA = kTcStages * kStageBytes;           // [2][kABytes], 1 KiB aligned
-constexpr int kOffAValid = kOffA + 2 * kABytes;          // [2][kBT / 32] rows with a usable page
-constexpr int kOffBars = kOffAValid + 2 * (kBT / 32) * 4;
+constexpr int kOffBars = kOffA + 2 * kABytes;
 // barriers: full[S], empty[S], tfull[2], tempty[2], afull[2]
 constexpr int kNumBars = 2 * kTcStages + 6;
 constexpr int kOffMisc = kOffBars + kNumBars * 8;   // tmem base, abort, never
-constexpr int kOffDone = kOffMisc + 16;              // items finished, per epilogue warp
 constexpr int kSeqCache = 1024;                      // cu_q and seq_lens entries staged in shared memory
-constexpr int kOffCuq = kOffDone + 4 * kEpiWarps;    // [kSeqCache] cu_q, then [kSeqCache] seq_lens
+constexpr int kOffCuq = kOffMisc + 16;               // [kSeqCache] cu_q, then [kSeqCache] seq_lens
 constexpr int kBatch = 32;                           // items decided together, one per lane
 constexpr int kOffPos = kOffCuq + 2 * kSeqCache * 4; // [2][kBatch][kQT] int32 query positions
+constexpr int kOffOwn = kOffPos + 2 * kBatch * kQT * 4;   // [2][kBatch][kQT] int32 own blocks
 constexpr int kWBytes = kQT * kMaxIdxHeads * 4;      // one tile's head weights
 // + alignment slack; at least 116 KiB so that two CTAs never share an SM (each
 // holds all 512 tensor-memory columns)
-constexpr int kSmemUsed = kOffPos + 2 * kBatch * kQT * 4 + 1024;
+constexpr int kSmemUsed = kOffOwn + 2 * kBatch * kQT * 4 + 1024;
 constexpr int kSmemBytes = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
 // full barrier: the loader's arrival with the TMA bytes, plus 32 cp.async
 // arrivals when the weights are copied by cp.async (H not a multiple of 4)
@@ -92,7 +92,8 @@ constexpr int kEmptyCount = 1 + kEpiWarps;           // MMA commit + the epilogu
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 static_assert(kOffA % 1024 == 0, "A buffers keep the 64-byte swizzle's 512-byte alignment");
-static_assert(kOffPos % 16 == 0, "positions are copied and read in 16-byte pieces");
+static_assert(kOffPos % 16 == 0 && kOffOwn % 16 == 0, "positions and own blocks move in 16-byte pieces");
+static_assert(kOffInfo % 16 == 0, "the stage info is written and read in 16-byte pieces");
 
 struct Bars {
     uint32_t base;
@@ -126,7 +127,6 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     Bars bars{base};
     // [0] tmem base, [1] abort, [2] never set
     volatile int *misc = reinterpret_cast<volatile int *>(g + kOffMisc);
-    volatile int *s_done = reinterpret_cast<volatile int *>(g + kOffDone);
     volatile int *s_abort = misc + 1;
     const volatile int *s_never = misc + 2;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -143,7 +143,6 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         misc[1] = 0;
         misc[2] = 0;
-        for (int e = 0; e < kEpiWarps; ++e) s_done[e] = 0;
         fence_barrier_init();
     }
     if (warp == kMmaWarp) {
@@ -208,16 +207,39 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         pdl_wait();   // coarse keys may come from the preceding append
         fetch_batch(i0, 0);
         fetch_batch(i0 + kBatch, 1);
+        int *s_own = reinterpret_cast<int *>(g + kOffOwn);
         int k = 0;          // items published
         int a_s = -1, a_bt = -1, ab = 1;
         int agen0 = 0, agen1 = 0, alast0 = -1, alast1 = -1;   // per A buffer: fill number, last item
+        uint32_t vb0[kBT / 32] = {0, 0, 0, 0}, vb1[kBT / 32] = {0, 0, 0, 0};   // per A buffer: valid rows
+        int olast0 = 0, olast1 = 0;   // per own buffer: items published from it so far (exclusive end)
         uint32_t err_bits = 0;
         bool stop = false;
         int pbuf = 0;
+        // Until the items before `end` are finished (false on abort).  Item j is
+        // finished when its stage's empty barrier completes the phase of j: the
+        // epilogue warps take items in order, so every earlier item is finished
+        // too.  Only items already published are asked for; a phase of item j
+        // cannot be confused with item j + 4's, which waits for this very
+        // barrier before it is published (j < k - 4 is known finished already).
+        int k_seen = -1;   // the latest item known to be finished
+        auto wait_done = [&](int end) {
+            const int j = end - 1;
+            if (j <= k_seen) return true;
+            if (!mbar_wait(bars.empty(j & (kTcStages - 1)), (j / kTcStages) & 1, s_abort)) {
+                *s_abort = 1;
+                return false;
+            }
+            k_seen = j;
+            return true;
+        };
         for (unsigned b0 = i0; b0 < i1 && !stop; b0 += kBatch, pbuf ^= 1) {
             cp_async_wait<1>();   // this batch's positions (the next batch may still be in flight)
             __syncwarp();
             const int *posb = s_posb + pbuf * kBatch * kQT;
+            int *ownb = s_own + pbuf * kBatch * kQT;
+            // the own buffer is free once the items published from it two batches ago are done
+            if (!wait_done(pbuf ? olast1 : olast0)) break;
             // ---- decisions: lane L takes item b0 + L
             int d_bt = 0, d_y = 0, d_slo = 0, d_shi = -1, d_len = 0, d_vis = 0;
             {
@@ -232,22 +254,30 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         // one sequence: visible when a member's own block reaches the tile
                         d_len = seq_len(d_slo);
                         const int4 *pp = reinterpret_cast<const int4 *>(posb + lane * kQT);
+                        int4 *po = reinterpret_cast<int4 *>(ownb + lane * kQT);
                         int mx = -1;
                         bool bad = false;
                         auto take = [&](int pos, int t) {
+                            int own = -1;
                             if (t < tn) {
-                                const int own = pos / kBlockSize;
-                                if (pos < 0 || pos >= d_len || own >= a.max_blocks) bad = true;
-                                else mx = max(mx, own);
+                                own = pos / kBlockSize;
+                                if (pos < 0 || pos >= d_len || own >= a.max_blocks) {
+                                    bad = true;
+                                    own = -1;
+                                }
+                                mx = max(mx, own);
                             }
+                            return own;
                         };
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
                             const int4 p = pp[v];
-                            take(p.x, t0 + 4 * v);
-                            take(p.y, t0 + 4 * v + 1);
-                            take(p.z, t0 + 4 * v + 2);
-                            take(p.w, t0 + 4 * v + 3);
+                            int4 o;
+                            o.x = take(p.x, t0 + 4 * v);
+                            o.y = take(p.y, t0 + 4 * v + 1);
+                            o.z = take(p.z, t0 + 4 * v + 2);
+                            o.w = take(p.w, t0 + 4 * v + 3);
+                            po[v] = o;
                         }
                         if (bad) err_bits |= DSA_DEV_ERR_POS;
                         d_vis = mx >= d_bt * kBT;
@@ -264,43 +294,40 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const int y = __shfl_sync(0xffffffffu, d_y, i);
                 const int s_lo = __shfl_sync(0xffffffffu, d_slo, i);
                 const int s_hi = __shfl_sync(0xffffffffu, d_shi, i);
-                const int len_lo = __shfl_sync(0xffffffffu, d_len, i);
                 const bool single = s_lo == s_hi;
                 const int t0 = kQT * y;
-                const int t = t0 + (lane & (kQT - 1));
-                const int pos = posb[i * kQT + (lane & (kQT - 1))];
                 for (int s = s_lo; s <= s_hi; ++s) {
-                    const int len = single ? len_lo : seq_len(s);
-                    int own = -1;
-                    if (t < a.total_q && (single || (cu(s) <= t && t < cu(s + 1)))) {
-                        own = pos / kBlockSize;
-                        if (pos < 0 || pos >= len || own >= a.max_blocks) {
-                            err_bits |= DSA_DEV_ERR_POS;
-                            own = -1;
+                    int mask = 0xffff;
+                    if (!single) {
+                        // several sequences: this sequence's queries, their own blocks
+                        const int t = t0 + (lane & (kQT - 1));
+                        const int pos = posb[i * kQT + (lane & (kQT - 1))];
+                        const int len = seq_len(s);
+                        const bool member = lane < kQT && t < a.total_q && cu(s) <= t && t < cu(s + 1);
+                        int own = -1;
+                        if (member) {
+                            own = pos / kBlockSize;
+                            if (pos < 0 || pos >= len || own >= a.max_blocks) {
+                                err_bits |= DSA_DEV_ERR_POS;
+                                own = -1;
+                            }
+                            ownb[i * kQT + lane] = own;
                         }
+                        mask = (int)__ballot_sync(0xffffffffu, member);
+                        if (__reduce_max_sync(0xffffffffu, own) < bt * kBT) continue;   // nothing visible
                     }
-                    if (!single && __reduce_max_sync(0xffffffffu, own) < bt * kBT) continue;   // nothing visible
                     if (s != a_s || bt != a_bt) {
                         // a new block tile: into the other A buffer once the items
                         // still reading it have all finished
                         a_s = s;
                         a_bt = bt;
                         ab ^= 1;
-                        const int last = ab ? alast1 : alast0;
-                        if (last >= 0) {
-                            const long long t_start = clock64();
-                            while (__reduce_min_sync(0xffffffffu, lane < kEpiWarps ? s_done[lane] : INT_MAX) <=
-                                   last) {
-                                if (*s_abort || clock64() - t_start > kWaitLimitCycles) {
-                                    *s_abort = 1;
-                                    stop = true;
-                                    break;
-                                }
-                                __nanosleep(64);
-                            }
-                            if (stop) break;
+                        if (!wait_done((ab ? alast1 : alast0) + 1)) {
+                            stop = true;
+                            break;
                         }
                         if (ab) ++agen1; else ++agen0;
+                        const int len = single ? __shfl_sync(0xffffffffu, d_len, i) : seq_len(s);
                         const int n_blocks = (len + kBlockSize - 1) / kBlockSize;
                         const int32_t *row = a.block_table + (size_t)s * a.max_blocks;
                         int page[kBT / 32];
@@ -310,7 +337,6 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                             page[j] = b < n_blocks && b < a.max_blocks ? __ldg(row + b) : -1;
                         }
                         const uint32_t sa = base + kOffA + ab * kABytes;
-                        uint32_t *vbits = reinterpret_cast<uint32_t *>(g + kOffAValid) + ab * (kBT / 32);
 #pragma unroll
                         for (int j = 0; j < kBT / 32; ++j) {
                             const int b = bt * kBT + 32 * j + lane;
@@ -319,7 +345,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                                 page[j] = -1;
                             }
                             const uint32_t bits = __ballot_sync(0xffffffffu, page[j] >= 0);
-                            if (lane == 0) vbits[j] = bits;
+                            if (ab) vb1[j] = bits; else vb0[j] = bits;
                             const int r = 32 * j + lane;
                             const int8_t *src = a.kc_pool + (size_t)max(page[j], 0) * kIdxDim;
 #pragma unroll
@@ -335,21 +361,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     }
                     if (ab) alast1 = k; else alast0 = k;
                     const int st = k & (kTcStages - 1);
-                    if (k >= kTcStages && !mbar_wait(bars.empty(st), ((k / kTcStages) - 1) & 1, s_abort)) {
-                        *s_abort = 1;
+                    if (k >= kTcStages && !wait_done(k - kTcStages + 1)) {   // the stage's previous item
                         stop = true;
                         break;
                     }
-                    StageInfo *info = reinterpret_cast<StageInfo *>(g + st * kStageBytes + kOffInfo);
                     const uint32_t sb = base + st * kStageBytes;
-                    if (lane == 0) {
-                        info->end = 0;
-                        info->bt = bt;
-                        info->y = y;
-                        info->abuf = ab;
-                        info->agen = ab ? agen1 : agen0;
-                    }
-                    if (lane < kQT) info->own[lane] = own;
                     if (!w_tma) {
                         // the tile's head weights (16 queries x 16 heads, zero past H and the last query)
 #pragma unroll
@@ -360,8 +376,13 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         }
                         tc::cp_async_arrive_noinc(bars.full(st));
                     }
-                    __syncwarp();   // the info words above, before the release arrival
+                    __syncwarp();   // the own blocks written above, before the release arrival
                     if (lane == 0) {
+                        int4 *info = reinterpret_cast<int4 *>(g + st * kStageBytes + kOffInfo);
+                        info[0] = make_int4(bt, y, ab | ((ab ? agen1 : agen0) << 1), mask);
+                        info[1] = ab ? make_int4((int)vb1[0], (int)vb1[1], (int)vb1[2], (int)vb1[3])
+                                     : make_int4((int)vb0[0], (int)vb0[1], (int)vb0[2], (int)vb0[3]);
+                        info[2].x = (pbuf * kBatch + i) * kQT;
                         // the queries' rows: box (64 B, 16 heads, 16 queries) at query t0, and
                         // their weights: box (16 heads, 16 queries), zero past H and the last query
                         mbar_arrive_expect_tx(bars.full(st), kBBytes + (w_tma ? kWBytes : 0));
@@ -371,6 +392,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     ++k;
                 }
             }
+            if (pbuf) olast1 = k; else olast0 = k;
             // every lane is done with this batch's positions: refill the buffer
             __syncwarp();
             fetch_batch(b0 + 2 * kBatch, pbuf);
@@ -383,7 +405,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 *s_abort = 1;
             } else {
                 StageInfo *info = reinterpret_cast<StageInfo *>(g + st * kStageBytes + kOffInfo);
-                if (lane == 0) info->end = 1;
+                if (lane == 0) info->bt = -1;
                 if (!w_tma) tc::cp_async_arrive_noinc(bars.full(st));
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bars.full(st));
@@ -407,8 +429,9 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const int st = k % kTcStages, buf = k & 1;
             bool ok = mbar_wait(bars.full(st), (k / kTcStages) & 1, s_abort);
             const StageInfo *info = reinterpret_cast<const StageInfo *>(g + st * kStageBytes + kOffInfo);
-            const bool end = ok && info->end != 0;
-            if (ok && !end) ok = mbar_wait(bars.afull(info->abuf), (info->agen - 1) & 1, s_abort);
+            const bool end = ok && info->bt < 0;
+            const int abw = ok ? info->abw : 0;
+            if (ok && !end) ok = mbar_wait(bars.afull(abw & 1), ((abw >> 1) - 1) & 1, s_abort);
             // the accumulator's previous item has been read (the end marker's
             // arrival on tfull must not run two phases ahead of the epilogue)
             if (ok && k >= 2) ok = mbar_wait(bars.tempty(buf), ((k >> 1) - 1) & 1, s_abort);
@@ -422,7 +445,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 } else {
                     tc::fence_proxy_async_smem();   // the cp.async-written keys, for the tensor core
                     tc::fence_after_sync();
-                    const uint32_t sa = base + kOffA + info->abuf * kABytes;
+                    const uint32_t sa = base + kOffA + (abw & 1) * kABytes;
                     const uint32_t sb = base + st * kStageBytes;
                     const uint32_t d = tmem + (uint32_t)(buf * kN);
                     const uint64_t da = tc::smem_desc_k64_sw64(sa), db = tc::smem_desc_k64_sw64(sb);
@@ -447,6 +470,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
         const int qgrp = ew >> 2;                // queries 4*qgrp .. +3 (columns 64*qgrp ..)
         const int row = quarter * 32 + lane;     // block row of the tile
+        const int *s_own_e = reinterpret_cast<const int *>(g + kOffOwn);
         int k = 0;
         while (true) {
             const int st = k % kTcStages, buf = k & 1;
@@ -458,37 +482,33 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             tc::fence_after_sync();
             const StageInfo *info = reinterpret_cast<const StageInfo *>(g + st * kStageBytes + kOffInfo);
-            if (info->end) break;
-            // acquire the A buffer's valid bits (cannot be refilled before this warp finishes the item)
-            if (!mbar_wait(bars.afull(info->abuf), (info->agen - 1) & 1, s_abort)) {
-                if (lane == 0) *s_abort = 1;
-                break;
-            }
-            const int bt = info->bt, y = info->y;
+            const int4 i0w = *reinterpret_cast<const int4 *>(info);
+            if (i0w.x < 0) break;   // the end marker
+            const int bt = i0w.x, y = i0w.y, mask = i0w.w;
             const int b = bt * kBT + row;
-            const uint32_t vbits = reinterpret_cast<const uint32_t *>(g + kOffAValid)[info->abuf * (kBT / 32) + (row >> 5)];
-            const bool row_ok = (vbits >> (row & 31)) & 1u;
+            const bool row_ok = (info->vbits[quarter] >> lane) & 1u;
             const uint32_t taddr =
                 tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kN + qgrp * 64);
-            // weights (shared-space vector loads) and own blocks of this warp's 4 queries
-            const uint32_t s_w = base + st * kStageBytes + kOffW + (uint32_t)(4 * qgrp * kMaxIdxHeads * 4);
-            int own4[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) own4[u] = info->own[4 * qgrp + u];
+            // own blocks of this warp's 4 queries (-1 outside this item's sequence) and their weights
+            const int4 o4 = *reinterpret_cast<const int4 *>(s_own_e + info->own_off + 4 * qgrp);
+            const int own4[4] = {(mask >> (4 * qgrp)) & 1 ? o4.x : -1, (mask >> (4 * qgrp + 1)) & 1 ? o4.y : -1,
+                                 (mask >> (4 * qgrp + 2)) & 1 ? o4.z : -1, (mask >> (4 * qgrp + 3)) & 1 ? o4.w : -1};
+            const int4 *w4 = reinterpret_cast<const int4 *>(g + st * kStageBytes + kOffW) + qgrp * kMaxIdxHeads;
             uint32_t v[2][32];
             tc::ld_32x32b_x32(taddr, v[0]);
             tc::ld_32x32b_x32(taddr + 32, v[1]);
             tc::wait_ld();
+            // the accumulator is in registers: release it to the next MMA now
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bars.tempty(buf));
 #pragma unroll
             for (int u = 0; u < 4; ++u) {   // query 4*qgrp + u: columns 16u .. 16u+15 of this warp's 64
                 const uint32_t *x = v[u >> 1] + 16 * (u & 1);
                 int part[4];
 #pragma unroll
                 for (int h4 = 0; h4 < 4; ++h4) {   // four independent chains
-                    int4 wv;
-                    asm volatile("ld.shared.v4.s32 {%0,%1,%2,%3}, [%4];"
-                                 : "=r"(wv.x), "=r"(wv.y), "=r"(wv.z), "=r"(wv.w)
-                                 : "r"(s_w + (uint32_t)((u * kMaxIdxHeads + 4 * h4) * 4)));
+                    const int4 wv = w4[u * (kMaxIdxHeads / 4) + h4];
                     part[h4] = wv.x * max((int)x[4 * h4 + 0], 0) + wv.y * max((int)x[4 * h4 + 1], 0) +
                                wv.z * max((int)x[4 * h4 + 2], 0) + wv.w * max((int)x[4 * h4 + 3], 0);
                 }
@@ -496,14 +516,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 if (row_ok && b <= own4[u])
                     a.scores[(size_t)(kQT * y + 4 * qgrp + u) * a.max_blocks + b] = sum;
             }
-            tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bars.tempty(buf));
-                mbar_arrive(bars.empty(st));
-                __threadfence_block();
-                s_done[ew] = k + 1;   // lets the loaders refill the A buffer
-            }
+            if (lane == 0) mbar_arrive(bars.empty(st));   // the stage (info, weights, own blocks) is read
             ++k;
         }
     }
