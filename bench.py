@@ -5,9 +5,13 @@ One step = one pass of the whole hot path over one batch:
   kv_append (the batch's new tokens) -> index_score -> topk_blocks -> attention.
 Default workload: 1M-context decode (8 sequences x 1,048,576 tokens, Top-K 32
 blocks of 64 tokens, 64 query / 8 KV heads, 16 indexer heads).  The step is
-captured in a CUDA graph; before every timed step the L2 is made cold (a
-512 MiB write, then a 256 MiB read so no dirty lines remain) and each step is
-timed with CUDA events on the launching stream.
+captured in a CUDA graph.  The timed steps run back to back and rotate through
+several independent batches (their own sequences, KV pools and queries) whose
+step traffic together exceeds the L2 by half, so no step finds its data in L2;
+the K steps are timed with one pair of CUDA events on the launching stream.
+Workloads too small for that are timed one step at a time after a cold-L2
+flush (512 MiB written, then 256 MiB read so no dirty lines remain), which is
+also reported for the first batch as the isolated step time.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun every rank runs its own batch (weak scaling, no collective on
@@ -33,6 +37,9 @@ if ROOT not in sys.path:
 METRIC = "sparse-attn decode tokens/s @1M ctx; achieved HBM GB/s vs ~8 TB/s peak"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 512 << 20
+L2_BYTES = 126 << 20            # B200 L2
+ROTATE_L2_MULTIPLE = 1.5        # rotated batches' step traffic, in L2 capacities
+MAX_ROTATE = 4
 # DRAM bytes (read + write) per launch of the roofline kernel, from an ncu
 # capture of the current kernel ((workload, path) -> bytes); absent = not
 # captured since the kernel last changed.  The decode attention figure comes
@@ -100,7 +107,7 @@ class ClockSampler:
         0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.samples, self.reasons = [], set()
         self.max_mhz = None
         self._stop = threading.Event()
@@ -178,10 +185,6 @@ def run_ours(args, world, rank, device):
     from dynamic_block_sparse_dsa_b200 import workloads as wk
 
     spec = wk.NAMED[args.workload]()
-    wl = wk.make_workload(spec, seed=args.seed + rank, device=device)
-    cache = dsa.PagedKVCache(wl.k_pool, wl.v_pool, wl.kc_pool)
-    seqs = dsa.SeqBatch(wl.block_table, wl.seq_lens)
-    queries = dsa.QueryBatch(wl.cu_q, wl.q_pos)
     decode = all(n == 1 for n in spec.n_new)
     path = args.path
     if path == "auto":   # decode batches: the fused select chain; otherwise the separate calls
@@ -195,62 +198,88 @@ def run_ours(args, world, rank, device):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     flush_rd = torch.ones(L2_FLUSH_BYTES // 2 // 4, dtype=torch.int32, device=device)
 
-    def front(b):
-        if fused and decode:   # a decode batch: the append may overlap the selection
-            dsa.select_blocks_append(cache, seqs, queries, queries.cu_q, wl.k_new, wl.v_new, wl.kc_new, wl.q_idx,
-                                     wl.w, wl.k_per_seq, spec.k_max, 16, sel=b["sel"], cnt=b["cnt"],
-                                     workspace=b["select_ws"], dev_err=err)
-            return
-        dsa.kv_append(cache, seqs, queries.cu_q, wl.k_new, wl.v_new, wl.kc_new, dev_err=err)
-        if fused:
-            dsa.select_blocks(cache, seqs, queries, wl.q_idx, wl.w, wl.k_per_seq, spec.k_max, 16, sel=b["sel"],
-                              cnt=b["cnt"], workspace=b["select_ws"], dev_err=err)
-        else:
-            dsa.index_score(cache, seqs, queries, wl.q_idx, wl.w, 16, scores=b["scores"], dev_err=err)
-            dsa.topk_blocks(seqs, queries, b["scores"], wl.k_per_seq, spec.k_max, sel=b["sel"], cnt=b["cnt"],
-                            dev_err=err)
+    class Case:
+        """One independent batch of the workload (its own sequences, KV pool,
+        queries and output buffers) with its captured step and attention graphs."""
 
-    def attn(b):
-        if decode:
-            dsa.sparse_attn_decode(cache, seqs, queries, wl.q, b["sel"], b["cnt"], out=b["out"], lse=b["lse"],
-                                   workspace=b["workspace"], dev_err=err)
-        else:
-            dsa.sparse_attn_prefill(cache, seqs, queries, wl.q, b["sel"], b["cnt"], out=b["out"], lse=b["lse"],
-                                    dev_err=err)
+        def __init__(self, seed):
+            self.wl = wl = wk.make_workload(spec, seed=seed, device=device)
+            self.cache = dsa.PagedKVCache(wl.k_pool, wl.v_pool, wl.kc_pool)
+            self.seqs = dsa.SeqBatch(wl.block_table, wl.seq_lens)
+            self.queries = dsa.QueryBatch(wl.cu_q, wl.q_pos)
+            with torch.cuda.stream(stream):
+                self.bufs = dsa.step(self.cache, self.seqs, self.queries, k_new=wl.k_new, v_new=wl.v_new,
+                                     kc_new=wl.kc_new, q=wl.q, q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq,
+                                     k_max=spec.k_max, decode=decode, fused_select=fused,
+                                     overlap_append=fused and decode, fused_decode=fused_decode, dev_err=err)
+            torch.cuda.synchronize(device)
+            if int(err.item()) != 0:
+                raise RuntimeError(f"device error bits {int(err.item())} in the first step")
+            # one graph for the whole step (events only at its ends, so the
+            # kernels' programmatic dependent launches overlap) and one for the
+            # attention kernel alone, which times the dominant kernel
+            self.ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+            self.graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.graph, stream=stream):
+                self.ev[0].record()
+                if fused_decode:
+                    self.whole_step()
+                else:
+                    self.front()
+                    self.attn()
+                self.ev[1].record()
+            self.graph_attn = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.graph_attn, stream=stream):
+                self.ev[2].record()
+                self.attn()
+                self.ev[3].record()
+            torch.cuda.synchronize(device)
 
-    def whole_step(b):
-        dsa.decode_fused(cache, seqs, queries, queries.cu_q, wl.k_new, wl.v_new, wl.kc_new, wl.q_idx, wl.w,
-                         wl.k_per_seq, spec.k_max, wl.q, sel=b["sel"], cnt=b["cnt"], out=b["out"], lse=b["lse"],
-                         workspace=b["fused_ws"], dev_err=err)
+        def front(self):
+            wl, b = self.wl, self.bufs
+            if fused and decode:   # a decode batch: the append may overlap the selection
+                dsa.select_blocks_append(self.cache, self.seqs, self.queries, self.queries.cu_q, wl.k_new, wl.v_new,
+                                         wl.kc_new, wl.q_idx, wl.w, wl.k_per_seq, spec.k_max, 16, sel=b["sel"],
+                                         cnt=b["cnt"], workspace=b["select_ws"], dev_err=err)
+                return
+            dsa.kv_append(self.cache, self.seqs, self.queries.cu_q, wl.k_new, wl.v_new, wl.kc_new, dev_err=err)
+            if fused:
+                dsa.select_blocks(self.cache, self.seqs, self.queries, wl.q_idx, wl.w, wl.k_per_seq, spec.k_max, 16,
+                                  sel=b["sel"], cnt=b["cnt"], workspace=b["select_ws"], dev_err=err)
+            else:
+                dsa.index_score(self.cache, self.seqs, self.queries, wl.q_idx, wl.w, 16, scores=b["scores"],
+                                dev_err=err)
+                dsa.topk_blocks(self.seqs, self.queries, b["scores"], wl.k_per_seq, spec.k_max, sel=b["sel"],
+                                cnt=b["cnt"], dev_err=err)
 
-    with torch.cuda.stream(stream):
-        bufs = dsa.step(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
-                        q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=spec.k_max, decode=decode,
-                        fused_select=fused, overlap_append=fused and decode, fused_decode=fused_decode,
-                        dev_err=err)
-    torch.cuda.synchronize(device)
-    if int(err.item()) != 0:
-        raise RuntimeError(f"device error bits {int(err.item())} in the first step")
+        def attn(self):
+            wl, b = self.wl, self.bufs
+            if decode:
+                dsa.sparse_attn_decode(self.cache, self.seqs, self.queries, wl.q, b["sel"], b["cnt"], out=b["out"],
+                                       lse=b["lse"], workspace=b["workspace"], dev_err=err)
+            else:
+                dsa.sparse_attn_prefill(self.cache, self.seqs, self.queries, wl.q, b["sel"], b["cnt"], out=b["out"],
+                                        lse=b["lse"], dev_err=err)
 
-    # one graph for the whole step (events only at its ends, so the kernels'
-    # programmatic dependent launches overlap) and one for the attention kernel
-    # alone, which times the dominant kernel for the roofline
-    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        ev[0].record()
-        if fused_decode:
-            whole_step(bufs)
-        else:
-            front(bufs)
-            attn(bufs)
-        ev[1].record()
-    graph_attn = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_attn, stream=stream):
-        ev[2].record()
-        attn(bufs)
-        ev[3].record()
-    torch.cuda.synchronize(device)
+        def whole_step(self):
+            wl, b = self.wl, self.bufs
+            dsa.decode_fused(self.cache, self.seqs, self.queries, self.queries.cu_q, wl.k_new, wl.v_new, wl.kc_new,
+                             wl.q_idx, wl.w, wl.k_per_seq, spec.k_max, wl.q, sel=b["sel"], cnt=b["cnt"],
+                             out=b["out"], lse=b["lse"], workspace=b["fused_ws"], dev_err=err)
+
+    # independent batches whose step traffic together exceeds the L2: the timed
+    # steps rotate through them back to back, so no step finds its data in L2
+    # (workloads too small for that, more than MAX_ROTATE batches, are timed one
+    # step at a time after a cold-L2 flush instead)
+    cases = [Case(args.seed + rank)]
+    ab = algorithmic_bytes(cases[0].wl)
+    need = max(args.rotate, math.ceil(ROTATE_L2_MULTIPLE * L2_BYTES / ab["total"]))
+    rotate = need <= MAX_ROTATE
+    while rotate and len(cases) < need:
+        cases.append(Case(args.seed + rank + 7919 * len(cases)))
+    case0 = cases[0]
+    wl, cache, seqs, queries, bufs = case0.wl, case0.cache, case0.seqs, case0.queries, case0.bufs
+    n_case = len(cases)
 
     def cold_l2():
         # write a buffer larger than the L2, then read another one so that the
@@ -258,49 +287,98 @@ def run_ours(args, world, rank, device):
         flush.fill_(1)
         flush_rd.sum(dtype=torch.int32)
 
-    def one_step(g, e0, e1):
-        with torch.cuda.stream(stream):
-            cold_l2()
-            g.replay()
-        stream.synchronize()
-        return e0.elapsed_time(e1)
+    # one graph holding a step of every batch in turn (as consecutive layers'
+    # steps would sit in one graph), and one holding their attention launches
+    rot_graph, rot_attn = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    if rotate:
+        with torch.cuda.graph(rot_graph, stream=stream):
+            for c in cases:
+                if fused_decode:
+                    c.whole_step()
+                else:
+                    c.front()
+                    c.attn()
+        with torch.cuda.graph(rot_attn, stream=stream):
+            for c in cases:
+                c.attn()
+        torch.cuda.synchronize(device)
 
+    def rotated(which, n):
+        """n steps (or attention launches) back to back over the batches in
+        turn; seconds on the device."""
+        whole, single = (rot_graph, lambda c: c.graph) if which == "step" else (rot_attn, lambda c: c.graph_attn)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record()
+            for _ in range(n // n_case):
+                whole.replay()
+            for i in range(n % n_case):
+                single(cases[i]).replay()
+            e1.record()
+        stream.synchronize()
+        return e0.elapsed_time(e1) / 1e3
+
+    def isolated(graph_of, ev_of, n):
+        """n replays of the first batch, each after a cold-L2 flush; ms per replay (in-graph events)."""
+        ms = []
+        for _ in range(n):
+            with torch.cuda.stream(stream):
+                cold_l2()
+                graph_of(case0).replay()
+            stream.synchronize()
+            e0, e1 = ev_of(case0)
+            ms.append(e0.elapsed_time(e1))
+        return ms
+
+    step_graph = lambda c: c.graph
+    attn_graph = lambda c: c.graph_attn
     for _ in range(args.warmup):
-        one_step(graph, ev[0], ev[1])
-        one_step(graph_attn, ev[2], ev[3])
+        if rotate:
+            rotated("step", n_case)
+            rotated("attn", n_case)
+        else:
+            isolated(step_graph, lambda c: (c.ev[0], c.ev[1]), 1)
     barrier(world)
     torch.cuda.synchronize(device)
-    step_ms = []
     with ClockSampler(device.index if device.index is not None else 0) as clk:
-        for _ in range(args.steps):
-            step_ms.append(one_step(graph, ev[0], ev[1]))
+        if rotate:
+            total_s = rotated("step", args.steps)
+        else:
+            total_s = sum(isolated(step_graph, lambda c: (c.ev[0], c.ev[1]), args.steps)) / 1e3
     torch.cuda.synchronize(device)
     barrier(world)
-    attn_ms = [one_step(graph_attn, ev[2], ev[3]) for _ in range(max(10, min(args.steps, 100)))]
+    n_attn = max(3 * n_case, min(args.steps, 300))
+    iso_step_ms = isolated(step_graph, lambda c: (c.ev[0], c.ev[1]), max(5, min(args.steps, 50)))
+    iso_attn_ms = isolated(attn_graph, lambda c: (c.ev[2], c.ev[3]), max(5, min(args.steps, 50)))
+    attn_mean_s = rotated("attn", n_attn) / n_attn if rotate else statistics.mean(iso_attn_ms) / 1e3
     if int(err.item()) != 0:
         raise RuntimeError(f"device error bits {int(err.item())} during timing")
 
-    total_s = sum(step_ms) / 1e3
     total_s_max = max_over_ranks(total_s, world, device)
     tokens_per_step = spec.total_q
     value = weak_scaling_throughput(tokens_per_step, args.steps, world, total_s_max)
-    ab = algorithmic_bytes(wl)
-    attn_mean_s = sum(attn_ms) / len(attn_ms) / 1e3
     step_mean_s = total_s / args.steps
     peak, peak_kind = _peaks()
     if fused_decode:
         # the step is one kernel: its bytes are the coarse keys plus the selected K/V
         achieved = ab["total"] / step_mean_s / 1e9
-        roofline = {"bound": "hbm", "kernel": "sparse_attn_kernel<1,true> (single-launch decode step, cold L2)",
+        roofline = {"bound": "hbm", "kernel": "sparse_attn_kernel<1,true> (single-launch decode step)",
                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                     "peak_source": peak_kind, "bytes_per_launch": ab["total"],
                     "traffic": TRAFFIC.get((spec.name, "fused_decode"))}
     else:
         achieved = ab["kv"] / attn_mean_s / 1e9
-        roofline = {"bound": "hbm", "kernel": "sparse_attn_kernel (decode entry; timed alone, cold L2)",
+        iso = statistics.median(iso_attn_ms) * 1e-3
+        roofline = {"bound": "hbm", "kernel": "sparse_attn_kernel (decode entry)",
                     "achieved": round(achieved, 1),
                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": peak_kind,
-                    "bytes_per_launch": ab["kv"], "traffic": TRAFFIC.get((spec.name, "attention"))}
+                    "bytes_per_launch": ab["kv"], "traffic": TRAFFIC.get((spec.name, "attention")),
+                    "timing": (f"mean over {n_attn} launches back to back ({n_case} per graph, one per "
+                               f"independent batch, PDL between them)"
+                               if rotate else "mean of single launches after a cold-L2 flush"),
+                    "isolated": {"us": round(iso * 1e6, 2), "achieved": round(ab["kv"] / iso / 1e9, 1),
+                                 "frac": round(ab["kv"] / iso / 1e9 / peak, 4),
+                                 "how": "one launch after a cold-L2 flush, in-graph events (median)"}}
     step_gbs = ab["total"] / step_mean_s / 1e9
     step_roof = {"bytes_per_step": ab["total"], "achieved_gbs": round(step_gbs, 1),
                  "frac_of_measured": round(step_gbs / peak, 4), "frac_of_8tbs": round(step_gbs / 8000.0, 4)}
@@ -356,7 +434,7 @@ def run_ours(args, world, rank, device):
            "how": "dsa.step called from Python every step, H2D input copies and D2H output copies inside the timed region",
            "graph_value": e2e_graph,
            "graph_how": "the same copies and calls captured once in a CUDA graph, replayed every step"}
-    del graph_e2e
+    del graph_e2e, rot_graph, rot_attn
 
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -367,15 +445,18 @@ def run_ours(args, world, rank, device):
                    "top_k": spec.k_max, "block_size": spec.block_size,
                    "heads_q_kv_idx": [spec.num_q_heads, spec.num_kv_heads, spec.num_idx_heads],
                    "global_batch": spec.num_seqs * world, "parallelism": f"dp{world} (independent sequences)",
-                   "l2": "cold before every timed step: 512 MiB written, then 256 MiB read (no dirty lines)",
-                   "graph": "one CUDA graph per step" + ("" if fused_decode else " (PDL between kernels)"),
+                   "l2": (f"inputs larger than L2: steps back to back over {n_case} independent batches "
+                          f"({n_case * ab['total'] / 2**20:.0f} MiB of step traffic, L2 126 MiB)" if rotate else
+                          "cold before every timed step: 512 MiB written, then 256 MiB read (no dirty lines)"),
+                   "graph": (f"one CUDA graph per {n_case} steps, one step of each batch in turn"
+                             if rotate else "one CUDA graph per step") + ("" if fused_decode else " (PDL between kernels)"),
                    "path": {"fused_decode": "single launch: append + fused score/Top-K + attention",
                             "fused_select": "fused score+Top-K with the token append overlapping it, attention",
                             "score_topk": "kv_append, index_score, topk_blocks, attention"}[path]},
         "roofline": roofline,
         "step_roofline": step_roof,
         "attn_ms_mean": round(attn_mean_s * 1e3, 5),
-        "step_ms_median": round(statistics.median(step_ms), 5),
+        "step_isolated_ms_median": round(statistics.median(iso_step_ms), 5),
         "e2e": e2e,
         "gpu_launches": (1 if fused_decode else 3 if fused else 4) * args.steps,
         "clocks": clk.summary(),
@@ -477,6 +558,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode_1m")
     ap.add_argument("--seed", type=int, default=1003)
+    ap.add_argument("--rotate", type=int, default=2,
+                    help="independent batches the timed steps rotate through (more if needed to exceed the L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-indexer measurement")
     ap.add_argument("--path", choices=["auto", "fused_decode", "fused_select", "score_topk"], default="auto",
