@@ -204,6 +204,26 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             cp_async_commit();
         };
+        {
+            // warm the L2 with what the first items read while a preceding kernel
+            // may still run (prefetches only: nothing is read before the wait):
+            // the first batch's positions, the first query tiles and weights, and
+            // the first block tile's table entries
+            const unsigned j = i0 + (unsigned)lane;
+            if (j < i1) {
+                const unsigned bt = j / (unsigned)n_qt;
+                const int y = (int)(j - bt * (unsigned)n_qt);
+                prefetch_l2_line(a.q_pos + kQT * y);
+                if (lane < kTcStages) {
+                    tma_prefetch_3d(&tm_q, 0, 0, kQT * y);
+                    if (w_tma) tma_prefetch_2d(&tm_w, 0, kQT * y);
+                }
+            }
+            const unsigned bt0 = i0 / (unsigned)n_qt;
+            const int s0 = seq_of(kQT * (int)(i0 - bt0 * (unsigned)n_qt));
+            if (lane < kBT * 4 / 128 && (int)bt0 * kBT + 32 * lane < a.max_blocks)
+                prefetch_l2_line(a.block_table + (size_t)s0 * a.max_blocks + bt0 * kBT + 32 * lane);
+        }
         pdl_wait();   // coarse keys may come from the preceding append
         fetch_batch(i0, 0);
         fetch_batch(i0 + kBatch, 1);
