@@ -458,7 +458,7 @@ def run_ours(args, world, rank, device):
         "attn_ms_mean": round(attn_mean_s * 1e3, 5),
         "step_isolated_ms_median": round(statistics.median(iso_step_ms), 5),
         "e2e": e2e,
-        "gpu_launches": (1 if fused_decode else 3 if fused else 4) * args.steps,
+        "gpu_launches": (1 if fused_decode else 2 if fused and decode else 3 if fused else 4) * args.steps,
         "clocks": clk.summary(),
     }
     return res, wl

@@ -159,7 +159,7 @@ int attn_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queri
 int select_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
                   const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads, int32_t w_abs_max,
                   const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt, void *workspace,
-                  size_t workspace_bytes, const int32_t *cu_new, int32_t *dev_err, dsa_stream_t stream);
+                  size_t workspace_bytes, const KvAppendArgs *app, int32_t *dev_err, dsa_stream_t stream);
 
 }  // namespace
 
@@ -295,9 +295,6 @@ int dsa_select_blocks_append(const dsa_kv_cache *cache, const dsa_seqs *seqs, co
         if (!cu_new || !k_new || !v_new) return DSA_ERR_INVALID_ARG;
         if (!aligned16(k_new) || !aligned16(v_new) || (kc_new && !aligned16(kc_new))) return DSA_ERR_INVALID_ARG;
     }
-    rc = select_common(cache, seqs, queries, q_idx, w, num_idx_heads, w_abs_max, k_per_seq, k_max, sel, cnt,
-                       workspace, workspace_bytes, total_new > 0 ? cu_new : nullptr, dev_err, stream);
-    if (rc || total_new == 0) return rc;
     KvAppendArgs a{};
     a.k_pool = cache->k_pool;
     a.v_pool = cache->v_pool;
@@ -314,7 +311,12 @@ int dsa_select_blocks_append(const dsa_kv_cache *cache, const dsa_seqs *seqs, co
     a.v_new = v_new;
     a.kc_new = kc_new;
     a.dev_err = dev_err;
-    a.overlap_prev = queries->total_q > 0 ? 1 : 0;   // nothing launched before it when there are no queries
+    a.overlap_prev = 0;
+    // the append runs as extra CTAs of the selection's grid; with no queries
+    // there is no selection launch, so it is launched on its own
+    rc = select_common(cache, seqs, queries, q_idx, w, num_idx_heads, w_abs_max, k_per_seq, k_max, sel, cnt,
+                       workspace, workspace_bytes, total_new > 0 ? &a : nullptr, dev_err, stream);
+    if (rc || total_new == 0 || queries->total_q > 0) return rc;
     return from_cuda(launch_kv_append(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -324,7 +326,7 @@ namespace {
 int select_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
                   const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads, int32_t w_abs_max,
                   const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt, void *workspace,
-                  size_t workspace_bytes, const int32_t *cu_new, int32_t *dev_err, dsa_stream_t stream) {
+                  size_t workspace_bytes, const KvAppendArgs *app, int32_t *dev_err, dsa_stream_t stream) {
     int rc;
     if ((rc = check_cache(cache)) || (rc = check_seqs(seqs)) || (rc = check_queries(queries))) return rc;
     if (num_idx_heads < 1 || w_abs_max < 0 || k_max < 1) return DSA_ERR_INVALID_ARG;
@@ -357,7 +359,8 @@ int select_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_que
     a.counters = reinterpret_cast<int32_t *>(ws + L.counters);
     a.cand = reinterpret_cast<unsigned long long *>(ws + L.cand);
     a.dev_err = dev_err;
-    a.cu_new = cu_new;
+    a.cu_new = app ? app->cu_new : nullptr;
+    if (app) a.app = *app;
     return from_cuda(launch_select_blocks(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 }  // namespace

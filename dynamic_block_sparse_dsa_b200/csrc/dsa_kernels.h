@@ -102,6 +102,10 @@ struct SelectArgs {
     // (DSA_DEV_ERR_POS, cnt 0) -- the selection must not read those keys; and
     // the kernel is launched after everything before it has completed
     const int32_t *cu_new;   // null: no append follows
+    // the append itself (app.total_new > 0): extra CTAs of the selection grid,
+    // rows sel_rows.. of blockIdx.y, copy the new tokens while the selection runs
+    KvAppendArgs app;
+    int sel_rows;            // set by the launcher: grid rows that select
 };
 
 struct AttnArgs {

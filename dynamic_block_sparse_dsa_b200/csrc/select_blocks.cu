@@ -20,7 +20,9 @@
 // selection.  Result is identical to dsa_index_score followed by
 // dsa_topk_blocks.
 #include "dsa_kernels.h"
+#include "dsa_tma.cuh"
 #include "indexer_core.cuh"
+#include "kv_append.cuh"
 #include "warp_topk.cuh"
 
 namespace dsa {
@@ -44,6 +46,13 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     const int H = a.num_idx_heads;
 
     pdl_trigger();
+    if ((int)blockIdx.y >= a.sel_rows) {
+        // an append CTA: one new token per CTA, overlapping the selection (which
+        // never reads the rows written here -- see SelectArgs::cu_new)
+        const int i = t + ((int)blockIdx.y - a.sel_rows) * (int)gridDim.x;
+        if (i < a.app.total_new) append_token(a.app, i, tid, kSelThreads);
+        return;
+    }
     // ---- query facts.  The position and cu_q travel together; then, once the
     // sequence is known, its length, Top-K and the first group's page ids
     // travel together: two round trips before the coarse keys
@@ -222,6 +231,11 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
             a.counters[t] = 0;          // ready for the next call
         }
         for (int i = km + 1 + lane; i < a.k_max; i += 32) out[i] = -1;
+        // the attention that follows looks these blocks' pages up first: warm
+        // their block-table lines in L2 (a prefetch, no value is read)
+        const int32_t *row = a.block_table + (size_t)s * a.max_blocks;
+        if (v0) prefetch_l2_line(row + ids[0]);
+        if (v1) prefetch_l2_line(row + ids[1]);
     }
 }
 
@@ -231,12 +245,16 @@ cudaError_t launch_select_blocks(const SelectArgs &a, cudaStream_t stream) {
     const int need = (a.max_blocks + kSelMaxChunks - 1) / kSelMaxChunks;   // blocks per chunk
     const int gr = (need + kSelWarps * 64 - 1) / (kSelWarps * 64);
     auto go = [&](auto kern, int G) {
-        const int chunks = (a.max_blocks + kSelWarps * 64 * G - 1) / (kSelWarps * 64 * G);
+        SelectArgs b = a;
+        b.sel_rows = (a.max_blocks + kSelWarps * 64 * G - 1) / (kSelWarps * 64 * G);   // chunks
+        const int app_rows = a.app.total_new > 0 ? (a.app.total_new + a.total_q - 1) / a.total_q : 0;
+        if (b.sel_rows + app_rows > 65535) return cudaErrorInvalidValue;
+        const dim3 grid(a.total_q, b.sel_rows + app_rows);
         if (a.cu_new) {   // the overlapping append relies on nothing earlier still running
-            kern<<<dim3(a.total_q, chunks), dim3(kSelThreads), 0, stream>>>(a);
+            kern<<<grid, dim3(kSelThreads), 0, stream>>>(b);
             return cudaGetLastError();
         }
-        return launch_pdl(kern, dim3(a.total_q, chunks), dim3(kSelThreads), 0, stream, a);
+        return launch_pdl(kern, grid, dim3(kSelThreads), 0, stream, b);
     };
     if (gr <= 1) return go(select_blocks_kernel<1>, 1);
     if (gr <= 2) return go(select_blocks_kernel<2>, 2);

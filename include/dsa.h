@@ -177,12 +177,13 @@ int dsa_select_blocks(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa
                       void *workspace, size_t workspace_bytes, int32_t *dev_err, dsa_stream_t stream);
 
 /*
- * dsa_select_blocks_append -- dsa_select_blocks, then dsa_kv_append, for a
- * decode batch: the two are ordered so that the token copies overlap the
- * selection (the selection never reads them), and whatever is launched
- * after this call on `stream` sees both finished.  Same arguments and
- * results as the two calls; the selection kernel waits for all earlier work
- * on the stream before it starts.
+ * dsa_select_blocks_append -- dsa_select_blocks and dsa_kv_append in one
+ * launch, for a decode batch: the token copies run in extra CTAs of the
+ * selection's grid, overlapping the selection (which never reads them), and
+ * whatever is launched after this call on `stream` sees both finished.  Same
+ * arguments and results as the two calls; the kernel waits for all earlier
+ * work on the stream before it starts.  With no queries only the append is
+ * launched.
  *  - Every appended block of a sequence must lie at or after the own block of
  *    each of that sequence's queries; a query that breaks this gets
  *    DSA_DEV_ERR_POS and cnt 0 (its selection would read keys being written).
