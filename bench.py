@@ -274,7 +274,7 @@ def run_ours(args, world, rank, device):
     cases = [Case(args.seed + rank)]
     ab = algorithmic_bytes(cases[0].wl)
     need = max(args.rotate, math.ceil(ROTATE_L2_MULTIPLE * L2_BYTES / ab["total"]))
-    rotate = need <= MAX_ROTATE
+    rotate = need <= MAX_ROTATE and not args.no_rotate
     while rotate and len(cases) < need:
         cases.append(Case(args.seed + rank + 7919 * len(cases)))
     case0 = cases[0]
@@ -560,6 +560,8 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=1003)
     ap.add_argument("--rotate", type=int, default=2,
                     help="independent batches the timed steps rotate through (more if needed to exceed the L2)")
+    ap.add_argument("--no-rotate", action="store_true",
+                    help="one batch, each step timed after a cold-L2 flush (small profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill-indexer measurement")
     ap.add_argument("--path", choices=["auto", "fused_decode", "fused_select", "score_topk"], default="auto",

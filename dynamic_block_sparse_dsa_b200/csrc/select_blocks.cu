@@ -57,6 +57,27 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     // sequence is known, its length, Top-K and the first group's page ids
     // travel together: two round trips before the coarse keys
     const int p = __ldg(a.q_pos + t);
+    // a decode batch has one query per sequence (query t in sequence t): the
+    // sequence's facts and first page ids are loaded with the position on that
+    // guess, and reloaded below only if cu_q says otherwise
+    const bool guess = t < a.num_seqs;
+    int len = 0, K = 0, pg0[4][2];
+    auto load_seq_facts = [&](int sq) {
+        len = __ldg(a.seq_lens + sq);
+        K = __ldg(a.k_per_seq + sq);
+        // page ids of this warp's first group, before the facts are checked
+        // (rows end at max_blocks; ids past the own block are never used)
+        const int32_t *row = a.block_table + (size_t)sq * a.max_blocks;
+        const int base = c * CH + (warp * G) * 64;
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int b = base + 16 * mt + g + 8 * h;
+                pg0[mt][h] = b < a.max_blocks ? __ldg(row + b) : -1;
+            }
+    };
+    if (guess) load_seq_facts(t);
     const bool cached = a.num_seqs + 1 <= kCuqCache;
     if (cached)
         for (int i = tid; i <= a.num_seqs; i += kSelThreads) s_cuq[i] = __ldg(a.cu_q + i);
@@ -76,24 +97,9 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     } else {
         s = find_seq(a.cu_q, a.num_seqs, t);
     }
-    const int len = __ldg(a.seq_lens + s);
-    const int K = __ldg(a.k_per_seq + s);
+    if (!guess || s != t) load_seq_facts(s);
     const int n_vis = p / kBlockSize + 1;
     const int32_t *table = a.block_table + (size_t)s * a.max_blocks;
-    // page ids of this warp's first group, before the facts are checked (the
-    // bound min(own, max_blocks) keeps every load inside the table row)
-    int pg0[4][2];
-    {
-        const int lim = min(n_vis - 1, a.max_blocks);
-        const int base = c * CH + (warp * G) * 64;
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int b = base + 16 * mt + g + 8 * h;
-                pg0[mt][h] = b < lim ? __ldg(table + b) : -1;
-            }
-    }
     int32_t *out = a.sel + (size_t)t * a.k_max;
     bool bad_pos = p < 0 || p >= len || n_vis > a.max_blocks;
     if (a.cu_new && !bad_pos) {
