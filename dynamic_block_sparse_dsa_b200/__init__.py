@@ -192,9 +192,9 @@ def select_blocks_append(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatc
                          w_abs_max: int = 16, sel: Optional[torch.Tensor] = None, cnt: Optional[torch.Tensor] = None,
                          workspace: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
                          stream=None):
-    """select_blocks then kv_append for a decode batch, the copies overlapping
-    the selection: (sel, cnt).  Queries whose sequence appends a block before
-    their own block are refused (DEV_ERR_POS, cnt 0)."""
+    """select_blocks and kv_append in one launch for a decode batch, the
+    copies overlapping the selection: (sel, cnt).  Queries whose sequence
+    appends a block before their own block are refused (DEV_ERR_POS, cnt 0)."""
     lib = load()
     _expect(q_idx, torch.int8, "q_idx")
     _expect(w, torch.int32, "w")
