@@ -412,6 +412,69 @@ def test_select_append_flags_non_decode_queries(cuda_device):
     assert (bufs["cnt"].cpu().numpy()[~ok] == 0).all()
 
 
+def _appended_rows_match(wl, n_tokens):
+    """Every new token's K and V rows sit in their page slots, and the coarse
+    key of the last new token of each touched block is that block's key."""
+    spec = wl.spec
+    table = wl.block_table.cpu().numpy()
+    cu = wl.cu_q.cpu().numpy()
+    lens = wl.seq_lens.cpu().numpy()
+    kp, vp, kcp = wl.k_pool.cpu(), wl.v_pool.cpu(), wl.kc_pool.cpu()
+    kn, vn, kcn = wl.k_new.cpu(), wl.v_new.cpu(), wl.kc_new.cpu()
+    for s_ in range(spec.num_seqs):
+        n = int(cu[s_ + 1] - cu[s_])
+        for j in range(n):
+            i = int(cu[s_]) + j
+            pos = int(lens[s_]) - n + j
+            page, slot = int(table[s_, pos // 64]), pos % 64
+            assert torch.equal(kp[page, slot], kn[i]) and torch.equal(vp[page, slot], vn[i]), (s_, j)
+            if j == n - 1 or slot == 63:
+                assert torch.equal(kcp[page], kcn[i]), (s_, j)
+    assert n_tokens == int(cu[-1])
+
+
+def test_select_append_more_tokens_than_queries(cuda_device):
+    """Three new tokens per sequence, all in its last block, but only the last
+    one queries: the selection's grid carries three rows of append CTAs.  The
+    selection equals the oracle's for those queries and the pool holds every
+    new token."""
+    spec = wk.WorkloadSpec("append3", seq_lens=(700, 1300, 70, 4000), n_new=(3, 3, 3, 3), k_per_seq=(4, 6, 2, 8),
+                           k_max=8, num_q_heads=16, num_kv_heads=2, num_idx_heads=16)
+    wl = wk.make_workload(spec, seed=321, device=cuda_device)
+    cu = wl.cu_q.cpu().numpy()
+    last = [int(cu[s_ + 1] - 1) for s_ in range(spec.num_seqs)]
+    ref = oracle_step(wl, queries=last)
+    idx = torch.as_tensor(last, device=cuda_device)
+    cache, seqs, _ = _handles(wl)
+    queries = dsa.QueryBatch(torch.arange(spec.num_seqs + 1, dtype=torch.int32, device=cuda_device),
+                             wl.q_pos.index_select(0, idx).contiguous())
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    sel, cnt = dsa.select_blocks_append(cache, seqs, queries, wl.cu_q, wl.k_new, wl.v_new, wl.kc_new,
+                                        wl.q_idx.index_select(0, idx).contiguous(),
+                                        wl.w.index_select(0, idx).contiguous(), wl.k_per_seq, spec.k_max,
+                                        dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert np.array_equal(cnt.cpu().numpy(), ref["cnt"])
+    assert np.array_equal(sel.cpu().numpy(), ref["sel"])
+    _appended_rows_match(wl, 12)
+
+
+def test_select_append_without_queries_still_appends(cuda_device):
+    """No queries: no selection launch, only the append."""
+    wl = wk.make_workload(_small_spec("many_seqs_decode"), seed=322, device=cuda_device)
+    spec = wl.spec
+    cache, seqs, _ = _handles(wl)
+    queries = dsa.QueryBatch(torch.zeros(spec.num_seqs + 1, dtype=torch.int32, device=cuda_device),
+                             torch.empty(0, dtype=torch.int32, device=cuda_device))
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    sel, cnt = dsa.select_blocks_append(cache, seqs, queries, wl.cu_q, wl.k_new, wl.v_new, wl.kc_new,
+                                        wl.q_idx[:0], wl.w[:0], wl.k_per_seq, spec.k_max, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and sel.shape[0] == 0 and cnt.shape[0] == 0
+    _appended_rows_match(wl, spec.num_seqs)
+
+
 @pytest.mark.parametrize("q_scale", [1.0, 12.0])
 def test_select_append_batched_gqa_workload(q_scale, cuda_device):
     spec = wk.scaled(wk.batched_gqa_decode(), q_scale=q_scale)
