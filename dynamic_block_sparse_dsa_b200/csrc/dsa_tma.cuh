@@ -112,18 +112,20 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
 }
-__device__ __forceinline__ void st_cluster_f32x4(uint32_t addr, float x, float y, float z, float w) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(x), "f"(y), "f"(z), "f"(w)
+// asynchronous stores into another CTA's shared memory that complete their
+// bytes on that CTA's mbarrier (which must expect them): no fence, no arrival
+__device__ __forceinline__ void st_async_f32x4(uint32_t addr, float x, float y, float z, float w, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(addr), "f"(x), "f"(y), "f"(z), "f"(w), "r"(bar)
                  : "memory");
 }
-__device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float x, float y) {
-    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
+__device__ __forceinline__ void st_async_f32x2(uint32_t addr, float x, float y, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(addr),
+                 "f"(x), "f"(y), "r"(bar)
+                 : "memory");
 }
-// arrive on an mbarrier of another CTA of the cluster, releasing this
-// thread's (and, through a preceding barrier, its CTA's) earlier stores
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
-}
+// test-wait on this CTA's mbarrier with acquire at cluster scope, so that a
+// partner CTA's stores that completed on it are visible
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
     uint32_t done;
     asm volatile(

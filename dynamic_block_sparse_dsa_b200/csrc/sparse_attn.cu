@@ -60,6 +60,8 @@ constexpr int kNumWords = kWSelLast + 1;
 constexpr float kLn2 = 0.6931471805599453f;
 // most CTAs whose ranges can cover one pair (the host caps the split at 60)
 constexpr int kMaxSplitSlots = 63;
+// bytes rank 1 sends per head row in 2-CTA cluster mode: o[128] then (m, l)
+constexpr uint32_t kInboxRowBytes = 128 * 4 + 2 * 4;
 
 // shared-memory plan for NT head tiles: a group of <= 8 heads leaves room for
 // a sixth ring stage; 16-head groups need the larger merge buffer
@@ -176,6 +178,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         for (int s = 0; s < kSegSlots; ++s) W[kWSegEndTag + s] = -1;
         if (kFused) W[kWTag] = fused::ld_acquire(f.hdr + kHdrEpoch) + 1;
         fence_barrier_init();
+        // 2-CTA cluster mode: rank 0's inbox expects the partner's merged state
+        // (G rows of o[128], m, l) before the cluster barrier below lets the
+        // partner send it
+        if (a.cluster2 && !(blockIdx.x & 1)) mbar_arrive_expect_tx(sm.inbox_full(), (uint32_t)a.group * kInboxRowBytes);
     }
     pdl_trigger();
     __syncthreads();
@@ -581,19 +587,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 Ao[i][0] = acc[0]; Ao[i][1] = acc[1]; Ao[i][2] = acc[2]; Ao[i][3] = acc[3];
             }
             if (c & 1) {
+                // asynchronous stores that complete their bytes on rank 0's inbox
+                // barrier (armed with the full count before the cluster barrier)
                 const uint32_t remote = mapa_shared(sm.inbox(), 0);
+                const uint32_t remote_bar = mapa_shared(sm.inbox_full(), 0);
 #pragma unroll
                 for (int i = 0; i < kRowsPT; ++i) {
                     const int e = tid + i * kConsumerWarps * 32;
                     if (e >= G * 32) break;
                     const int r = e >> 5, d0 = (e & 31) * 4;
                     const uint32_t row = remote + (uint32_t)(r * kAttnPartStride * 4);
-                    st_cluster_f32x4(row + d0 * 4, Ao[i][0], Ao[i][1], Ao[i][2], Ao[i][3]);
-                    if (d0 == 0) st_cluster_f32x2(row + 128 * 4, Mo[i], Lo[i]);
+                    st_async_f32x4(row + d0 * 4, Ao[i][0], Ao[i][1], Ao[i][2], Ao[i][3], remote_bar);
+                    if (d0 == 0) st_async_f32x2(row + 128 * 4, Mo[i], Lo[i], remote_bar);
                 }
-                __syncwarp();
-                named_barrier(1, kConsumerWarps * 32);
-                if (tid == 0) mbar_arrive_remote(mapa_shared(sm.inbox_full(), 0));
             } else {
                 // the partner's state; the wait outlasts any bounded stall of the partner
                 bool got = mbar_try_wait_cluster(sm.inbox_full(), 0);
