@@ -19,16 +19,22 @@
 //     shared-memory ring
 //     guarded by full/empty mbarriers; it also TMA-loads the 16-row query tile
 //     of each (query, KV head) pair into a 2-slot ring;
-//   * four consumer warps take whole blocks round-robin.  Each runs the GQA
-//     group of query heads (rows of an m16 tile) against its 64 tokens on the
-//     tensor cores with mma.m16n8k16 bf16/fp32: S = Q K^T, online softmax in
-//     fp32 with base-2 exponents and the causal mask of the own block, then
-//     O += P V with P reused from the S accumulators as the A operand;
+//   * four consumer warps take whole blocks round-robin.  Each runs its 64
+//     tokens against the GQA group of query heads on the tensor cores with
+//     mma.m16n8k16 bf16/fp32 in swap-AB form (the keys are the M dimension,
+//     the <= 8 or 16 query heads N): S^T = K Q^T, online softmax in fp32 with
+//     base-2 exponents and the causal mask of the own block, then
+//     O^T += V^T P^T with P^T built from the score fragments by movmatrix;
 //   * at the end of each pair the four warps' softmax states are merged in a
 //     fixed order through shared memory.  A pair that lies wholly inside the
 //     CTA is written straight out; a pair split across CTAs leaves a partial
 //     (m, l, unnormalised O) in the workspace and the CTA completing its units
-//     -- counted with an atomic, no waiting -- merges the partials.
+//     -- counted with an atomic, no waiting -- merges the partials;
+//   * decode batches with between C/4 and C/2 pairs run one 2-CTA cluster per
+//     pair instead: each rank takes half of the pair's blocks, and rank 1 hands
+//     its merged state to rank 0 with st.async stores that complete their
+//     bytes on rank 0's inbox mbarrier (armed with the full count before the
+//     start-of-kernel cluster barrier); rank 0 combines and writes the output.
 // All waits are bounded (DSA_DEV_ERR_WAIT on timeout, no hang).
 #include "dsa_kernels.h"
 #include "dsa_tma.cuh"
