@@ -32,8 +32,9 @@
 //   1     MMA issuer (one thread): two K = 32 MMAs per item into one of two
 //         256-column accumulators;
 //   2-17  epilogue (four per SM sub-partition: a quarter of the rows and a
-//         quarter of the queries each): tcgen05.ld, relu * w summed over heads,
-//         one coalesced 128-byte store per (query, warp).
+//         quarter of the queries each): tcgen05.ld, after which the
+//         accumulator goes straight back to the MMA, then relu * w summed
+//         over heads and one coalesced 128-byte store per (query, warp).
 // A query tile spanning several sequences runs once per sequence with the
 // other queries masked; items past every query's own block are skipped.  All
 // waits are bounded.
