@@ -423,14 +423,21 @@ def run_ours(args, world, rank, device):
             self.bufs["out"] = view(self.dev_out_buf, out_offs["out"], c.bufs["out"])
             self.bufs["lse"] = view(self.dev_out_buf, out_offs["lse"], c.bufs["lse"])
             self.c = c
+            self.in_ready = torch.cuda.Event()   # graph only: this batch's inputs landed
+            self.consumed = torch.cuda.Event()   # its step ran
+            self.out_done = torch.cuda.Event()   # its outputs read back
 
-        def step(self):
+        def compute(self):
             c, d = self.c, self.dev_in
-            self.dev_in_buf.copy_(self.host_in, non_blocking=True)
             dsa.step(c.cache, c.seqs, c.queries, k_new=d["k_new"], v_new=d["v_new"], kc_new=d["kc_new"], q=d["q"],
                      q_idx=d["q_idx"], w=d["w"], k_per_seq=c.wl.k_per_seq, k_max=spec.k_max, decode=decode,
                      fused_select=fused, overlap_append=fused and decode, fused_decode=fused_decode,
                      bufs=self.bufs, dev_err=err)
+
+        def step(self):
+            """copy in, step, copy out, all on the current stream"""
+            self.dev_in_buf.copy_(self.host_in, non_blocking=True)
+            self.compute()
             self.host_out.copy_(self.dev_out_buf, non_blocking=True)
 
     staged = [Staged(c) for c in cases]
@@ -439,10 +446,30 @@ def run_ours(args, world, rank, device):
         with torch.cuda.stream(stream):
             st.step()
     torch.cuda.synchronize(device)
+    # the graph: all of a rotation's input copies on one side stream, its steps
+    # on the main stream, each step's read-back on another side stream as soon
+    # as that step is done, so the copies overlap the other batches' steps
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
     graph_e2e = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph_e2e, stream=stream):
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        s_in.wait_event(fork)
+        s_out.wait_event(fork)
         for st in staged:
-            st.step()
+            with torch.cuda.stream(s_in):
+                st.dev_in_buf.copy_(st.host_in, non_blocking=True)
+                st.in_ready.record(s_in)
+        for st in staged:
+            stream.wait_event(st.in_ready)
+            st.compute()
+            st.consumed.record(stream)
+            s_out.wait_event(st.consumed)
+            with torch.cuda.stream(s_out):
+                st.host_out.copy_(st.dev_out_buf, non_blocking=True)
+                st.out_done.record(s_out)
+        for st in staged:
+            stream.wait_event(st.out_done)
     torch.cuda.synchronize(device)
     n_e2e = max(3 * n_case, min(args.steps, 150)) // n_case * n_case
     e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -451,11 +478,15 @@ def run_ours(args, world, rank, device):
         if rotate:
             with torch.cuda.stream(stream):
                 e_s.record()
-                for i in range(n_e2e if eager else n_e2e // n_case):
-                    if eager:
+            if eager:
+                with torch.cuda.stream(stream):
+                    for i in range(n_e2e):
                         staged[i % n_case].step()
-                    else:
+            else:
+                with torch.cuda.stream(stream):
+                    for i in range(n_e2e // n_case):
                         graph_e2e.replay()
+            with torch.cuda.stream(stream):
                 e_e.record()
             stream.synchronize()
             total = e_s.elapsed_time(e_e) / 1e3
@@ -480,9 +511,10 @@ def run_ours(args, world, rank, device):
     e2e = {"value": e2e_eager, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "how": ("dsa.step called from Python every step, steps back to back over the independent batches; "
                    "each step's inputs staged in one pinned buffer (one H2D copy) and out/lse read back from one "
-                   "device buffer (one D2H copy), inside the timed region"),
+                   "device buffer (one D2H copy), on the step's stream, inside the timed region"),
            "graph_value": e2e_graph,
-           "graph_how": "the same copies and calls captured once in a CUDA graph per rotation, replayed"}
+           "graph_how": ("the same copies and calls captured once per rotation in a CUDA graph whose input copies "
+                         "and read-backs run on side streams, overlapping the other batches' steps; replayed")}
     del graph_e2e, rot_graph, rot_attn
 
     res = {
