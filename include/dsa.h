@@ -32,6 +32,14 @@
  *    offending item is skipped; the caller reads the word back when it likes.
  *  - Sizes in v1: block_size 64, head_dim 128, idx_dim 64; query heads per KV
  *    head 1..16; indexer heads 1..16.  Anything else is DSA_ERR_UNSUPPORTED.
+ *  - Consecutive calls on one stream overlap: each kernel lets the next one
+ *    start early (programmatic dependent launch) and waits for its
+ *    predecessor before it reads anything a library call writes (the pools,
+ *    scores, selections).  Before that wait a kernel may already read the
+ *    batch description and its own inputs (block_table, seq_lens, cu_q, q_pos,
+ *    k_per_seq, q_idx, w, q): these must not be outputs of the library call
+ *    issued just before it on the same stream.  Work from other kernels is
+ *    waited for in full, as usual.
  *
  * KV cache layout [P5 "KV Cache Layout"; P1 4(2) two storage types]:
  *   k_pool, v_pool : bf16  [num_pages][block_size][num_kv_heads][head_dim]
