@@ -120,3 +120,40 @@ def test_topk_and_append_validation_codes():
                              None) == _lib.DSA_ERR_INVALID_ARG
     assert lib.dsa_kv_append(ctypes.byref(c), ctypes.byref(s), FAKE, 0, FAKE, FAKE, None, None,
                              None) == _lib.DSA_OK
+
+
+def test_select_validation_codes():
+    lib = _lib.load()
+    c, s, q = _cache(), _seqs(), _queries()
+
+    def sel(queries=q, heads=16, wmax=16, k_max=32, ws=FAKE, ws_bytes=1 << 20):
+        return lib.dsa_select_blocks(ctypes.byref(c), ctypes.byref(s), ctypes.byref(queries), FAKE, FAKE, heads,
+                                     wmax, FAKE, k_max, FAKE, FAKE, ws, ws_bytes, None, None)
+
+    assert sel(k_max=65) == _lib.DSA_ERR_UNSUPPORTED        # the fused path keeps at most 64
+    assert sel(heads=17) == _lib.DSA_ERR_UNSUPPORTED
+    assert sel(wmax=128) == _lib.DSA_ERR_RANGE
+    assert sel(ws=None) == _lib.DSA_ERR_WORKSPACE
+    assert sel(ws_bytes=16) == _lib.DSA_ERR_WORKSPACE
+    assert sel(ws=FAKE + 8) == _lib.DSA_ERR_WORKSPACE        # misaligned workspace
+    assert sel(queries=_queries(total_q=0), ws=None, ws_bytes=0) == _lib.DSA_OK
+    assert lib.dsa_select_blocks_workspace_size(0) == 0
+    assert lib.dsa_select_blocks_workspace_size(8) > 0
+
+
+def test_select_append_validation_codes():
+    lib = _lib.load()
+    c, s = _cache(), _seqs()
+
+    def sa(queries=None, cu_new=FAKE, total_new=1, k_new=FAKE, v_new=FAKE):
+        queries = queries or _queries()
+        return lib.dsa_select_blocks_append(ctypes.byref(c), ctypes.byref(s), ctypes.byref(queries), cu_new,
+                                            total_new, k_new, v_new, None, FAKE, FAKE, 16, 16, FAKE, 32, FAKE,
+                                            FAKE, FAKE, 1 << 20, None, None)
+
+    assert sa(total_new=-1) == _lib.DSA_ERR_INVALID_ARG
+    assert sa(cu_new=None) == _lib.DSA_ERR_INVALID_ARG
+    assert sa(k_new=FAKE + 2) == _lib.DSA_ERR_INVALID_ARG     # misaligned token rows
+    assert sa(v_new=None) == _lib.DSA_ERR_INVALID_ARG
+    # no queries and no tokens: nothing to launch
+    assert sa(queries=_queries(total_q=0), total_new=0) == _lib.DSA_OK
