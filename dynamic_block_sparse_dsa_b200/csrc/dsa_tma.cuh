@@ -57,19 +57,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const v
     }
 }
 
-// wait until *word == value (a shared-memory word another warp writes);
-// false on timeout or when *abort becomes non-zero
-__device__ __forceinline__ bool wait_value(const volatile int *word, int value, const volatile int *abort) {
-    if (*word == value) return true;
-    const long long t0 = clock64();
-#pragma unroll 1
-    while (*word != value) {
-        if (*abort) return false;
-        if (clock64() - t0 > kWaitLimitCycles) return false;
-    }
-    return true;
-}
-
 // 2-D / 3-D tiled TMA loads into shared memory, completing on an mbarrier
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
     asm volatile(
