@@ -218,8 +218,10 @@ int dsa_select_blocks_append(const dsa_kv_cache *cache, const dsa_seqs *seqs, co
  *   lse fp32 [total_q][num_q_heads] (may be NULL)
  * Both entries run one persistent CTA per SM over the list of (query, KV
  * head, selected block) units, split evenly.  The decode entry may split a
- * (query, KV head) pair across CTAs and merge the partial softmax states; it
- * needs a workspace of dsa_sparse_attn_decode_workspace_size() bytes (a
+ * (query, KV head) pair across CTAs and merge the partial softmax states
+ * (through the workspace, or, when the batch has between a quarter and a half
+ * as many pairs as the GPU has SMs, inside a 2-CTA cluster through
+ * distributed shared memory); it needs a workspace of dsa_sparse_attn_decode_workspace_size() bytes (a
  * 4-byte counter per (query, KV head) pair plus room for two partial states
  * per CTA), zero-filled before its first use (each call leaves it zeroed
  * again).  The prefill entry keeps every pair
