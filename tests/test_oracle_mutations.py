@@ -35,6 +35,14 @@ MUTATIONS = {
                           "int last_in_block = (i == cu_new[s]) || (slot == 0);"),
     "kv_swapped": ("k_pool[dst + e] = k_new[(long)i * row + e];\n                v_pool[dst + e] = v_new[(long)i * row + e];",
                    "k_pool[dst + e] = v_new[(long)i * row + e];\n                v_pool[dst + e] = k_new[(long)i * row + e];"),
+    "lse_base2": ("n_tok > 0 ? m + log(denom) : -INFINITY;", "n_tok > 0 ? m + log2(denom) : -INFINITY;"),
+    "lse_max_dropped": ("n_tok > 0 ? m + log(denom) : -INFINITY;", "n_tok > 0 ? log(denom) : -INFINITY;"),
+    "v_rows_from_k": ("const uint16_t *vj = v_pool + (tok_row[j] * num_kv_heads + kvh) * head_dim;",
+                      "const uint16_t *vj = k_pool + (tok_row[j] * num_kv_heads + kvh) * head_dim;"),
+    "ids_not_sorted": ("qsort(out, (size_t)n, sizeof(int32_t), int_ascending);", "(void)int_ascending;"),
+    "one_candidate_short": ("for (int i = 0; i < k - 1; ++i) out[n++] = cand[i].block;",
+                            "for (int i = 0; i < k - 2; ++i) out[n++] = cand[i].block;"),
+    "append_one_slot_late": ("return seq_lens[s] - n + (i - cu_new[s]);", "return seq_lens[s] - n + (i - cu_new[s]) + 1;"),
 }
 
 
