@@ -8,7 +8,12 @@ the current CUDA stream); all of the method runs in the library's kernels:
     index_score          int8 indexer: block scores of each query
     topk_blocks          own block + Top-(K-1) blocks, ascending logical ids
     sparse_attn_decode   exact attention over the selected blocks (split-KV)
-    sparse_attn_prefill  same, one CTA per (query, KV head)
+    sparse_attn_prefill  same, each (query, KV head) pair inside one CTA
+
+and the fused forms: select_blocks (score + Top-K, no score matrix),
+select_blocks_append (the same with the append in one launch, decode),
+decode_fused (a whole decode step in one launch), sparse_attn_decode_noalloc
+(decode attention without a caller workspace), and step() chaining one pass.
 
 Pages followed (cited by title and section): "Day-0 Adaptation for Massive
 LLMs: Overcoming Sparse Attention and MXFP4 Expert Weights", section 4;
@@ -30,8 +35,9 @@ from ._lib import DsaError, load
 
 __all__ = [
     "PagedKVCache", "SeqBatch", "QueryBatch", "DsaError", "load",
-    "kv_append", "index_score", "topk_blocks", "select_blocks", "sparse_attn_decode", "sparse_attn_prefill",
-    "decode_workspace_size", "select_workspace_size", "sparse_attn_decode_noalloc", "step",
+    "kv_append", "index_score", "topk_blocks", "select_blocks", "select_blocks_append", "sparse_attn_decode",
+    "sparse_attn_prefill", "decode_fused", "decode_workspace_size", "select_workspace_size",
+    "decode_fused_workspace_size", "sparse_attn_decode_noalloc", "step",
 ]
 
 BLOCK_SIZE = 64
