@@ -157,3 +157,27 @@ def test_select_append_validation_codes():
     assert sa(v_new=None) == _lib.DSA_ERR_INVALID_ARG
     # no queries and no tokens: nothing to launch
     assert sa(queries=_queries(total_q=0), total_new=0) == _lib.DSA_OK
+
+
+def test_binding_refuses_host_tensors():
+    """The binding has no CPU path: host tensors are refused with an error
+    before anything is called, whatever the entry point."""
+    import torch
+
+    import dynamic_block_sparse_dsa_b200 as dsa
+    k = torch.zeros(4, 64, 1, 128, dtype=torch.bfloat16)
+    cache = dsa.PagedKVCache(k, k.clone(), torch.zeros(4, 64, dtype=torch.int8))
+    seqs = dsa.SeqBatch(torch.zeros(1, 4, dtype=torch.int32), torch.tensor([100], dtype=torch.int32))
+    queries = dsa.QueryBatch(torch.tensor([0, 1], dtype=torch.int32), torch.tensor([99], dtype=torch.int32))
+    q_idx = torch.zeros(1, 4, 64, dtype=torch.int8)
+    w = torch.zeros(1, 4, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        dsa.index_score(cache, seqs, queries, q_idx, w)
+    with pytest.raises(ValueError, match="CUDA"):
+        dsa.kv_append(cache, seqs, queries.cu_q, torch.zeros(1, 1, 128, dtype=torch.bfloat16),
+                      torch.zeros(1, 1, 128, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="CUDA"):
+        dsa.step(cache, seqs, queries, k_new=torch.zeros(1, 1, 128, dtype=torch.bfloat16),
+                 v_new=torch.zeros(1, 1, 128, dtype=torch.bfloat16), kc_new=None,
+                 q=torch.zeros(1, 8, 128, dtype=torch.bfloat16), q_idx=q_idx, w=w,
+                 k_per_seq=torch.tensor([2], dtype=torch.int32), k_max=2)
