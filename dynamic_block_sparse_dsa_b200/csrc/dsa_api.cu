@@ -163,6 +163,15 @@ int select_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_que
 
 }  // namespace
 
+namespace dsa {
+int check_decode_attn_args(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                           const void *q, int32_t num_q_heads, const int32_t *sel, const int32_t *cnt,
+                           int32_t k_max, float sm_scale, void *out, float *lse) {
+    AttnArgs a;
+    return attn_common(cache, seqs, queries, q, num_q_heads, sel, cnt, k_max, sm_scale, out, lse, nullptr, a);
+}
+}  // namespace dsa
+
 extern "C" {
 
 int dsa_version(void) { return 100; }

@@ -179,6 +179,11 @@ int topk_max_blocks();   // longest block table the standalone Top-K kernel acce
 // the K/V pool and Q tensor maps are built by the launcher from AttnArgs
 cudaError_t launch_sparse_attn(const AttnArgs &a, cudaStream_t stream);
 cudaError_t launch_decode_fused(const AttnArgs &a, const FusedArgs &f, cudaStream_t stream);
+// host-side checks of dsa_sparse_attn_decode's arguments, without any CUDA
+// call: DSA_OK or the status the entry point would return
+int check_decode_attn_args(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                           const void *q, int32_t num_q_heads, const int32_t *sel, const int32_t *cnt,
+                           int32_t k_max, float sm_scale, void *out, float *lse);
 // largest grid the attention kernel uses (sizes the partial-state workspace)
 constexpr int kAttnMaxCtas = 256;
 // floats per partial-state row: o[128], m, l, padded to a 16-byte multiple

@@ -20,9 +20,12 @@ Every workload is a batch of sequences sharing one block-paged KV pool:
   (``k_new``/``v_new``) and coarse-key rows (``kc_new``) are inputs of the
   append step.
 
-Value distributions: bf16 q/k/v ~ N(0,1)/sqrt(head_dim) (times ``q_scale`` for
-the sharpened-softmax cases); int8 indexer queries and coarse keys uniform in
-[-127, 127]; int32 head weights uniform in [0, w_max].
+Value distributions: bf16 q/k/v ~ N(0,1)/sqrt(head_dim), q times ``q_scale``
+and v times ``v_scale`` for the discriminative cases (``sharp()``: logits with
+standard deviation 2 and unit-variance values, so that attention outputs are
+O(0.1) rather than O(0.002)); int8 indexer queries and coarse keys uniform in
+[-127, 127]; int32 head weights uniform in [w_min, w_max] (w_min = 0 unless a
+case asks for signed weights).
 """
 from __future__ import annotations
 
@@ -51,10 +54,12 @@ class WorkloadSpec:
     idx_dim: int = 64
     block_size: int = 64
     w_max: int = 16
+    w_min: int = 0             # signed-weight cases draw w uniformly from [w_min, w_max]
     occupancy: float = 1.0     # fraction of pool pages that hold a sequence's block
     plant: int = 0             # planted blocks per sequence (decode sequences)
     plant_sigma: float = 3.0
     q_scale: float = 1.0       # multiplies q before bf16 rounding (sharper softmax)
+    v_scale: float = 1.0       # multiplies v (pool and new tokens) before bf16 rounding
 
     @property
     def num_seqs(self) -> int:
@@ -223,16 +228,16 @@ def make_workload(spec: WorkloadSpec, seed: int = 0, device="cpu") -> Workload:
     hd = spec.head_dim
     scale = 1.0 / math.sqrt(hd)
     k_pool = _normal_bf16((num_pages, bs, spec.num_kv_heads, hd), scale, gdev, device)
-    v_pool = _normal_bf16((num_pages, bs, spec.num_kv_heads, hd), scale, gdev, device)
+    v_pool = _normal_bf16((num_pages, bs, spec.num_kv_heads, hd), scale * spec.v_scale, gdev, device)
     kc_pool = torch.randint(-127, 128, (num_pages, spec.idx_dim), generator=gdev, device=device,
                             dtype=torch.int8)
     q = _normal_bf16((T, spec.num_q_heads, hd), scale * spec.q_scale, gdev, device)
     q_idx = torch.randint(-127, 128, (T, spec.num_idx_heads, spec.idx_dim), generator=gdev,
                           device=device, dtype=torch.int8)
-    w = torch.randint(0, spec.w_max + 1, (T, spec.num_idx_heads), generator=gdev, device=device,
+    w = torch.randint(spec.w_min, spec.w_max + 1, (T, spec.num_idx_heads), generator=gdev, device=device,
                       dtype=torch.int32)
     k_new = _normal_bf16((T, spec.num_kv_heads, hd), scale, gdev, device)
-    v_new = _normal_bf16((T, spec.num_kv_heads, hd), scale, gdev, device)
+    v_new = _normal_bf16((T, spec.num_kv_heads, hd), scale * spec.v_scale, gdev, device)
     kc_new = torch.randint(-127, 128, (T, spec.idx_dim), generator=gdev, device=device,
                            dtype=torch.int8)
 
@@ -298,3 +303,17 @@ def _plant(wl: Workload, gcpu: torch.Generator) -> None:
 def scaled(spec: WorkloadSpec, **kw) -> WorkloadSpec:
     """A copy of ``spec`` with fields replaced (e.g. q_scale, name)."""
     return replace(spec, **kw)
+
+
+# q x 256 makes the logit q.k/sqrt(128) a N(0, 2^2) variable (q, k ~ N(0,1)/sqrt(128)
+# per element), so the softmax over a few thousand tokens is dominated by a few
+# dozen of them; v x sqrt(128) makes the values N(0,1).  The attention output
+# is then O(0.1-1), far above the 2e-3 mean tolerance, and a wrong head, page
+# or weight moves it by O(0.1).
+SHARP_Q_SCALE = 256.0
+SHARP_V_SCALE = math.sqrt(128.0)
+
+
+def sharp(spec: WorkloadSpec) -> WorkloadSpec:
+    """``spec`` with the discriminative value scales (see SHARP_Q_SCALE)."""
+    return replace(spec, q_scale=SHARP_Q_SCALE, v_scale=SHARP_V_SCALE)

@@ -181,3 +181,32 @@ def test_binding_refuses_host_tensors():
                  v_new=torch.zeros(1, 1, 128, dtype=torch.bfloat16), kc_new=None,
                  q=torch.zeros(1, 8, 128, dtype=torch.bfloat16), q_idx=q_idx, w=w,
                  k_per_seq=torch.tensor([2], dtype=torch.int32), k_max=2)
+
+
+def test_noalloc_refuses_bad_calls_before_any_device_work():
+    """The allocation-free decode entry runs every host check of the regular
+    decode entry before it enqueues anything on its shared scratch.  Without a
+    GPU any CUDA call would fail with DSA_ERR_CUDA, so getting the argument
+    error back here shows that the check came first.  The pointers are
+    dummies that are never dereferenced."""
+    lib = _lib.load()
+    s = _seqs()
+
+    def na(cache=None, total_q=4_500_000, hq=64, k_max=32, scale=0.088, out=FAKE):
+        cache = cache or _cache()
+        q = _queries(total_q=total_q)
+        return lib.dsa_sparse_attn_decode_noalloc(ctypes.byref(cache), ctypes.byref(s), ctypes.byref(q), FAKE, hq,
+                                                  FAKE, FAKE, k_max, scale, out, None, None, None)
+
+    # 63 query heads over 8 KV heads: the workspace size query says 0 for this,
+    # and 4.5M queries x 8 KV heads of split counters would overrun the scratch
+    assert na(hq=63) == _lib.DSA_ERR_INVALID_ARG
+    assert na(hq=8 * 17, total_q=4) == _lib.DSA_ERR_UNSUPPORTED
+    assert na(k_max=0) == _lib.DSA_ERR_INVALID_ARG
+    assert na(scale=0.0) == _lib.DSA_ERR_INVALID_ARG
+    assert na(out=FAKE + 2) == _lib.DSA_ERR_INVALID_ARG
+    assert na(cache=_cache(block_size=32)) == _lib.DSA_ERR_UNSUPPORTED
+    # valid arguments, but more scratch than the fixed array holds
+    assert na() == _lib.DSA_ERR_WORKSPACE
+    # nothing to do: accepted without touching the device
+    assert na(total_q=0) == _lib.DSA_OK

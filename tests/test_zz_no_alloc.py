@@ -4,8 +4,10 @@ dsa_sparse_attn_decode_noalloc serves callers that cannot call cudaMalloc
 (an engine plugin's enqueue path, a runtime that owns all device memory): its
 split-KV scratch is a fixed array inside the library.  Two calls in a row --
 the second one finds the first one's leftovers in that shared array -- must
-match dsa_sparse_attn_decode on the same selection, within the parity
-tolerance of the other GPU tests.  This file is collected last on purpose.
+match dsa_sparse_attn_decode on the same selection, and the oracle, within the
+parity tolerance of the other GPU tests.  The inputs use the discriminative
+value scales (q x 256, v x sqrt(128)), so the outputs are O(0.1), far above
+the tolerance.  This file is collected last on purpose.
 """
 import numpy as np
 import pytest
@@ -13,6 +15,7 @@ import torch
 
 import dynamic_block_sparse_dsa_b200 as dsa
 from dynamic_block_sparse_dsa_b200 import workloads as wk
+from oracle.harness import oracle_step
 
 pytestmark = pytest.mark.gpu
 
@@ -30,13 +33,19 @@ def _setup(spec, seed, device):
 
 
 @pytest.mark.parametrize("name,spec", [
-    ("decode_8x32_blocks", wk.WorkloadSpec("na1", seq_lens=(1 << 16,) * 8, n_new=(1,) * 8, k_per_seq=(32,) * 8,
-                                           k_max=32, q_scale=8.0)),
-    ("ragged_small", wk.WorkloadSpec("na2", seq_lens=(900, 70, 4000), n_new=(1, 1, 1), k_per_seq=(8, 2, 16),
-                                     k_max=16, num_q_heads=16, num_kv_heads=2)),
+    # 64 (query, KV head) pairs: the 2-CTA cluster split
+    ("decode_8x32_blocks", wk.sharp(wk.WorkloadSpec("na1", seq_lens=(1 << 16,) * 8, n_new=(1,) * 8,
+                                                    k_per_seq=(32,) * 8, k_max=32))),
+    # 6 pairs: the split through the scratch's partial states and counters
+    ("ragged_small", wk.sharp(wk.WorkloadSpec("na2", seq_lens=(900, 70, 4000), n_new=(1, 1, 1),
+                                              k_per_seq=(8, 2, 16), k_max=16, num_q_heads=16, num_kv_heads=2))),
 ])
 def test_noalloc_matches_regular_decode_twice(name, spec, cuda_device):
     wl, cache, seqs, queries, sel, cnt = _setup(spec, 77, cuda_device)
+    # the oracle on the same (un-appended) pool and its own selection
+    orc = oracle_step(wl, with_append=False)
+    assert np.array_equal(sel.cpu().numpy(), orc["sel"]) and np.array_equal(cnt.cpu().numpy(), orc["cnt"])
+    assert np.abs(orc["out"]).mean() >= 10 * OUT_MEAN     # the case can tell a wrong output from a right one
     err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
     ref_out, ref_lse = dsa.sparse_attn_decode(cache, seqs, queries, wl.q, sel, cnt, dev_err=err)
     for _ in range(2):
@@ -48,6 +57,9 @@ def test_noalloc_matches_regular_decode_twice(name, spec, cuda_device):
         d = (out.double() - ref_out.double()).abs()
         assert float(d.max()) <= OUT_MAX and float(d.mean()) <= OUT_MEAN
         assert float((lse - ref_lse).abs().max()) <= LSE_MAX
+        do = np.abs(out.double().cpu().numpy() - orc["out"])
+        assert do.max() <= OUT_MAX and do.mean() <= OUT_MEAN, (do.max(), do.mean())
+        assert np.abs(lse.double().cpu().numpy() - orc["lse"]).max() <= LSE_MAX
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(cuda_device):
