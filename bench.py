@@ -690,9 +690,19 @@ def measure_workload(name, device, steps=30, iso=15, seed=None):
         rec["step_bytes"] = ab["total"]
         rec["step_gbs"] = round(ab["total"] / step_s / 1e9, 1)
         rec["step_frac_of_measured_hbm"] = round(ab["total"] / step_s / 1e9 / peak, 4)
-    for pname, fn in c0.phases():
-        g, ev = c0.capture(fn)
-        us = statistics.median(tm.isolated(g, ev, iso)) * 1e3
+    for i, (pname, _) in enumerate(c0.phases()):
+        if rotate:
+            # the launch alone, back to back over the batches (as in the step)
+            singles = [c.capture(c.phases()[i][1])[0] for c in cases]
+            whole = rotation_graph(cases, lambda c: c.phases()[i][1], stream, device)
+            tm.rotated(whole, singles, len(cases))
+            n = max(steps, 3 * len(cases))
+            us = tm.rotated(whole, singles, n) / n * 1e6
+            del whole, singles
+        else:
+            g, ev = c0.capture(c0.phases()[i][1])
+            us = statistics.median(tm.isolated(g, ev, iso)) * 1e3
+            del g
         ph = {"us": round(us, 2)}
         if pname == "attention":
             gbs = kv_gb / us / 1e3
@@ -707,8 +717,9 @@ def measure_workload(name, device, steps=30, iso=15, seed=None):
             ph.update({"int8_ops": ops, "tops": round(ops / us / 1e6, 1), "frac_of_int8_peak": round(ops / us / 1e6 / ipk, 4),
                        "coarse_key_bytes": ab["coarse_keys"]})
         rec["phases"][pname] = ph
-        del g
-    rec["phase_timing"] = "each launch alone after a cold-L2 flush (median of %d, in-graph events)" % iso
+    rec["phase_timing"] = (f"each launch alone, back to back over the {len(cases)} batches (mean)" if rotate else
+                           "each launch alone after a cold-L2 flush (median of %d, in-graph events; includes one "
+                           "graph launch)" % iso)
     if int(err.item()) != 0:
         raise RuntimeError(f"device error bits {int(err.item())} while timing {name}")
     del cases
