@@ -223,6 +223,8 @@ class StepCase:
         self.graph_attn, self.ev_attn = self.capture(self.attn)
 
     def capture(self, fn):
+        """A graph of ``fn`` between two events it records; the graph keeps
+        the events alive (they must outlive every replay)."""
         ev = (torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=self.stream):
@@ -230,6 +232,7 @@ class StepCase:
             fn()
             ev[1].record()
         torch.cuda.synchronize(self.device)
+        g.dsa_events = ev
         return g, ev
 
     def run_step(self):

@@ -58,6 +58,18 @@ DecodeLayout decode_layout(int total_q, int hq, int hkv) {
     return L;
 }
 
+// select workspace: [counters int32 T][candidate keys u64 T*kSelMaxChunks*(kSelMaxK-1)]
+struct SelectLayout {
+    size_t counters, cand, total;
+};
+SelectLayout select_layout(int total_q) {
+    SelectLayout L;
+    L.counters = 0;
+    L.cand = align_up((size_t)total_q * sizeof(int32_t), 256);
+    L.total = align_up(L.cand + (size_t)total_q * kSelMaxChunks * (kSelMaxK - 1) * sizeof(unsigned long long), 256);
+    return L;
+}
+
 // single-launch decode workspace: [header 256 B][sel_count T][flags T]
 // [split counters T*Hkv][candidates kAttnMaxCtas*2*(kSelMaxK-1) u64][partials]
 struct FusedLayout {
@@ -267,8 +279,8 @@ int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int3
 }
 
 size_t dsa_select_blocks_workspace_size(int32_t total_q) {
-    (void)total_q;
-    return 0;   // the selection merges inside thread-block clusters
+    if (total_q <= 0) return 0;
+    return select_layout(total_q).total;
 }
 
 int dsa_select_blocks(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
@@ -327,15 +339,14 @@ int select_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_que
     int rc;
     if ((rc = check_cache(cache)) || (rc = check_seqs(seqs)) || (rc = check_queries(queries))) return rc;
     if (num_idx_heads < 1 || w_abs_max < 0 || k_max < 1) return DSA_ERR_INVALID_ARG;
-    if (num_idx_heads > kMaxIdxHeads || k_max > kSelMaxK || seqs->max_blocks > kSelMaxBlocks)
+    if (num_idx_heads > kMaxIdxHeads || k_max > kSelMaxK || seqs->max_blocks > kSelMaxChunks * 4096)
         return DSA_ERR_UNSUPPORTED;
     const long long bound = (long long)num_idx_heads * w_abs_max * kIdxDim * 128LL * 128LL;
     if (bound >= (1LL << 31)) return DSA_ERR_RANGE;
     if (queries->total_q == 0) return DSA_OK;
     if (!q_idx || !w || !k_per_seq || !sel || !cnt || !aligned16(q_idx)) return DSA_ERR_INVALID_ARG;
-    (void)workspace;   // the clusters merge on chip: no workspace is used
-    (void)workspace_bytes;
-    if ((long long)queries->total_q * kSelMaxCluster > 0x7fffffffLL) return DSA_ERR_UNSUPPORTED;
+    const SelectLayout L = select_layout(queries->total_q);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < L.total) return DSA_ERR_WORKSPACE;
     SelectArgs a{};
     a.kc_pool = cache->kc_pool;
     a.num_pages = cache->num_pages;
@@ -353,13 +364,10 @@ int select_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_que
     a.k_max = k_max;
     a.sel = sel;
     a.cnt = cnt;
+    char *ws = static_cast<char *>(workspace);
+    a.counters = reinterpret_cast<int32_t *>(ws + L.counters);
+    a.cand = reinterpret_cast<unsigned long long *>(ws + L.cand);
     a.dev_err = dev_err;
-    // the selected pages of the whole call, K and V: when they fit in L2 with
-    // room to spare, the selection starts streaming them for the attention
-    a.k_pool = cache->k_pool;
-    a.v_pool = cache->v_pool;
-    a.kv_page_bytes = kBlockSize * cache->num_kv_heads * kHeadDim * 2;
-    a.prefetch_kv = (double)queries->total_q * k_max * 2.0 * a.kv_page_bytes <= kSelPrefetchBytes ? 1 : 0;
     a.cu_new = app ? app->cu_new : nullptr;
     if (app) a.app = *app;
     return from_cuda(launch_select_blocks(a, reinterpret_cast<cudaStream_t>(stream)));

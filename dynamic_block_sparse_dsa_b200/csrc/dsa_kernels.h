@@ -74,15 +74,9 @@ struct TopkArgs {
     int32_t *dev_err;
 };
 
-// fused score + Top-K: one thread-block cluster of up to kSelMaxCluster CTAs
-// per query, each CTA covering up to 16 groups of 512 candidate blocks
-constexpr int kSelMaxCluster = 16;
-constexpr int kSelMaxBlocks = kSelMaxCluster * 16 * 512;   // 131072 blocks: an 8M-token context
-constexpr int kSelMaxChunks = 32;   // candidate lists per query of the single-launch decode step
+// fused score + Top-K (decode-oriented): candidate workspace layout
+constexpr int kSelMaxChunks = 32;   // chunks per query
 constexpr int kSelMaxK = 64;        // largest k_max of the fused path
-// largest K/V footprint of one call's selected pages that the selection
-// prefetches into L2 for the attention (the B200 L2 holds 126 MB)
-constexpr double kSelPrefetchBytes = 72.0 * 1024 * 1024;
 struct SelectArgs {
     const int8_t *kc_pool;
     int num_pages;
@@ -100,22 +94,18 @@ struct SelectArgs {
     int k_max;
     int32_t *sel;            // [T][k_max]
     int32_t *cnt;            // [T]
+    unsigned long long *cand;   // [T][kSelMaxChunks][kSelMaxK-1] 64-bit selection keys, sorted descending
+    int32_t *counters;       // [T] chunk CTAs done per query
     int32_t *dev_err;
     // append ordered after this selection (dsa_select_blocks_append): a
     // query whose sequence appends a block before its own block is refused
     // (DSA_DEV_ERR_POS, cnt 0) -- the selection must not read those keys; and
     // the kernel is launched after everything before it has completed
     const int32_t *cu_new;   // null: no append follows
-    // the append itself (app.total_new > 0): the non-leader CTAs of the
-    // selection's clusters copy the new tokens once their lists are sent
+    // the append itself (app.total_new > 0): extra CTAs of the selection grid,
+    // rows sel_rows.. of blockIdx.y, copy the new tokens while the selection runs
     KvAppendArgs app;
-    int cluster;             // set by the launcher: CTAs per query (the cluster size)
-    // 1: the leader of each query also starts moving the selected blocks' K/V
-    // pages (kv_page_bytes each, whole pages of every KV head) into L2 for
-    // the attention that follows
-    int prefetch_kv;
-    const void *k_pool, *v_pool;
-    int kv_page_bytes;
+    int sel_rows;            // set by the launcher: grid rows that select
 };
 
 struct AttnArgs {

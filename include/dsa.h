@@ -170,14 +170,12 @@ int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int3
  * intermediate written to memory, block-wise reduction + partial selection;
  * P5 "Differentiated Adaptation of Prefill and Decode": fuse selection in
  * decode].  Same arguments and the same sel / cnt results as the two calls;
- * k_max <= 64, max_blocks <= 131072 (an 8M-token context) and total_q <=
- * 2^27 in v1.  Each query's visible blocks are scored by the CTAs of one
- * thread-block cluster (up to 16), each keeping the Top-(K-1) of its share;
- * the cluster's leader merges the lists through distributed shared memory.
- * No workspace is used: dsa_select_blocks_workspace_size() returns 0 and the
- * workspace arguments are ignored (they may be NULL).
- * Device errors: DSA_DEV_ERR_PAGE, DSA_DEV_ERR_POS, DSA_DEV_ERR_K,
- * DSA_DEV_ERR_WAIT (a cluster's merge gave up waiting; that query gets cnt 0).
+ * k_max <= 64 and max_blocks <= 131072 (an 8M-token context) in v1.  Each
+ * query's visible blocks are scored in chunks by separate CTAs that keep their
+ * local Top-(K-1); the last CTA of the query merges them.  Needs a workspace
+ * of dsa_select_blocks_workspace_size(total_q) bytes, zero-filled before its
+ * first use (each call leaves its counters at zero again).
+ * Device errors: DSA_DEV_ERR_PAGE, DSA_DEV_ERR_POS, DSA_DEV_ERR_K.
  */
 size_t dsa_select_blocks_workspace_size(int32_t total_q);
 

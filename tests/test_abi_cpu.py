@@ -133,10 +133,12 @@ def test_select_validation_codes():
     assert sel(k_max=65) == _lib.DSA_ERR_UNSUPPORTED        # the fused path keeps at most 64
     assert sel(heads=17) == _lib.DSA_ERR_UNSUPPORTED
     assert sel(wmax=128) == _lib.DSA_ERR_RANGE
+    assert sel(ws=None) == _lib.DSA_ERR_WORKSPACE
+    assert sel(ws_bytes=16) == _lib.DSA_ERR_WORKSPACE
+    assert sel(ws=FAKE + 8) == _lib.DSA_ERR_WORKSPACE        # misaligned workspace
     assert sel(queries=_queries(total_q=0), ws=None, ws_bytes=0) == _lib.DSA_OK
-    # the selection merges inside thread-block clusters: no workspace at all
     assert lib.dsa_select_blocks_workspace_size(0) == 0
-    assert lib.dsa_select_blocks_workspace_size(8) == 0
+    assert lib.dsa_select_blocks_workspace_size(8) > 0
 
 
 def test_select_append_validation_codes():
