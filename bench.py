@@ -264,7 +264,7 @@ class StepCase:
     def topk(self):
         wl, b = self.wl, self.bufs
         self.dsa.topk_blocks(self.seqs, self.queries, b["scores"], wl.k_per_seq, self.spec.k_max, sel=b["sel"],
-                             cnt=b["cnt"], dev_err=self.err)
+                             cnt=b["cnt"], dev_err=self.err, block_size=self.spec.block_size)
 
     def front(self):
         if self.fused and self.decode:
@@ -666,7 +666,7 @@ def measure_workload(name, device, steps=30, iso=15, seed=None):
     stream = torch.cuda.Stream(device)
     tm = Timer(device, stream)
     seed = {"tiny_decode": 1001, "batched_gqa_decode": 1002, "chunked_prefill": 1004,
-            "mixed_ragged": 1005}.get(name, 1000) if seed is None else seed
+            "mixed_ragged": 1005}.get(name, 1003) if seed is None else seed
     cases = [StepCase(spec, seed, device, stream, err, path)]
     ab = algorithmic_bytes(cases[0].wl)
     need = max(2, math.ceil(ROTATE_L2_MULTIPLE * L2_BYTES / ab["total"]))
@@ -686,7 +686,8 @@ def measure_workload(name, device, steps=30, iso=15, seed=None):
         step_s = statistics.median(tm.isolated(c0.graph, c0.ev, steps)) / 1e3
         how = "one step at a time after a cold-L2 flush (median; includes one graph launch)"
     peak, peak_kind = _peaks()
-    rec = {"path": path, "queries": spec.total_q, "step_us": round(step_s * 1e6, 2),
+    rec = {"path": path, "queries": spec.total_q, "block_size": spec.block_size, "top_k": spec.k_max,
+           "step_us": round(step_s * 1e6, 2),
            "tokens_per_s": round(spec.total_q / step_s, 1), "step_timing": how, "phases": {}}
     kv_gb, flops = ab["kv"], ab["flops"]
     if decode:
@@ -932,7 +933,8 @@ def main(argv=None):
     if world == 1 and not args.no_configs:
         # the other workloads, one GPU: step time and each launch against its roofline
         res["configs"] = {n: measure_workload(n, device) for n in
-                          ("tiny_decode", "batched_gqa_decode", "chunked_prefill", "mixed_ragged")
+                          ("tiny_decode", "batched_gqa_decode", "chunked_prefill", "mixed_ragged",
+                           "decode_1m_b128", "decode_1m_b256", "decode_1m_b512")
                           if n != args.workload}
     if rank == 0:
         print(json.dumps(res), flush=True)

@@ -72,7 +72,8 @@ def _expect(t: torch.Tensor, dtype, name):
 
 @dataclass
 class PagedKVCache:
-    """Block-paged pools: k/v bf16 [num_pages][64][num_kv_heads][128], kc int8 [num_pages][64]."""
+    """Block-paged pools: k/v bf16 [num_pages][block_size][num_kv_heads][128], kc int8
+    [num_pages][64]; block_size (64, 128, 256 or 512 tokens) is the pools' second dimension."""
     k_pool: torch.Tensor
     v_pool: torch.Tensor
     kc_pool: torch.Tensor
@@ -88,6 +89,10 @@ class PagedKVCache:
     @property
     def num_kv_heads(self) -> int:
         return self.k_pool.shape[2]
+
+    @property
+    def block_size(self) -> int:
+        return self.k_pool.shape[1]
 
 
 @dataclass
@@ -148,8 +153,9 @@ def index_score(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, q_idx:
 
 def topk_blocks(seqs: SeqBatch, queries: QueryBatch, scores: torch.Tensor, k_per_seq: torch.Tensor,
                 k_max: int, sel: Optional[torch.Tensor] = None, cnt: Optional[torch.Tensor] = None,
-                dev_err: Optional[torch.Tensor] = None, stream=None):
-    """(sel int32 [total_q][k_max] ascending logical ids, -1 padded; cnt int32 [total_q])."""
+                dev_err: Optional[torch.Tensor] = None, stream=None, block_size: int = BLOCK_SIZE):
+    """(sel int32 [total_q][k_max] ascending logical ids, -1 padded; cnt int32 [total_q]).
+    ``block_size`` is the tokens per block of the cache the scores came from."""
     lib = load()
     dev = scores.device
     if sel is None:
@@ -158,7 +164,7 @@ def topk_blocks(seqs: SeqBatch, queries: QueryBatch, scores: torch.Tensor, k_per
         cnt = torch.empty((queries.total_q,), dtype=torch.int32, device=dev)
     s, q = seqs.ctype(), queries.ctype()
     _lib.check("dsa_topk_blocks", lib.dsa_topk_blocks(
-        ctypes.byref(s), ctypes.byref(q), _ptr(scores), _ptr(k_per_seq), int(k_max), _ptr(sel),
+        ctypes.byref(s), ctypes.byref(q), _ptr(scores), _ptr(k_per_seq), int(k_max), int(block_size), _ptr(sel),
         _ptr(cnt), _ptr(dev_err), _stream(stream)))
     return sel, cnt
 
@@ -381,7 +387,7 @@ def step(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, *, k_new, v_n
         index_score(cache, seqs, queries, q_idx, w, w_abs_max, scores=b["scores"], dev_err=dev_err,
                     stream=stream)
         topk_blocks(seqs, queries, b["scores"], k_per_seq, k_max, sel=b["sel"], cnt=b["cnt"], dev_err=dev_err,
-                    stream=stream)
+                    stream=stream, block_size=cache.block_size)
     if decode:
         sparse_attn_decode(cache, seqs, queries, q, b["sel"], b["cnt"], out=b["out"], lse=b["lse"],
                            workspace=b["workspace"], dev_err=dev_err, stream=stream)

@@ -42,7 +42,7 @@ SIGNATURES = {
     "dsa_kv_append": ([P(KvCacheC), P(SeqsC), c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp], c_i32),
     "dsa_index_score": ([P(KvCacheC), P(SeqsC), P(QueriesC), c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp],
                         c_i32),
-    "dsa_topk_blocks": ([P(SeqsC), P(QueriesC), c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp], c_i32),
+    "dsa_topk_blocks": ([P(SeqsC), P(QueriesC), c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp], c_i32),
     "dsa_select_blocks_workspace_size": ([c_i32], ctypes.c_size_t),
     "dsa_select_blocks": ([P(KvCacheC), P(SeqsC), P(QueriesC), c_vp, c_vp, c_i32, c_i32, c_vp, c_i32, c_vp, c_vp,
                            c_vp, ctypes.c_size_t, c_vp, c_vp], c_i32),

@@ -11,11 +11,18 @@ using namespace dsa;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// log2 of a supported block size (64, 128, 256, 512 tokens), or -1
+int block_shift_of(int block_size) {
+    for (int sh = kMinBlockShift; sh <= kMaxBlockShift; ++sh)
+        if (block_size == (1 << sh)) return sh;
+    return -1;
+}
+
 int check_cache(const dsa_kv_cache *c) {
     if (!c || !c->k_pool || !c->v_pool || !c->kc_pool) return DSA_ERR_INVALID_ARG;
     if (!aligned16(c->k_pool) || !aligned16(c->v_pool) || !aligned16(c->kc_pool)) return DSA_ERR_INVALID_ARG;
     if (c->num_pages < 1 || c->num_kv_heads < 1) return DSA_ERR_INVALID_ARG;
-    if (c->block_size != kBlockSize || c->head_dim != kHeadDim || c->idx_dim != kIdxDim)
+    if (block_shift_of(c->block_size) < 0 || c->head_dim != kHeadDim || c->idx_dim != kIdxDim)
         return DSA_ERR_UNSUPPORTED;
     return DSA_OK;
 }
@@ -91,13 +98,13 @@ FusedLayout fused_layout(int total_q, int hq, int hkv) {
 // than work items so that every CTA owns a non-empty range
 void attn_schedule(AttnArgs &a, bool allow_split, bool allow_cluster = false) {
     const long long pairs = (long long)a.total_q * a.num_kv_heads;
-    a.total_units = pairs * a.k_max;
+    a.total_units = (pairs * a.k_max) << a.tile_shift;
     long long C = sm_count();
     if (C > kAttnMaxCtas) C = kAttnMaxCtas;
     a.cluster2 = 0;
     // between a quarter and a half as many pairs as SMs: one 2-CTA cluster per
     // pair keeps at least half of the SMs streaming and merges on chip
-    if (allow_cluster && allow_split && a.k_max >= 2 && 4 * pairs >= C && 2 * pairs <= C) {
+    if (allow_cluster && allow_split && (a.k_max << a.tile_shift) >= 2 && 4 * pairs >= C && 2 * pairs <= C) {
         a.cluster2 = 1;
         a.pair_aligned = 0;
         a.num_ctas = (int)(2 * pairs);
@@ -127,11 +134,14 @@ int attn_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queri
     if (!(sm_scale > 0.f)) return DSA_ERR_INVALID_ARG;
     // TMA coordinates are int32: pool rows (page*64+token) and query rows (t*Hq+h);
     // work units (query, KV head, selection slot) are counted in 32 bits
-    if ((long long)cache->num_pages * kBlockSize >= (1LL << 31) ||
+    const int bsh = block_shift_of(cache->block_size);
+    if (((long long)cache->num_pages << bsh) >= (1LL << 31) ||
         (long long)queries->total_q * num_q_heads >= (1LL << 31) ||
-        (long long)queries->total_q * cache->num_kv_heads * k_max >= (1LL << 31))
+        (((long long)queries->total_q * cache->num_kv_heads * k_max) << (bsh - 6)) >= (1LL << 31))
         return DSA_ERR_UNSUPPORTED;
     a = AttnArgs{};
+    a.block_shift = bsh;
+    a.tile_shift = bsh - 6;
     a.k_pool = static_cast<const __nv_bfloat16 *>(cache->k_pool);
     a.v_pool = static_cast<const __nv_bfloat16 *>(cache->v_pool);
     a.num_pages = cache->num_pages;
@@ -198,6 +208,7 @@ int dsa_kv_append(const dsa_kv_cache *cache, const dsa_seqs *seqs, const int32_t
     if (!cu_new || !k_new || !v_new) return DSA_ERR_INVALID_ARG;
     if (!aligned16(k_new) || !aligned16(v_new) || (kc_new && !aligned16(kc_new))) return DSA_ERR_INVALID_ARG;
     KvAppendArgs a{};
+    a.block_shift = block_shift_of(cache->block_size);
     a.k_pool = cache->k_pool;
     a.v_pool = cache->v_pool;
     a.kc_pool = cache->kc_pool;
@@ -229,6 +240,7 @@ int dsa_index_score(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_q
     if (queries->total_q == 0) return DSA_OK;
     if (!q_idx || !w || !scores || !aligned16(q_idx)) return DSA_ERR_INVALID_ARG;
     IndexScoreArgs a{};
+    a.block_shift = block_shift_of(cache->block_size);
     a.kc_pool = cache->kc_pool;
     a.num_pages = cache->num_pages;
     a.block_table = seqs->block_table;
@@ -254,15 +266,17 @@ int dsa_index_score(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_q
 }
 
 int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int32_t *scores,
-                    const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt,
+                    const int32_t *k_per_seq, int32_t k_max, int32_t block_size, int32_t *sel, int32_t *cnt,
                     int32_t *dev_err, dsa_stream_t stream) {
     int rc;
     if ((rc = check_seqs(seqs)) || (rc = check_queries(queries))) return rc;
     if (k_max < 1) return DSA_ERR_INVALID_ARG;
+    if (block_shift_of(block_size) < 0) return DSA_ERR_UNSUPPORTED;
     if (k_max > kSelMaxK || seqs->max_blocks > topk_max_blocks()) return DSA_ERR_UNSUPPORTED;
     if (queries->total_q == 0) return DSA_OK;
     if (!scores || !k_per_seq || !sel || !cnt) return DSA_ERR_INVALID_ARG;
     TopkArgs a{};
+    a.block_shift = block_shift_of(block_size);
     a.seq_lens = seqs->seq_lens;
     a.num_seqs = seqs->num_seqs;
     a.max_blocks = seqs->max_blocks;
@@ -305,6 +319,7 @@ int dsa_select_blocks_append(const dsa_kv_cache *cache, const dsa_seqs *seqs, co
         if (!aligned16(k_new) || !aligned16(v_new) || (kc_new && !aligned16(kc_new))) return DSA_ERR_INVALID_ARG;
     }
     KvAppendArgs a{};
+    a.block_shift = block_shift_of(cache->block_size);
     a.k_pool = cache->k_pool;
     a.v_pool = cache->v_pool;
     a.kc_pool = cache->kc_pool;
@@ -348,6 +363,7 @@ int select_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_que
     const SelectLayout L = select_layout(queries->total_q);
     if (!workspace || !aligned16(workspace) || workspace_bytes < L.total) return DSA_ERR_WORKSPACE;
     SelectArgs a{};
+    a.block_shift = block_shift_of(cache->block_size);
     a.kc_pool = cache->kc_pool;
     a.num_pages = cache->num_pages;
     a.block_table = seqs->block_table;
@@ -417,7 +433,8 @@ int dsa_decode_fused(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_
     int rc = attn_common(cache, seqs, queries, q, num_q_heads, sel, cnt, k_max, sm_scale, out, lse, dev_err, a);
     if (rc) return rc;
     if (num_idx_heads < 1 || w_abs_max < 0 || total_new < 0) return DSA_ERR_INVALID_ARG;
-    if (num_idx_heads > kMaxIdxHeads || k_max > kSelMaxK || queries->total_q > kFusedMaxQ)
+    if (num_idx_heads > kMaxIdxHeads || k_max > kSelMaxK || queries->total_q > kFusedMaxQ ||
+        cache->block_size != kBlockSize)   // the single-launch step keeps 64-token blocks
         return DSA_ERR_UNSUPPORTED;
     const long long bound = (long long)num_idx_heads * w_abs_max * kIdxDim * 128LL * 128LL;
     if (bound >= (1LL << 31)) return DSA_ERR_RANGE;

@@ -9,7 +9,8 @@
 
 namespace dsa {
 
-constexpr int kBlockSize = 64;   // tokens per KV block (= one page)
+constexpr int kBlockSize = 64;   // tokens per attention tile (a KV block is 1, 2, 4 or 8 of them)
+constexpr int kMinBlockShift = 6, kMaxBlockShift = 9;   // KV blocks (= pages) of 64 .. 512 tokens
 constexpr int kHeadDim = 128;    // attention head dim
 constexpr int kIdxDim = 64;      // indexer dim (bytes of one coarse key)
 constexpr int kMaxGroup = 16;    // query heads per KV head handled by one CTA

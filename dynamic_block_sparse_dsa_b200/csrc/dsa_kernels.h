@@ -25,6 +25,7 @@ struct KvAppendArgs {
     void *k_pool, *v_pool;
     int8_t *kc_pool;
     int num_pages, num_kv_heads;
+    int block_shift;         // tokens per KV block = 1 << block_shift (6..9)
     const int32_t *block_table;
     int max_blocks;
     const int32_t *seq_lens;
@@ -45,6 +46,7 @@ struct KvAppendArgs {
 struct IndexScoreArgs {
     const int8_t *kc_pool;
     int num_pages;
+    int block_shift;
     const int32_t *block_table;
     int max_blocks;
     const int32_t *seq_lens;
@@ -60,6 +62,7 @@ struct IndexScoreArgs {
 };
 
 struct TopkArgs {
+    int block_shift;
     const int32_t *seq_lens;
     int num_seqs;
     int max_blocks;
@@ -80,6 +83,7 @@ constexpr int kSelMaxK = 64;        // largest k_max of the fused path
 struct SelectArgs {
     const int8_t *kc_pool;
     int num_pages;
+    int block_shift;
     const int32_t *block_table;
     int max_blocks;
     const int32_t *seq_lens;
@@ -111,6 +115,9 @@ struct SelectArgs {
 struct AttnArgs {
     const __nv_bfloat16 *k_pool, *v_pool;
     int num_pages, num_kv_heads;
+    // tokens per KV block = 1 << block_shift; the kernel works in 64-token
+    // tiles, tile_shift = block_shift - 6 of them per block
+    int block_shift, tile_shift;
     const int32_t *block_table;
     int max_blocks;
     const int32_t *seq_lens;
@@ -127,9 +134,10 @@ struct AttnArgs {
     float scale_log2;        // sm_scale * log2(e)
     __nv_bfloat16 *out;      // [T][Hq][128]
     float *lse;              // [T][Hq] or null
-    // persistent schedule: work unit u = (query t, KV head, selection slot j),
-    // u = (t * Hkv + kvh) * k_max + j; CTA c owns [c*U/C, (c+1)*U/C), rounded to
-    // whole (t, kvh) pairs when pair_aligned
+    // persistent schedule: work unit u = (query t, KV head, selection slot j,
+    // 64-token tile i of that block), u = ((t * Hkv + kvh) * k_max + j) * m + i
+    // with m = 1 << tile_shift; CTA c owns [c*U/C, (c+1)*U/C), rounded to whole
+    // (t, kvh) pairs when pair_aligned
     long long total_units;   // U
     int num_ctas;            // C (= gridDim.x)
     int pair_aligned;

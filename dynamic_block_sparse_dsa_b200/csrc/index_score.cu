@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_dp4a_kernel(IndexSc
     const int H = a.num_idx_heads;
 
     // the coarse key of this thread's block (if it can be visible to anyone)
-    const int n_blocks = (len + kBlockSize - 1) / kBlockSize;
+    const int n_blocks = (len + (1 << a.block_shift) - 1) >> a.block_shift;
     bool have = false;
     int kc[16];
     if (blockIdx.x * kScoreThreads >= n_blocks) return;   // the whole chunk is past the end
@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_dp4a_kernel(IndexSc
             s_w[e / H][e % H] = __ldg(a.w + (size_t)(qb + e / H) * H + e % H);
         if (threadIdx.x < nq) {
             const int p = __ldg(a.q_pos + qb + threadIdx.x);
-            int own = p / kBlockSize;
+            int own = p >> a.block_shift;
             if (p < 0 || p >= len || own >= a.max_blocks) {
                 if (blockIdx.x == 0) set_err(a.dev_err, DSA_DEV_ERR_POS);
                 own = -1;

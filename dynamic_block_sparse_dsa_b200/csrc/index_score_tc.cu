@@ -281,7 +281,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         auto take = [&](int pos, int t) {
                             int own = -1;
                             if (t < tn) {
-                                own = pos / kBlockSize;
+                                own = pos >> a.block_shift;
                                 if (pos < 0 || pos >= d_len || own >= a.max_blocks) {
                                     bad = true;
                                     own = -1;
@@ -327,7 +327,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         const bool member = lane < kQT && t < a.total_q && cu(s) <= t && t < cu(s + 1);
                         int own = -1;
                         if (member) {
-                            own = pos / kBlockSize;
+                            own = pos >> a.block_shift;
                             if (pos < 0 || pos >= len || own >= a.max_blocks) {
                                 err_bits |= DSA_DEV_ERR_POS;
                                 own = -1;
@@ -349,7 +349,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         }
                         if (ab) ++agen1; else ++agen0;
                         const int len = single ? __shfl_sync(0xffffffffu, d_len, i) : seq_len(s);
-                        const int n_blocks = (len + kBlockSize - 1) / kBlockSize;
+                        const int n_blocks = (len + (1 << a.block_shift) - 1) >> a.block_shift;
                         const int32_t *row = a.block_table + (size_t)s * a.max_blocks;
                         int page[kBT / 32];
 #pragma unroll

@@ -5,8 +5,8 @@
 // blocks in batch, decode appends one token and maintains the block table,
 // and both share one block-index semantics.  One CTA per new token copies its
 // K and V rows (num_kv_heads * 256 bytes each) with 16-byte vector stores into
-// the page slot block_table[s][pos / 64], token pos % 64; the last new token
-// of each touched block also writes that block's coarse key.
+// the page slot block_table[s][pos / B], token pos % B (B the block size);
+// the last new token of each touched block also writes that block's coarse key.
 #include "dsa_kernels.h"
 #include "kv_append.cuh"
 

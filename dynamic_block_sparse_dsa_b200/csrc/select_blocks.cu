@@ -98,14 +98,14 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
         s = find_seq(a.cu_q, a.num_seqs, t);
     }
     if (!guess || s != t) load_seq_facts(s);
-    const int n_vis = p / kBlockSize + 1;
+    const int n_vis = (p >> a.block_shift) + 1;
     const int32_t *table = a.block_table + (size_t)s * a.max_blocks;
     int32_t *out = a.sel + (size_t)t * a.k_max;
     bool bad_pos = p < 0 || p >= len || n_vis > a.max_blocks;
     if (a.cu_new && !bad_pos) {
         // an append follows and overlaps this kernel: no candidate block may be appended to
         const int n_new = __ldg(a.cu_new + s + 1) - __ldg(a.cu_new + s);
-        if (n_new > len || (n_new > 0 && n_vis - 1 > (len - n_new) / kBlockSize)) bad_pos = true;
+        if (n_new > len || (n_new > 0 && n_vis - 1 > ((len - n_new) >> a.block_shift))) bad_pos = true;
     }
     const bool bad_k = K < 1 || K > a.k_max;
     if (bad_pos || bad_k) {

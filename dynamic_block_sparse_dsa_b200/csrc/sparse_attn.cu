@@ -113,8 +113,9 @@ using unit_t = uint32_t;
 // first unit of CTA c (64-bit products; computed once per CTA)
 __device__ __forceinline__ unit_t range_begin(const AttnArgs &a, int c) {
     if (a.pair_aligned) {
-        const unsigned long long pairs = (unsigned long long)a.total_units / (unsigned)a.k_max;
-        return (unit_t)((unsigned long long)c * pairs / (unsigned)a.num_ctas * (unsigned)a.k_max);
+        const unsigned up = (unsigned)a.k_max << a.tile_shift;   // units per pair
+        const unsigned long long pairs = (unsigned long long)a.total_units / up;
+        return (unit_t)((unsigned long long)c * pairs / (unsigned)a.num_ctas * up);
     }
     return (unit_t)((unsigned long long)c * (unsigned long long)a.total_units / (unsigned)a.num_ctas);
 }
@@ -156,17 +157,18 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     unit_t *s_rb = reinterpret_cast<unit_t *>(gbase + P::kOffRb);
     for (int i = tid; i <= a.num_ctas; i += kAttnThreads) s_rb[i] = range_begin(a, i);
     unit_t u0, u1;
+    // units per (query, KV head) pair: every selection slot's 64-token tiles
+    const unit_t K = (unit_t)a.k_max << a.tile_shift;
     if (a.cluster2) {   // half of pair c/2: units [0, h0) for rank 0, [h0, K) for rank 1
-        const unit_t p0 = (unit_t)(c >> 1) * (unit_t)a.k_max;
-        const int h0 = (a.k_max + 1) / 2;
+        const unit_t p0 = (unit_t)(c >> 1) * K;
+        const unit_t h0 = (K + 1) / 2;
         u0 = p0 + ((c & 1) ? h0 : 0);
-        u1 = p0 + ((c & 1) ? a.k_max : h0);
+        u1 = p0 + ((c & 1) ? K : h0);
     } else {
         u0 = range_begin(a, c);
         u1 = range_begin(a, c + 1);
     }
     const int G = a.group;
-    const unit_t K = (unit_t)a.k_max;
     const unit_t Hkv = (unit_t)a.num_kv_heads;
 
     if (tid == 0) {
@@ -244,10 +246,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         for (unit_t base = u0; base < u1 && !stop; base += 32) {
             const unit_t uu = base + lane;
             const bool in = uu < u1;
+            // per unit: its pair's facts, the 64-token tile index within the
+            // sequence (blk) and the tile's first pool row (page); n_vis counts
+            // the query's visible 64-token tiles
             int t = 0, kvh = 0, s = 0, p = 0, n_vis = 0, blk = -1, page = -1;
             if (in) {
                 const unit_t pair = uu / K;
-                const int j = (int)(uu - pair * K);
+                const int ju = (int)(uu - pair * K);
+                const int j = ju >> a.tile_shift, sub = ju & ((1 << a.tile_shift) - 1);
                 t = (int)(pair / Hkv);
                 kvh = (int)(pair - (unit_t)t * Hkv);
                 s = seq_of(a, s_cuq, t);
@@ -257,15 +263,18 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 // the selection may have been written during this launch: read it through L2
                 int n_sel = sel_ready ? __ldcg(a.cnt + t) : 0;
                 const int b = sel_ready ? __ldcg(a.sel + (size_t)t * a.k_max + j) : -1;
-                n_vis = p / kBlockSize + 1;
-                if (p < 0 || p >= len || n_vis > a.max_blocks || n_sel < 0 || n_sel > a.k_max) n_sel = 0;
+                const int n_vis_blocks = (p >> a.block_shift) + 1;
+                n_vis = (p >> 6) + 1;
+                if (p < 0 || p >= len || n_vis_blocks > a.max_blocks || n_sel < 0 || n_sel > a.k_max) n_sel = 0;
                 if (j < n_sel) {
-                    if (b < 0 || b >= n_vis) {
+                    if (b < 0 || b >= n_vis_blocks) {
                         err_bits |= DSA_DEV_ERR_SEL;
                     } else {
                         const int pg = __ldg(a.block_table + (size_t)s * a.max_blocks + b);
+                        const int tile = (b << a.tile_shift) + sub;
                         if (pg < 0 || pg >= a.num_pages) err_bits |= DSA_DEV_ERR_PAGE;
-                        else { blk = b; page = pg; }
+                        else if (tile < n_vis) { blk = tile; page = (pg << a.block_shift) + (sub << 6); }
+                        // tiles past the query's position (own block only) hold no visible token
                     }
                 }
             }
@@ -321,7 +330,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                             W[kWFill + st] = item;
                             const uint32_t dst = sm.stage(st);
                             mbar_arrive_expect_tx(sm.full(st), kStageBytes);
-                            const int z = ipg * kBlockSize;
+                            const int z = ipg;   // the tile's first row in the pool
                             tma_load_3d(dst, &tm_k, 0, pkvh, z, sm.full(st));
                             tma_load_3d(dst + kHalf, &tm_k, 64, pkvh, z, sm.full(st));
                             tma_load_3d(dst + 2 * kHalf, &tm_v, 0, pkvh, z, sm.full(st));
@@ -686,7 +695,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             if (tid == 0) {
                 const int covered = (int)(seg_end - seg_begin);
                 const int old = atomic_add_acq_rel_gpu(a.counters + pair, covered);
-                W[kWLast] = (old + covered == a.k_max);
+                W[kWLast] = (old + covered == (int)K);
             }
             __syncwarp();
             named_barrier(1, kConsumerWarps * 32);
@@ -816,9 +825,9 @@ struct AttnMaps {
 cudaError_t make_maps(const AttnArgs &a, AttnMaps &m) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    // K / V pool: dims (head_dim, kv_head, page*64+token), boxes of 64 dims x 1 head x 64 tokens
+    // K / V pool: dims (head_dim, kv_head, page*B+token), boxes of 64 dims x 1 head x 64 tokens (one tile)
     const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)a.num_kv_heads,
-                                (cuuint64_t)a.num_pages * kBlockSize};
+                                (cuuint64_t)a.num_pages << a.block_shift};
     const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)a.num_kv_heads * kHeadDim * 2};
     const cuuint32_t box[3] = {64, 1, kBlockSize};
     const cuuint32_t estr[3] = {1, 1, 1};

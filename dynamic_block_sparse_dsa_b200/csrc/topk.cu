@@ -32,7 +32,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     const int p = __ldg(a.q_pos + t);
     const int len = __ldg(a.seq_lens + s);
     const int K = __ldg(a.k_per_seq + s);
-    const int n_vis = p / kBlockSize + 1;
+    const int n_vis = (p >> a.block_shift) + 1;
     const bool bad_pos = p < 0 || p >= len || n_vis > a.max_blocks;
     const bool bad_k = K < 1 || K > a.k_max;
     if (bad_pos || bad_k) {

@@ -111,6 +111,14 @@ def decode_1m(batch: int = 8) -> WorkloadSpec:
                         k_per_seq=(32,) * batch, k_max=32, plant=32)
 
 
+def decode_1m_blocks(block_size: int, batch: int = 8) -> WorkloadSpec:
+    """decode_1m with blocks of ``block_size`` tokens and the same selected-token
+    budget (Top-K = 2048 / block_size blocks, that many planted blocks)."""
+    k = 2048 // block_size
+    return WorkloadSpec(f"decode_1m_b{block_size}", seq_lens=(1 << 20,) * batch, n_new=(1,) * batch,
+                        k_per_seq=(k,) * batch, k_max=k, plant=k, block_size=block_size)
+
+
 def decode_128k(batch: int = 8) -> WorkloadSpec:
     """decode_1m's shape at a 131,072-token context (2,048 blocks): the same
     Top-K 32 attention work with a 4 GiB pool, small enough for profiling."""
@@ -148,6 +156,9 @@ NAMED = {
     "batched_gqa_decode": batched_gqa_decode,
     "decode_1m": decode_1m,
     "decode_128k": decode_128k,
+    "decode_1m_b128": lambda: decode_1m_blocks(128),
+    "decode_1m_b256": lambda: decode_1m_blocks(256),
+    "decode_1m_b512": lambda: decode_1m_blocks(512),
     "chunked_prefill": chunked_prefill,
     "mixed_ragged": mixed_ragged,
 }

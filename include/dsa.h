@@ -30,8 +30,10 @@
  *    selection outside the visible range) ORs a DSA_DEV_ERR_* bit into
  *    *dev_err (an int32 in device memory, may be NULL to ignore) and the
  *    offending item is skipped; the caller reads the word back when it likes.
- *  - Sizes in v1: block_size 64, head_dim 128, idx_dim 64; query heads per KV
- *    head 1..16; indexer heads 1..16.  Anything else is DSA_ERR_UNSUPPORTED.
+ *  - Sizes in v1: block_size 64, 128, 256 or 512 tokens (one KV block is one
+ *    page of the pools; dsa_decode_fused keeps 64), head_dim 128, idx_dim 64;
+ *    query heads per KV head 1..16; indexer heads 1..16.  Anything else is
+ *    DSA_ERR_UNSUPPORTED.
  *  - Consecutive calls on one stream overlap: each kernel lets the next one
  *    start early (programmatic dependent launch) and waits for its
  *    predecessor before it reads anything a library call writes (the pools,
@@ -86,7 +88,7 @@ typedef struct {
     void *v_pool;          /* bf16, same shape */
     int8_t *kc_pool;       /* int8 [num_pages][idx_dim] */
     int32_t num_pages;
-    int32_t block_size;    /* 64 */
+    int32_t block_size;    /* tokens per block (= page): 64, 128, 256 or 512 */
     int32_t num_kv_heads;
     int32_t head_dim;      /* 128 */
     int32_t idx_dim;       /* 64 */
@@ -157,12 +159,13 @@ int dsa_index_score(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_q
  *   k_per_seq int32 [num_seqs], each in [1, k_max]
  *   sel      int32 [total_q][k_max]: LOGICAL block ids ascending, then -1
  *   cnt      int32 [total_q]: number of ids written
+ *   block_size: tokens per block, as in the cache the scores were taken from
  * k_max <= 64 in v1.
  * Device errors: DSA_DEV_ERR_K (that query gets cnt 0), DSA_DEV_ERR_POS.
  */
 int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int32_t *scores,
-                    const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt,
-                    int32_t *dev_err, dsa_stream_t stream);
+                    const int32_t *k_per_seq, int32_t k_max, int32_t block_size, int32_t *sel,
+                    int32_t *cnt, int32_t *dev_err, dsa_stream_t stream);
 
 /*
  * dsa_select_blocks -- dsa_index_score and dsa_topk_blocks in one pass, with

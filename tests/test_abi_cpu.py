@@ -74,6 +74,8 @@ def _score(cache, seqs, queries, heads=16, wmax=16, qidx=FAKE):
 def test_host_validation_codes():
     c, s, q = _cache(), _seqs(), _queries()
     assert _score(_cache(block_size=32), s, q) == _lib.DSA_ERR_UNSUPPORTED
+    assert _score(_cache(block_size=96), s, q) == _lib.DSA_ERR_UNSUPPORTED
+    assert _score(_cache(block_size=1024), s, q) == _lib.DSA_ERR_UNSUPPORTED
     assert _score(_cache(head_dim=64), s, q) == _lib.DSA_ERR_UNSUPPORTED
     assert _score(_cache(k_pool=FAKE + 8), s, q) == _lib.DSA_ERR_INVALID_ARG      # misaligned
     assert _score(_cache(num_pages=0), s, q) == _lib.DSA_ERR_INVALID_ARG
@@ -109,9 +111,12 @@ def test_attention_validation_codes():
 def test_topk_and_append_validation_codes():
     lib = _lib.load()
     s, q = _seqs(), _queries()
-    assert lib.dsa_topk_blocks(ctypes.byref(s), ctypes.byref(q), FAKE, FAKE, 0, FAKE, FAKE, None,
+    assert lib.dsa_topk_blocks(ctypes.byref(s), ctypes.byref(q), FAKE, FAKE, 0, 64, FAKE, FAKE, None,
                                None) == _lib.DSA_ERR_INVALID_ARG
-    assert lib.dsa_topk_blocks(ctypes.byref(s), ctypes.byref(_queries(total_q=0)), FAKE, FAKE, 8, FAKE, FAKE,
+    for bad in (32, 96, 1024):
+        assert lib.dsa_topk_blocks(ctypes.byref(s), ctypes.byref(q), FAKE, FAKE, 8, bad, FAKE, FAKE, None,
+                                   None) == _lib.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_topk_blocks(ctypes.byref(s), ctypes.byref(_queries(total_q=0)), FAKE, FAKE, 8, 64, FAKE, FAKE,
                                None, None) == _lib.DSA_OK
     c = _cache()
     assert lib.dsa_kv_append(ctypes.byref(c), ctypes.byref(s), FAKE, -1, FAKE, FAKE, None, None,

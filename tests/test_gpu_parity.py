@@ -210,6 +210,63 @@ def test_mixed_ragged_workload_sampled(profile, decode, fused, cuda_device):
     compare(wl, ref, bufs, fused=fused)
 
 
+# ----------------------------------------------------------------------------- blocks of 128 / 256 / 512 tokens
+BLOCK_SIZES = [128, 256, 512]
+BLOCK_CASES = {
+    # decode queries, some contexts shorter than K blocks, one inside its first block
+    "decode_mix": dict(seq_lens=(5000, 700, 20000, 129, 64 * 40 + 5, 3), n_new=(1,) * 6,
+                       k_per_seq=(4, 2, 6, 3, 5, 2), k_max=6),
+    # prefill chunks (>= 16 queries per sequence: the tensor-core indexer), ragged tails
+    "prefill_chunks": dict(seq_lens=(9000, 3000, 1100), n_new=(70, 33, 17), k_per_seq=(5, 3, 4), k_max=5,
+                           occupancy=0.8),
+    # 48 (query, KV head) pairs: 2-CTA clusters in the decode entry
+    "cluster_pairs": dict(seq_lens=tuple(range(700, 700 + 24 * 913, 913)), n_new=(1,) * 24,
+                          k_per_seq=(3,) * 24, k_max=3),
+}
+
+
+@pytest.mark.parametrize("fused", [False, True], ids=["score_topk", "fused_select"])
+@pytest.mark.parametrize("decode", [True, False], ids=["decode_entry", "prefill_entry"])
+@pytest.mark.parametrize("block_size", BLOCK_SIZES)
+@pytest.mark.parametrize("name", sorted(BLOCK_CASES))
+def test_block_sizes_all_outputs(name, block_size, decode, fused, cuda_device):
+    kw = dict(num_q_heads=16, num_kv_heads=2, num_idx_heads=16, block_size=block_size)
+    kw.update(BLOCK_CASES[name])
+    spec = wk.sharp(wk.WorkloadSpec(f"{name}_b{block_size}", **kw))
+    wl, ref, bufs = _run(spec, 300 + block_size + len(name), cuda_device, decode=decode, fused=fused)
+    compare(wl, ref, bufs, fused=fused)
+
+
+@pytest.mark.parametrize("block_size", BLOCK_SIZES)
+def test_block_sizes_select_append(block_size, cuda_device):
+    """The decode chain of the bench (selection with the append in its grid,
+    then decode attention) with larger blocks: appended rows land in the
+    right slots of the big pages and the results equal the oracle's."""
+    kw = dict(num_q_heads=16, num_kv_heads=2, num_idx_heads=16, block_size=block_size)
+    kw.update(BLOCK_CASES["decode_mix"])
+    wl = wk.make_workload(wk.sharp(wk.WorkloadSpec("sa_b%d" % block_size, **kw)), seed=17, device=cuda_device)
+    ref = oracle_step(wl)
+    bufs, err = gpu_step(wl, overlap=True)
+    assert err == 0
+    compare(wl, ref, bufs, fused=True)
+    _appended_rows_match(wl, wl.spec.num_seqs)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("block_size", BLOCK_SIZES)
+def test_decode_1m_block_sizes(block_size, cuda_device):
+    wl, ref, bufs = _run(wk.sharp(wk.decode_1m_blocks(block_size)), 1003, cuda_device, fused=True, scores=False)
+    compare(wl, ref, bufs, fused=True)
+
+
+def test_single_launch_decode_refuses_larger_blocks(cuda_device):
+    kw = dict(num_q_heads=16, num_kv_heads=2, num_idx_heads=16, block_size=128)
+    kw.update(BLOCK_CASES["decode_mix"])
+    wl = wk.make_workload(wk.WorkloadSpec("fd_b128", **kw), seed=18, device=cuda_device)
+    with pytest.raises(dsa.DsaError):
+        gpu_step(wl, fused_decode=True)
+
+
 # ----------------------------------------------------------------------------- invariants on the GPU
 def test_page_permutation_is_bit_identical(cuda_device):
     spec = _small_spec("prefill_two_chunks", "sharp")
@@ -450,9 +507,10 @@ def _appended_rows_match(wl, n_tokens):
         for j in range(n):
             i = int(cu[s_]) + j
             pos = int(lens[s_]) - n + j
-            page, slot = int(table[s_, pos // 64]), pos % 64
+            bs = spec.block_size
+            page, slot = int(table[s_, pos // bs]), pos % bs
             assert torch.equal(kp[page, slot], kn[i]) and torch.equal(vp[page, slot], vn[i]), (s_, j)
-            if j == n - 1 or slot == 63:
+            if j == n - 1 or slot == bs - 1:
                 assert torch.equal(kcp[page], kcn[i]), (s_, j)
     assert n_tokens == int(cu[-1])
 

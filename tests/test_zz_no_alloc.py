@@ -28,7 +28,7 @@ def _setup(spec, seed, device):
     seqs = dsa.SeqBatch(wl.block_table, wl.seq_lens)
     queries = dsa.QueryBatch(wl.cu_q, wl.q_pos)
     scores = dsa.index_score(cache, seqs, queries, wl.q_idx, wl.w)
-    sel, cnt = dsa.topk_blocks(seqs, queries, scores, wl.k_per_seq, spec.k_max)
+    sel, cnt = dsa.topk_blocks(seqs, queries, scores, wl.k_per_seq, spec.k_max, block_size=spec.block_size)
     return wl, cache, seqs, queries, sel, cnt
 
 
