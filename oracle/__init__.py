@@ -64,6 +64,10 @@ def _load():
             lib.oracle_kc_append.argtypes = [I, P, I, P, P, I, I, I, P, P]
             lib.oracle_index_score.argtypes = [I, P, P, P, I, I, I, P, I, P, P, I, P]
             lib.oracle_topk.argtypes = [I, P, P, I, P, I, P, I, P, P]
+            lib.oracle_index_score_fp8.argtypes = [I, P, P, P, I, I, I, P, I, P, P, I, P]
+            lib.oracle_index_score_fp8.restype = I
+            lib.oracle_e4m3_times_512.argtypes = [ctypes.c_uint8, ctypes.POINTER(ctypes.c_int)]
+            lib.oracle_e4m3_times_512.restype = ctypes.c_int64
             lib.oracle_sparse_attention.argtypes = [I, P, P, P, I, I, I, I, I, I, P, P, P,
                                                     P, P, I, ctypes.c_double, P, P]
             for f in (lib.oracle_kv_append, lib.oracle_kc_append, lib.oracle_index_score,
@@ -137,6 +141,29 @@ def index_score(q_seq, q_pos, block_table, block_size, kc_pool, q_idx, w):
         T, _ptr(_c(q_seq, np.int32)), _ptr(_c(q_pos, np.int32)), _ptr(bt), bt.shape[1],
         block_size, kc.shape[0], _ptr(kc), dd, _ptr(qi), _ptr(ww), H, _ptr(out))
     _check(rc, "index_score")
+    return out
+
+
+def e4m3_times_512(code: int):
+    """(value of the FP8 E4M3 code times 2^9 as an int, is_nan)."""
+    nan = ctypes.c_int(0)
+    v = _load().oracle_e4m3_times_512(int(code) & 0xFF, ctypes.byref(nan))
+    return int(v), bool(nan.value)
+
+
+def index_score_fp8(q_seq, q_pos, block_table, block_size, kc_pool, q_idx, w):
+    """Exact FP8 E4M3 block scores times 2^18, int64 [T][max_blocks]; INT64_MIN where
+    not visible.  kc_pool and q_idx hold E4M3 codes (uint8)."""
+    bt = _c(block_table, np.int32)
+    kc = _c(kc_pool, np.uint8)
+    qi = _c(q_idx, np.uint8)
+    ww = _c(w, np.int32)
+    T, H, dd = qi.shape
+    out = np.empty((T, bt.shape[1]), dtype=np.int64)
+    rc = _load().oracle_index_score_fp8(
+        T, _ptr(_c(q_seq, np.int32)), _ptr(_c(q_pos, np.int32)), _ptr(bt), bt.shape[1],
+        block_size, kc.shape[0], _ptr(kc), dd, _ptr(qi), _ptr(ww), H, _ptr(out))
+    _check(rc, "index_score_fp8")
     return out
 
 

@@ -170,6 +170,68 @@ int oracle_index_score(int total_q, const int32_t *q_seq, const int32_t *q_pos,
     return ORC_OK;
 }
 
+/*
+ * The value of an FP8 E4M3 code times 2^9 ("low-precision inputs" of the
+ * indexer [P5 "Index Selection Path"]; the format is the OCP 8-bit floating
+ * point E4M3: one sign bit, four exponent bits with bias 7, three mantissa
+ * bits, exponent field 0 for subnormals, codes 0x7F and 0xFF for NaN, no
+ * infinities).  A subnormal is (f/8) * 2^-6 = f * 2^-9 and a normal is
+ * (1 + f/8) * 2^(e-7) = (8 + f) * 2^(e-10), so every finite value times 2^9 is
+ * an integer of magnitude at most 448 * 2^9.  *is_nan is set for a NaN code.
+ */
+int64_t oracle_e4m3_times_512(uint8_t code, int *is_nan)
+{
+    int sign = code >> 7, e = (code >> 3) & 15, f = code & 7;
+    *is_nan = (e == 15 && f == 7);
+    if (*is_nan) return 0;
+    int64_t mag = (e == 0) ? (int64_t)f : ((int64_t)(8 + f) << (e - 1));
+    return sign ? -mag : mag;
+}
+
+/*
+ * Block scores of the FP8 indexer: the same formula as oracle_index_score
+ * with q_idx and the coarse keys as E4M3 codes, computed EXACTLY and returned
+ * times 2^18: S[t,b] * 2^18 = sum_h w[t,h] * max(0, sum_d (2^9 q[d]) (2^9 kc[d])).
+ * Each factor is an integer (oracle_e4m3_times_512), so the sum is exact in
+ * 128-bit integers; ORC_BAD_ARG if a code is NaN or a score does not fit int64.
+ */
+int oracle_index_score_fp8(int total_q, const int32_t *q_seq, const int32_t *q_pos,
+                           const int32_t *block_table, int max_blocks, int block_size,
+                           int num_pages, const uint8_t *kc_pool, int idx_dim,
+                           const uint8_t *q_idx, const int32_t *w, int num_idx_heads,
+                           int64_t *scores)
+{
+    for (int t = 0; t < total_q; ++t) {
+        int s = q_seq[t], p = q_pos[t];
+        if (p < 0) return ORC_BAD_POS;
+        int n_vis = p / block_size + 1;
+        if (n_vis > max_blocks) return ORC_BAD_POS;
+        for (int b = 0; b < max_blocks; ++b) scores[(long)t * max_blocks + b] = INT64_MIN;
+        for (int b = 0; b < n_vis; ++b) {
+            int page = block_table[(long)s * max_blocks + b];
+            if (page < 0 || page >= num_pages) return ORC_BAD_PAGE;
+            const uint8_t *kc = kc_pool + (long)page * idx_dim;
+            __int128 total = 0;
+            for (int h = 0; h < num_idx_heads; ++h) {
+                const uint8_t *q = q_idx + ((long)t * num_idx_heads + h) * idx_dim;
+                __int128 dot = 0;
+                for (int d = 0; d < idx_dim; ++d) {
+                    int nan_q, nan_k;
+                    int64_t qv = oracle_e4m3_times_512(q[d], &nan_q);
+                    int64_t kv = oracle_e4m3_times_512(kc[d], &nan_k);
+                    if (nan_q || nan_k) return ORC_BAD_ARG;
+                    dot += (__int128)qv * kv;
+                }
+                __int128 relu = dot > 0 ? dot : 0;
+                total += (__int128)w[(long)t * num_idx_heads + h] * relu;
+            }
+            if (total > (__int128)INT64_MAX || total <= (__int128)INT64_MIN) return ORC_BAD_ARG;
+            scores[(long)t * max_blocks + b] = (int64_t)total;
+        }
+    }
+    return ORC_OK;
+}
+
 /* candidate of the Top-K step: higher score first, then lower block id */
 typedef struct { int64_t score; int32_t block; } orc_cand;
 

@@ -43,6 +43,10 @@ MUTATIONS = {
     "one_candidate_short": ("for (int i = 0; i < k - 1; ++i) out[n++] = cand[i].block;",
                             "for (int i = 0; i < k - 2; ++i) out[n++] = cand[i].block;"),
     "append_one_slot_late": ("return seq_lens[s] - n + (i - cu_new[s]);", "return seq_lens[s] - n + (i - cu_new[s]) + 1;"),
+    "fp8_subnormal_as_normal": ("(e == 0) ? (int64_t)f :", "(e == 0) ? (int64_t)(8 + f) :"),
+    "fp8_exponent_bias_off": ("((int64_t)(8 + f) << (e - 1))", "((int64_t)(8 + f) << e)"),
+    "fp8_sign_ignored": ("return sign ? -mag : mag;", "return mag;"),
+    "fp8_relu_dropped": ("__int128 relu = dot > 0 ? dot : 0;", "__int128 relu = dot;"),
 }
 
 

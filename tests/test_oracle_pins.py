@@ -208,6 +208,108 @@ def test_topk_k_covers_all_visible():
     assert cnt[0] == 6 and sel[0, :6].tolist() == list(range(6))
 
 
+# ----------------------------------------------------------------------------- signed and wide weights
+def test_score_signed_weights_closed_form():
+    # negative weights subtract the ReLU term of their head:
+    # S = sum_h w_h max(0, 64 a c) with w = (-3, 5, -16)
+    H, D = 3, 64
+    for a, c in ((2, 9), (-4, 6), (0, 1)):
+        q = np.full((1, H, D), a, dtype=np.int8)
+        kc = np.full((1, D), c, dtype=np.int8)
+        w = np.array([[-3, 5, -16]], dtype=np.int32)
+        s = _single_seq_scores(q, w, kc, [0], [5], 64)
+        assert s[0, 0] == (-3 + 5 - 16) * max(0, D * a * c)
+
+
+def test_score_int32_overflowing_weights_exact_in_int64():
+    # weights near the int32 limit: the score leaves the int32 range and the
+    # oracle keeps it exact (python integers as the reference)
+    rng = np.random.default_rng(41)
+    H, D, nb = 16, 64, 6
+    q = _rand_int8(rng, (2, H, D))
+    kc = _rand_int8(rng, (nb, D))
+    w = rng.integers(-(2 ** 31) + 1, 2 ** 31 - 1, size=(2, H)).astype(np.int32)
+    s = _single_seq_scores(q, w, kc, np.arange(nb), [nb * 64 - 1] * 2, 64)
+    for t in range(2):
+        for b in range(nb):
+            ref = 0
+            for h in range(H):
+                dot = int(np.dot(q[t, h].astype(np.int64), kc[b].astype(np.int64)))
+                ref += int(w[t, h]) * max(0, dot)
+            assert int(s[t, b]) == ref
+    assert np.abs(s).max() > 2 ** 31
+
+
+# ----------------------------------------------------------------------------- FP8 (E4M3) scores
+def _e4m3_codes(rng, shape):
+    """finite E4M3 codes with magnitudes spread over the whole exponent range"""
+    mag = np.exp2(rng.uniform(-10, 9, size=shape)) * rng.choice([-1, 1], size=shape)
+    t = torch.from_numpy(np.clip(mag, -448, 448)).float().to(torch.float8_e4m3fn)
+    return t.view(torch.uint8).numpy()
+
+
+def test_fp8_decoding_matches_torch_float8():
+    codes = np.arange(256, dtype=np.uint8)
+    vals = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).double().numpy()
+    for c in range(256):
+        v, nan = orc.e4m3_times_512(c)
+        if np.isnan(vals[c]):
+            assert nan, c
+        else:
+            assert not nan and v == vals[c] * 512, c
+
+
+def test_fp8_scores_exact_against_python_integers():
+    # the definition with torch's float8 decoding and unbounded python integers
+    rng = np.random.default_rng(43)
+    H, D, nb, T, bs = 5, 64, 7, 3, 64
+    q = _e4m3_codes(rng, (T, H, D))
+    kc = _e4m3_codes(rng, (nb, D))
+    w = rng.integers(-20, 21, size=(T, H)).astype(np.int32)
+    perm = rng.permutation(nb)
+    pos = np.array([nb * bs - 1, 3 * bs + 1, 0])
+    s = orc.index_score_fp8(np.zeros(T, np.int32), pos.astype(np.int32), perm[None, :].astype(np.int32), bs, kc,
+                            q, w)
+    dq = torch.from_numpy(q.copy()).view(torch.float8_e4m3fn).double().numpy() * 512
+    dk = torch.from_numpy(kc.copy()).view(torch.float8_e4m3fn).double().numpy() * 512
+    for t in range(T):
+        for b in range(nb):
+            if b > pos[t] // bs:
+                assert s[t, b] == I64_MIN
+                continue
+            ref = 0
+            for h in range(H):
+                dot = sum(int(dq[t, h, d]) * int(dk[perm[b], d]) for d in range(D))
+                ref += int(w[t, h]) * max(0, dot)
+            assert int(s[t, b]) == ref
+
+
+def test_fp8_scores_on_integer_codes_equal_int8_scores():
+    # E4M3 holds every integer of magnitude <= 16 exactly: on such inputs the
+    # FP8 score is 2^18 times the int8 indexer's score
+    rng = np.random.default_rng(44)
+    H, D, nb, bs = 4, 64, 11, 64
+    qi = rng.integers(-16, 17, size=(2, H, D)).astype(np.int8)
+    ki = rng.integers(-16, 17, size=(nb, D)).astype(np.int8)
+    w = rng.integers(-16, 17, size=(2, H)).astype(np.int32)
+    to_codes = lambda x: torch.from_numpy(x.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    pos = [nb * bs - 1, 5 * bs]
+    s8 = _single_seq_scores(qi, w, ki, np.arange(nb), pos, bs)
+    sf = orc.index_score_fp8(np.zeros(2, np.int32), np.asarray(pos, np.int32), np.arange(nb, dtype=np.int32)[None, :],
+                             bs, to_codes(ki), to_codes(qi), w)
+    vis = s8 != I64_MIN
+    assert np.array_equal(sf[vis], s8[vis] * (1 << 18))
+    assert np.array_equal(sf[~vis], s8[~vis])
+
+
+def test_fp8_nan_code_is_refused():
+    q = np.zeros((1, 1, 64), np.uint8)
+    q[0, 0, 5] = 0x7F
+    with pytest.raises(ValueError):
+        orc.index_score_fp8(np.zeros(1, np.int32), np.array([10], np.int32), np.zeros((1, 1), np.int32), 64,
+                            np.zeros((1, 64), np.uint8), q, np.ones((1, 1), np.int32))
+
+
 # ----------------------------------------------------------------------------- attention
 def _tiny_spec(**kw):
     base = dict(name="tiny", seq_lens=(37,), n_new=(1,), k_per_seq=(64,), k_max=64,
