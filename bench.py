@@ -107,7 +107,7 @@ class ClockSampler:
         0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.001):
+    def __init__(self, device_index: int, period_s: float = 0.0002):
         self.samples, self.reasons = [], set()
         self.max_mhz = None
         self._stop = threading.Event()
@@ -429,6 +429,12 @@ def run_ours(args, world, rank, device):
             total_s = tm.rotated(rot_graph, steps_g, args.steps)
         else:
             total_s = sum(tm.isolated(case0.graph, case0.ev, args.steps)) / 1e3
+        torch.cuda.synchronize(device)
+        n_timed_samples = len(clk.samples)
+        # the same steps again, untimed, so that the clock record has more than
+        # a handful of samples of the load the timed region ran under
+        if rotate:
+            tm.rotated(rot_graph, steps_g, max(args.steps, 2000))
     torch.cuda.synchronize(device)
     barrier(world)
     n_attn = max(3 * n_case, min(args.steps, 300))
@@ -504,7 +510,8 @@ def run_ours(args, world, rank, device):
         "step_isolated_ms_median": round(statistics.median(iso_step_ms), 5),
         "e2e": e2e,
         "gpu_launches": len(case0.phases()) * args.steps,
-        "clocks": clk.summary(),
+        "clocks": dict(clk.summary(), samples_in_timed_region=n_timed_samples,
+                       how="NVML every 0.2 ms during the timed steps and the same steps repeated untimed"),
     }
     if rotate:
         del rot_graph, rot_attn
@@ -653,7 +660,7 @@ def end_to_end(cases, spec, path, decode, rotate, tm, world, device, stream, err
 
 
 # ----------------------------------------------------------------------------- the other workloads
-def measure_workload(name, device, steps=30, iso=15, seed=None):
+def measure_workload(name, device, steps=30, iso=15, seed=None, path="auto"):
     """A compact record of one of the other workloads: its step time (back to
     back over independent batches whose traffic exceeds the L2, or one step at
     a time after a cold-L2 flush when that would take more than MAX_ROTATE
@@ -661,7 +668,7 @@ def measure_workload(name, device, steps=30, iso=15, seed=None):
     roofline that bounds it."""
     from dynamic_block_sparse_dsa_b200 import workloads as wk
     spec = wk.NAMED[name]()
-    path, decode = pick_path(spec, "auto")
+    path, decode = pick_path(spec, path)
     err = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.Stream(device)
     tm = Timer(device, stream)
@@ -932,9 +939,12 @@ def main(argv=None):
         res["prefill_indexer"] = prefill_indexer(device)
     if world == 1 and not args.no_configs:
         # the other workloads, one GPU: step time and each launch against its roofline
-        res["configs"] = {n: measure_workload(n, device) for n in
-                          ("tiny_decode", "batched_gqa_decode", "chunked_prefill", "mixed_ragged",
-                           "decode_1m_b128", "decode_1m_b256", "decode_1m_b512")
+        # the prefill workloads also through the fused prefill pipeline:
+        # scoring and selection in one kernel (no score matrix), then attention
+        runs = [("tiny_decode", "auto"), ("batched_gqa_decode", "auto"), ("chunked_prefill", "auto"),
+                ("chunked_prefill", "fused_select"), ("mixed_ragged", "auto"), ("mixed_ragged", "fused_select"),
+                ("decode_1m_b128", "auto"), ("decode_1m_b256", "auto"), ("decode_1m_b512", "auto")]
+        res["configs"] = {(n if p == "auto" else f"{n}@{p}"): measure_workload(n, device, path=p) for n, p in runs
                           if n != args.workload}
     if rank == 0:
         print(json.dumps(res), flush=True)

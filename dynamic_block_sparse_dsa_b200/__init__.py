@@ -37,7 +37,8 @@ __all__ = [
     "PagedKVCache", "SeqBatch", "QueryBatch", "DsaError", "load",
     "kv_append", "index_score", "topk_blocks", "select_blocks", "select_blocks_append", "sparse_attn_decode",
     "sparse_attn_prefill", "decode_fused", "decode_workspace_size", "select_workspace_size",
-    "decode_fused_workspace_size", "sparse_attn_decode_noalloc", "step",
+    "decode_fused_workspace_size", "sparse_attn_decode_noalloc", "step", "index_score_i64", "index_score_fp8",
+    "topk_blocks_i64",
 ]
 
 BLOCK_SIZE = 64
@@ -81,7 +82,8 @@ class PagedKVCache:
     def ctype(self) -> _lib.KvCacheC:
         _expect(self.k_pool, torch.bfloat16, "k_pool")
         _expect(self.v_pool, torch.bfloat16, "v_pool")
-        _expect(self.kc_pool, torch.int8, "kc_pool")
+        if self.kc_pool.element_size() != 1:   # int8 codes, or E4M3 codes for index_score_fp8
+            raise ValueError(f"kc_pool must hold one byte per element, got {self.kc_pool.dtype}")
         n, bs, hkv, d = self.k_pool.shape
         return _lib.KvCacheC(_addr(self.k_pool), _addr(self.v_pool), _addr(self.kc_pool), n, bs, hkv, d,
                              self.kc_pool.shape[1])
@@ -164,6 +166,59 @@ def topk_blocks(seqs: SeqBatch, queries: QueryBatch, scores: torch.Tensor, k_per
         cnt = torch.empty((queries.total_q,), dtype=torch.int32, device=dev)
     s, q = seqs.ctype(), queries.ctype()
     _lib.check("dsa_topk_blocks", lib.dsa_topk_blocks(
+        ctypes.byref(s), ctypes.byref(q), _ptr(scores), _ptr(k_per_seq), int(k_max), int(block_size), _ptr(sel),
+        _ptr(cnt), _ptr(dev_err), _stream(stream)))
+    return sel, cnt
+
+
+def index_score_i64(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, q_idx: torch.Tensor, w: torch.Tensor,
+                    scores: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None, stream=None):
+    """int64 scores of the int8 indexer for any int32 weights: [total_q][max_blocks]."""
+    lib = load()
+    _expect(q_idx, torch.int8, "q_idx")
+    _expect(w, torch.int32, "w")
+    if scores is None:
+        scores = torch.empty((queries.total_q, seqs.block_table.shape[1]), dtype=torch.int64, device=q_idx.device)
+    c, s, q = cache.ctype(), seqs.ctype(), queries.ctype()
+    _lib.check("dsa_index_score_i64", lib.dsa_index_score_i64(
+        ctypes.byref(c), ctypes.byref(s), ctypes.byref(q), _ptr(q_idx), _ptr(w), q_idx.shape[1], _ptr(scores),
+        _ptr(dev_err), _stream(stream)))
+    return scores
+
+
+def index_score_fp8(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, q_idx_e4m3: torch.Tensor,
+                    w: torch.Tensor, w_abs_max: int = 16, scores: Optional[torch.Tensor] = None,
+                    dev_err: Optional[torch.Tensor] = None, stream=None):
+    """Exact FP8 (E4M3) block scores times 2^18, int64 [total_q][max_blocks].  ``q_idx_e4m3``
+    and ``cache.kc_pool`` hold E4M3 codes (uint8, or torch.float8_e4m3fn viewed as uint8)."""
+    lib = load()
+    if q_idx_e4m3.dtype == torch.float8_e4m3fn:
+        q_idx_e4m3 = q_idx_e4m3.view(torch.uint8)
+    _expect(q_idx_e4m3, torch.uint8, "q_idx_e4m3")
+    _expect(w, torch.int32, "w")
+    if scores is None:
+        scores = torch.empty((queries.total_q, seqs.block_table.shape[1]), dtype=torch.int64,
+                             device=q_idx_e4m3.device)
+    c, s, q = cache.ctype(), seqs.ctype(), queries.ctype()
+    _lib.check("dsa_index_score_fp8", lib.dsa_index_score_fp8(
+        ctypes.byref(c), ctypes.byref(s), ctypes.byref(q), _ptr(q_idx_e4m3), _ptr(w), q_idx_e4m3.shape[1],
+        int(w_abs_max), _ptr(scores), _ptr(dev_err), _stream(stream)))
+    return scores
+
+
+def topk_blocks_i64(seqs: SeqBatch, queries: QueryBatch, scores: torch.Tensor, k_per_seq: torch.Tensor, k_max: int,
+                    block_size: int = BLOCK_SIZE, sel: Optional[torch.Tensor] = None,
+                    cnt: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None, stream=None):
+    """topk_blocks over int64 scores (index_score_i64 / index_score_fp8)."""
+    lib = load()
+    _expect(scores, torch.int64, "scores")
+    dev = scores.device
+    if sel is None:
+        sel = torch.empty((queries.total_q, k_max), dtype=torch.int32, device=dev)
+    if cnt is None:
+        cnt = torch.empty((queries.total_q,), dtype=torch.int32, device=dev)
+    s, q = seqs.ctype(), queries.ctype()
+    _lib.check("dsa_topk_blocks_i64", lib.dsa_topk_blocks_i64(
         ctypes.byref(s), ctypes.byref(q), _ptr(scores), _ptr(k_per_seq), int(k_max), int(block_size), _ptr(sel),
         _ptr(cnt), _ptr(dev_err), _stream(stream)))
     return sel, cnt

@@ -17,7 +17,7 @@ _lock = threading.Lock()
 _lib = None
 
 DSA_OK, DSA_ERR_INVALID_ARG, DSA_ERR_UNSUPPORTED, DSA_ERR_RANGE, DSA_ERR_WORKSPACE, DSA_ERR_CUDA = range(6)
-DEV_ERR_PAGE, DEV_ERR_POS, DEV_ERR_SEL, DEV_ERR_K, DEV_ERR_WAIT = 1, 2, 4, 8, 16
+DEV_ERR_PAGE, DEV_ERR_POS, DEV_ERR_SEL, DEV_ERR_K, DEV_ERR_WAIT, DEV_ERR_VALUE = 1, 2, 4, 8, 16, 32
 
 c_i32 = ctypes.c_int32
 c_vp = ctypes.c_void_p
@@ -43,6 +43,10 @@ SIGNATURES = {
     "dsa_index_score": ([P(KvCacheC), P(SeqsC), P(QueriesC), c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp],
                         c_i32),
     "dsa_topk_blocks": ([P(SeqsC), P(QueriesC), c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp], c_i32),
+    "dsa_index_score_i64": ([P(KvCacheC), P(SeqsC), P(QueriesC), c_vp, c_vp, c_i32, c_vp, c_vp, c_vp], c_i32),
+    "dsa_index_score_fp8": ([P(KvCacheC), P(SeqsC), P(QueriesC), c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp],
+                            c_i32),
+    "dsa_topk_blocks_i64": ([P(SeqsC), P(QueriesC), c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp], c_i32),
     "dsa_select_blocks_workspace_size": ([c_i32], ctypes.c_size_t),
     "dsa_select_blocks": ([P(KvCacheC), P(SeqsC), P(QueriesC), c_vp, c_vp, c_i32, c_i32, c_vp, c_i32, c_vp, c_vp,
                            c_vp, ctypes.c_size_t, c_vp, c_vp], c_i32),

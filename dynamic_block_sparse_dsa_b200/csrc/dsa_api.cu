@@ -171,6 +171,32 @@ int select_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_que
                   const int32_t *k_per_seq, int32_t k_max, int32_t *sel, int32_t *cnt, void *workspace,
                   size_t workspace_bytes, const KvAppendArgs *app, int32_t *dev_err, dsa_stream_t stream);
 
+int wide_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries, const void *q_idx,
+                const int32_t *w, int32_t num_idx_heads, int64_t *scores, int32_t *dev_err, IndexScoreArgs &a) {
+    int rc;
+    if ((rc = check_cache(cache)) || (rc = check_seqs(seqs)) || (rc = check_queries(queries))) return rc;
+    if (num_idx_heads < 1) return DSA_ERR_INVALID_ARG;
+    if (num_idx_heads > kMaxIdxHeads) return DSA_ERR_UNSUPPORTED;
+    if (queries->total_q > 0 && (!q_idx || !w || !scores || !aligned16(q_idx))) return DSA_ERR_INVALID_ARG;
+    a = IndexScoreArgs{};
+    a.block_shift = block_shift_of(cache->block_size);
+    a.kc_pool = cache->kc_pool;
+    a.num_pages = cache->num_pages;
+    a.block_table = seqs->block_table;
+    a.max_blocks = seqs->max_blocks;
+    a.seq_lens = seqs->seq_lens;
+    a.num_seqs = seqs->num_seqs;
+    a.cu_q = queries->cu_q;
+    a.q_pos = queries->q_pos;
+    a.total_q = queries->total_q;
+    a.q_idx = static_cast<const int8_t *>(q_idx);
+    a.w = w;
+    a.num_idx_heads = num_idx_heads;
+    a.scores = nullptr;
+    a.dev_err = dev_err;
+    return DSA_OK;
+}
+
 }  // namespace
 
 namespace dsa {
@@ -290,6 +316,56 @@ int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int3
     a.cnt = cnt;
     a.dev_err = dev_err;
     return from_cuda(launch_topk(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+
+int dsa_index_score_i64(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                        const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads, int64_t *scores,
+                        int32_t *dev_err, dsa_stream_t stream) {
+    IndexScoreArgs a;
+    int rc = wide_common(cache, seqs, queries, q_idx, w, num_idx_heads, scores, dev_err, a);
+    if (rc || queries->total_q == 0) return rc;
+    return from_cuda(launch_index_score_wide(a, false, scores, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int dsa_index_score_fp8(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                        const uint8_t *q_idx_e4m3, const int32_t *w, int32_t num_idx_heads, int32_t w_abs_max,
+                        int64_t *scores, int32_t *dev_err, dsa_stream_t stream) {
+    IndexScoreArgs a;
+    int rc = wide_common(cache, seqs, queries, q_idx_e4m3, w, num_idx_heads, scores, dev_err, a);
+    if (rc) return rc;
+    if (w_abs_max < 0) return DSA_ERR_INVALID_ARG;
+    // |S| * 2^18 <= H * |w| * 64 * (448 * 2^9)^2 must stay below 2^63
+    const double bound = (double)num_idx_heads * w_abs_max * kIdxDim * (448.0 * 512.0) * (448.0 * 512.0);
+    if (bound >= 9.2e18) return DSA_ERR_RANGE;
+    if (queries->total_q == 0) return DSA_OK;
+    return from_cuda(launch_index_score_wide(a, true, scores, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int dsa_topk_blocks_i64(const dsa_seqs *seqs, const dsa_queries *queries, const int64_t *scores,
+                        const int32_t *k_per_seq, int32_t k_max, int32_t block_size, int32_t *sel,
+                        int32_t *cnt, int32_t *dev_err, dsa_stream_t stream) {
+    int rc;
+    if ((rc = check_seqs(seqs)) || (rc = check_queries(queries))) return rc;
+    if (k_max < 1) return DSA_ERR_INVALID_ARG;
+    if (block_shift_of(block_size) < 0 || k_max > kSelMaxK) return DSA_ERR_UNSUPPORTED;
+    if (queries->total_q == 0) return DSA_OK;
+    if (!scores || !k_per_seq || !sel || !cnt) return DSA_ERR_INVALID_ARG;
+    TopkArgs a{};
+    a.block_shift = block_shift_of(block_size);
+    a.seq_lens = seqs->seq_lens;
+    a.num_seqs = seqs->num_seqs;
+    a.max_blocks = seqs->max_blocks;
+    a.cu_q = queries->cu_q;
+    a.q_pos = queries->q_pos;
+    a.total_q = queries->total_q;
+    a.scores = nullptr;
+    a.k_per_seq = k_per_seq;
+    a.k_max = k_max;
+    a.sel = sel;
+    a.cnt = cnt;
+    a.dev_err = dev_err;
+    return from_cuda(launch_topk_wide(a, scores, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t dsa_select_blocks_workspace_size(int32_t total_q) {

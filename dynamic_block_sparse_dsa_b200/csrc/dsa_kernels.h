@@ -182,6 +182,10 @@ cudaError_t launch_index_score(const IndexScoreArgs &a, cudaStream_t stream);
 cudaError_t launch_index_score_tc(const IndexScoreArgs &a, int num_sms, cudaStream_t stream);
 int index_score_tc_min_queries_per_seq();
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t stream);
+// int64 scores: the int8 indexer without the int32 bound, or (fp8) the E4M3
+// indexer times 2^18; and the Top-K over such scores
+cudaError_t launch_index_score_wide(const IndexScoreArgs &a, bool fp8, int64_t *scores, cudaStream_t stream);
+cudaError_t launch_topk_wide(const TopkArgs &a, const int64_t *scores, cudaStream_t stream);
 cudaError_t launch_select_blocks(const SelectArgs &a, cudaStream_t stream);
 int topk_max_blocks();   // longest block table the standalone Top-K kernel accepts
 // the K/V pool and Q tensor maps are built by the launcher from AttnArgs

@@ -31,6 +31,7 @@ namespace {
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kCuqCache = 1024;   // cu_q entries staged in shared memory
+constexpr long long kSelBusyCtas = 8 * 148;   // a grid this large keeps every SM of a B200 busy
 }  // namespace
 
 template <int G>   // 64-block groups per warp: a chunk is kSelWarps * 64 * G blocks
@@ -188,41 +189,43 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
     }
     if (err_bits) set_err(a.dev_err, err_bits);
 
-    // ---- chunk Top-64 over the warps, kept sorted in the workspace
+    // ---- chunk Top-64 over the warps (the query's Top-64 when it has one chunk)
     cta_merge_top64<kSelWarps>(acc, s_lists);
-    key64 *cand = a.cand + ((size_t)t * kSelMaxChunks + c) * (kSelMaxK - 1);
-    if (warp == 0) {
-        if (lane < kk) cand[lane] = acc[0];
-        if (32 + lane < kk) cand[32 + lane] = acc[1];
-    }
-
-    // ---- the last chunk CTA of this query merges the chunks' lists: the
-    // barrier orders warp 0's list stores before tid 0's release-add, and the
-    // last adder's acquire (then the barrier) orders every list before the
-    // loads below
-    __syncthreads();
-    if (tid == 0) {
-        const int old = atomic_add_acq_rel_gpu(a.counters + t, 1);
-        s_last = (old == n_chunks - 1);
-    }
-    __syncthreads();
-    if (!s_last) return;
-    constexpr int kPer = (kSelMaxChunks + kSelWarps - 1) / kSelWarps;   // lists per warp
-    key64 lists[kPer][2];
+    if (n_chunks > 1) {
+        // kept sorted in the workspace
+        key64 *cand = a.cand + ((size_t)t * kSelMaxChunks + c) * (kSelMaxK - 1);
+        if (warp == 0) {
+            if (lane < kk) cand[lane] = acc[0];
+            if (32 + lane < kk) cand[32 + lane] = acc[1];
+        }
+        // ---- the last chunk CTA of this query merges the chunks' lists: the
+        // barrier orders warp 0's list stores before tid 0's release-add, and
+        // the last adder's acquire (then the barrier) orders every list before
+        // the loads below
+        __syncthreads();
+        if (tid == 0) {
+            const int old = atomic_add_acq_rel_gpu(a.counters + t, 1);
+            s_last = (old == n_chunks - 1);
+        }
+        __syncthreads();
+        if (!s_last) return;
+        constexpr int kPer = (kSelMaxChunks + kSelWarps - 1) / kSelWarps;   // lists per warp
+        key64 lists[kPer][2];
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) {   // every load in flight before the first merge
-        const int ci = warp + k * kSelWarps;
-        const key64 *src = a.cand + ((size_t)t * kSelMaxChunks + ci) * (kSelMaxK - 1);
-        const bool in = ci < n_chunks;
-        lists[k][0] = in && lane < kk ? __ldcg(src + lane) : 0ull;
-        lists[k][1] = in && 32 + lane < kk ? __ldcg(src + 32 + lane) : 0ull;
-    }
-    acc[0] = lists[0][0];
-    acc[1] = lists[0][1];
+        for (int k = 0; k < kPer; ++k) {   // every load in flight before the first merge
+            const int ci = warp + k * kSelWarps;
+            const key64 *src = a.cand + ((size_t)t * kSelMaxChunks + ci) * (kSelMaxK - 1);
+            const bool in = ci < n_chunks;
+            lists[k][0] = in && lane < kk ? __ldcg(src + lane) : 0ull;
+            lists[k][1] = in && 32 + lane < kk ? __ldcg(src + 32 + lane) : 0ull;
+        }
+        acc[0] = lists[0][0];
+        acc[1] = lists[0][1];
 #pragma unroll
-    for (int k = 1; k < kPer; ++k)
-        if (warp + k * kSelWarps < n_chunks) warp_merge64_desc(acc, lists[k]);
-    cta_merge_top64<kSelWarps>(acc, s_lists);
+        for (int k = 1; k < kPer; ++k)
+            if (warp + k * kSelWarps < n_chunks) warp_merge64_desc(acc, lists[k]);
+        cta_merge_top64<kSelWarps>(acc, s_lists);
+    }
     if (warp == 0) {
         // the winners (non-zero keys among the first kk) in ascending block order
         const bool v0 = lane < kk && acc[0] != 0ull, v1 = 32 + lane < kk && acc[1] != 0ull;
@@ -249,14 +252,22 @@ cudaError_t launch_select_blocks(const SelectArgs &a, cudaStream_t stream) {
     if (a.total_q == 0) return cudaSuccess;
     // the chunk size keeps every query at <= kSelMaxChunks chunks
     const int need = (a.max_blocks + kSelMaxChunks - 1) / kSelMaxChunks;   // blocks per chunk
-    const int gr = (need + kSelWarps * 64 - 1) / (kSelWarps * 64);
+    int gr = (need + kSelWarps * 64 - 1) / (kSelWarps * 64);
+    // with many queries (prefill) the grid fills the GPU anyway: larger chunks,
+    // down to one per query, leave fewer candidate lists to merge (none with
+    // one chunk: the query's only CTA writes its selection directly)
+    auto chunks = [&](int g) { return (a.max_blocks + kSelWarps * 64 * g - 1) / (kSelWarps * 64 * g); };
+    while (gr < 8 && chunks(gr) > 1 && (long long)a.total_q * chunks(2 * gr) >= kSelBusyCtas) gr *= 2;
     auto go = [&](auto kern, int G) {
         SelectArgs b = a;
         b.sel_rows = (a.max_blocks + kSelWarps * 64 * G - 1) / (kSelWarps * 64 * G);   // chunks
         const int app_rows = a.app.total_new > 0 ? (a.app.total_new + a.total_q - 1) / a.total_q : 0;
         if (b.sel_rows + app_rows > 65535) return cudaErrorInvalidValue;
         const dim3 grid(a.total_q, b.sel_rows + app_rows);
-        if (a.cu_new) {   // the overlapping append relies on nothing earlier still running
+        if (a.cu_new) {
+            // with the append in its grid: an ordinary launch, which starts once
+            // everything before it has finished (measured faster at 1M-token
+            // decode than a programmatic dependent of the attention before it)
             kern<<<grid, dim3(kSelThreads), 0, stream>>>(b);
             return cudaGetLastError();
         }

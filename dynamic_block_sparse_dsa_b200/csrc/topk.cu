@@ -7,18 +7,20 @@
 // Selection Path": the indices follow the gather's semantics; here they are
 // logical block ids, ascending, -1 padded.
 //
-// One CTA of 1024 threads per query.  Each warp streams groups of 64
-// candidates (coalesced loads), sorts each group with a warp bitonic network
-// and folds it into its running Top-64 (warp_topk.cuh); a merge tree over the
-// 32 warps leaves the query's Top-64 in warp 0, which appends the own block
-// and writes the winners in ascending block order.
+// One CTA of 256 threads per query (several resident per SM).  Each warp
+// streams groups of 64 candidates (coalesced loads): it sorts its first group
+// with a warp bitonic network and folds later ones into its running Top-64,
+// skipping, after one vote, every group with no key above the current
+// (K-1)-th (warp_topk.cuh); a merge tree over the 8 warps leaves the query's
+// Top-64 in warp 0, which appends the own block and writes the winners in
+// ascending block order.
 #include "dsa_kernels.h"
 #include "warp_topk.cuh"
 
 namespace dsa {
 
 namespace {
-constexpr int kTopkThreads = 1024;
+constexpr int kTopkThreads = 256;
 constexpr int kTopkWarps = kTopkThreads / 32;
 }  // namespace
 
@@ -57,9 +59,14 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
         const int i0 = g0 + lane, i1 = g0 + 32 + lane;
         key64 v[2] = {i0 < n ? make_key64(__ldg(row + i0), (uint32_t)i0) : 0ull,
                       i1 < n ? make_key64(__ldg(row + i1), (uint32_t)i1) : 0ull};
-        warp_sort64_desc(v);
-        if (first) { acc[0] = v[0]; acc[1] = v[1]; first = false; }
-        else warp_merge64_desc(acc, v);
+        if (first) {
+            warp_sort64_desc(v);
+            acc[0] = v[0];
+            acc[1] = v[1];
+            first = false;
+        } else {
+            warp_fold_topk(acc, v, kk);   // groups with nothing above the kk-th key cost one vote
+        }
     }
     cta_merge_top64<kTopkWarps>(acc, s_lists);
     if (warp == 0) {

@@ -311,6 +311,25 @@ def _plant(wl: Workload, gcpu: torch.Generator) -> None:
     wl.planted = planted.to(wl.device)
 
 
+def e4m3_indexer(wl: Workload, seed: int = 0):
+    """FP8 (E4M3) inputs for the FP8 indexer, drawn on the workload's device:
+    (q_idx codes uint8 [T][H][idx_dim], coarse-key codes uint8 [num_pages][idx_dim]).
+    Magnitudes are 2^u with u uniform in [-10, 9] and a random sign, clamped to
+    the E4M3 range (448) and rounded by torch's float8 conversion, so the codes
+    cover subnormals and the whole exponent range; no NaN code is drawn."""
+    spec = wl.spec
+    g = torch.Generator(device=wl.device)
+    g.manual_seed(seed + 104729)
+
+    def draw(shape):
+        u = torch.rand(shape, generator=g, device=wl.device) * 19.0 - 10.0
+        sign = torch.where(torch.rand(shape, generator=g, device=wl.device) < 0.5, -1.0, 1.0)
+        x = (torch.exp2(u) * sign).clamp(-448.0, 448.0)
+        return x.to(torch.float8_e4m3fn).view(torch.uint8)
+
+    return draw((spec.total_q, spec.num_idx_heads, spec.idx_dim)), draw((spec.num_pages, spec.idx_dim))
+
+
 def scaled(spec: WorkloadSpec, **kw) -> WorkloadSpec:
     """A copy of ``spec`` with fields replaced (e.g. q_scale, name)."""
     return replace(spec, **kw)

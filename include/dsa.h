@@ -82,6 +82,7 @@ enum {
 #define DSA_DEV_ERR_SEL 4u   /* selected block id outside the query's visible blocks */
 #define DSA_DEV_ERR_K 8u     /* k_per_seq[s] outside [1, k_max] */
 #define DSA_DEV_ERR_WAIT 16u /* a bounded in-kernel wait gave up (work of that unit skipped) */
+#define DSA_DEV_ERR_VALUE 32u /* an FP8 input code is NaN (read as 0) */
 
 typedef struct {
     void *k_pool;          /* bf16 [num_pages][block_size][num_kv_heads][head_dim] */
@@ -166,6 +167,43 @@ int dsa_index_score(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_q
 int dsa_topk_blocks(const dsa_seqs *seqs, const dsa_queries *queries, const int32_t *scores,
                     const int32_t *k_per_seq, int32_t k_max, int32_t block_size, int32_t *sel,
                     int32_t *cnt, int32_t *dev_err, dsa_stream_t stream);
+
+/*
+ * Wide scores [P5 "Index Selection Path": the scoring operator takes
+ * low-precision inputs; P1 4(1)].  The same formula as dsa_index_score, with
+ * int64 results, for the cases the int32 path refuses or does not take:
+ *
+ * dsa_index_score_i64 -- int8 q_idx and coarse keys, any int32 weights (no
+ *   w_abs_max bound): the dot products are exact in int32 and the weighted sum
+ *   is accumulated in int64.  scores int64 [total_q][max_blocks], visible
+ *   entries written as in dsa_index_score.
+ *
+ * dsa_index_score_fp8 -- q_idx and the coarse keys (cache->kc_pool, read as
+ *   bytes) hold FP8 E4M3 codes (OCP 8-bit float: bias 7, 3 mantissa bits,
+ *   subnormals, 0x7F and 0xFF are NaN).  Every finite E4M3 value times 2^9 is
+ *   an integer, so the score is computed exactly and returned times 2^18:
+ *       scores[t][b] = sum_h w[t][h] * max(0, sum_d (2^9 q[t][h][d]) (2^9 kc[d]))
+ *   (int64; the selection it gives is exact and does not depend on any
+ *   summation order).  |w| <= w_abs_max; DSA_ERR_RANGE when
+ *   num_idx_heads * w_abs_max * idx_dim * (448 * 2^9)^2 >= 2^63.  A NaN code is
+ *   read as 0 and sets DSA_DEV_ERR_VALUE.
+ *
+ * dsa_topk_blocks_i64 -- dsa_topk_blocks over int64 scores (either call above).
+ *
+ * Both scoring calls run on the CUDA cores (256 blocks of one sequence per
+ * CTA).  Device errors: those of the int32 calls, and DSA_DEV_ERR_VALUE.
+ */
+int dsa_index_score_i64(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                        const int8_t *q_idx, const int32_t *w, int32_t num_idx_heads, int64_t *scores,
+                        int32_t *dev_err, dsa_stream_t stream);
+
+int dsa_index_score_fp8(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,
+                        const uint8_t *q_idx_e4m3, const int32_t *w, int32_t num_idx_heads, int32_t w_abs_max,
+                        int64_t *scores, int32_t *dev_err, dsa_stream_t stream);
+
+int dsa_topk_blocks_i64(const dsa_seqs *seqs, const dsa_queries *queries, const int64_t *scores,
+                        const int32_t *k_per_seq, int32_t k_max, int32_t block_size, int32_t *sel,
+                        int32_t *cnt, int32_t *dev_err, dsa_stream_t stream);
 
 /*
  * dsa_select_blocks -- dsa_index_score and dsa_topk_blocks in one pass, with

@@ -135,6 +135,30 @@ def oracle_step(wl, queries=None, with_append: bool = True, want_scores: bool = 
     return run_host(host_inputs(wl, queries, with_append), want_scores=want_scores)
 
 
+def oracle_select(wl, q_idx=None, w=None, kc_pool=None, fp8: bool = False, queries=None):
+    """The oracle's scores and selection for the workload's queries (no append),
+    with optional replacement indexer inputs: int8 q_idx / kc_pool (any int32
+    weights), or, with ``fp8``, E4M3 codes for both (scores times 2^18).
+    Returns a dict with ``queries``, ``scores`` int64 [n][max_blocks], ``sel``, ``cnt``."""
+    spec = wl.spec
+    table = _np(wl.block_table).astype(np.int32)
+    cu = _np(wl.cu_q).astype(np.int32)
+    q_pos_all = _np(wl.q_pos).astype(np.int32)
+    q_seq_all = orc.queries_to_seq(cu)
+    T = len(q_pos_all)
+    qs = np.arange(T, dtype=np.int64) if queries is None else np.asarray(queries, dtype=np.int64)
+    qi = _np(wl.q_idx if q_idx is None else q_idx)[qs]
+    ww = _np(wl.w if w is None else w)[qs]
+    kc = _np(wl.kc_pool if kc_pool is None else kc_pool)
+    if fp8:
+        scores = orc.index_score_fp8(q_seq_all[qs], q_pos_all[qs], table, spec.block_size, kc, qi, ww)
+    else:
+        scores = orc.index_score(q_seq_all[qs], q_pos_all[qs], table, spec.block_size, kc, qi, ww)
+    sel, cnt = orc.topk(q_seq_all[qs], q_pos_all[qs], spec.block_size, scores, _np(wl.k_per_seq).astype(np.int32),
+                        spec.k_max)
+    return {"queries": qs, "scores": scores, "sel": sel, "cnt": cnt}
+
+
 def save_inputs(inp: dict, directory: str) -> None:
     """Write ``host_inputs``' arrays as .npy files (for worker processes)."""
     import os

@@ -215,3 +215,35 @@ def test_noalloc_refuses_bad_calls_before_any_device_work():
     assert na() == _lib.DSA_ERR_WORKSPACE
     # nothing to do: accepted without touching the device
     assert na(total_q=0) == _lib.DSA_OK
+
+
+def test_wide_score_validation_codes():
+    """int64 and FP8 scoring and the int64 Top-K refuse bad arguments on the
+    host (dummy pointers, never dereferenced)."""
+    lib = _lib.load()
+    c, s, q = _cache(), _seqs(), _queries()
+
+    def fp8(wmax=16, heads=16, qidx=FAKE):
+        return lib.dsa_index_score_fp8(ctypes.byref(c), ctypes.byref(s), ctypes.byref(q), qidx, FAKE, heads, wmax,
+                                       FAKE, None, None)
+
+    # 16 heads * 64 * (448 * 2^9)^2 * w must stay below 2^63: w = 1 << 20 is too large
+    assert fp8(wmax=1 << 20) == _lib.DSA_ERR_RANGE
+    assert fp8(wmax=-1) == _lib.DSA_ERR_INVALID_ARG
+    assert fp8(heads=17) == _lib.DSA_ERR_UNSUPPORTED
+    assert fp8(qidx=FAKE + 4) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_index_score_i64(ctypes.byref(c), ctypes.byref(s), ctypes.byref(q), FAKE, FAKE, 0, FAKE, None,
+                                   None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_index_score_i64(ctypes.byref(_cache(block_size=100)), ctypes.byref(s), ctypes.byref(q), FAKE,
+                                   FAKE, 4, FAKE, None, None) == _lib.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_index_score_i64(ctypes.byref(c), ctypes.byref(s), ctypes.byref(_queries(total_q=0)), FAKE, FAKE,
+                                   4, FAKE, None, None) == _lib.DSA_OK
+
+    def tk(k_max=8, bs=64, queries=q):
+        return lib.dsa_topk_blocks_i64(ctypes.byref(s), ctypes.byref(queries), FAKE, FAKE, k_max, bs, FAKE, FAKE,
+                                       None, None)
+
+    assert tk(k_max=0) == _lib.DSA_ERR_INVALID_ARG
+    assert tk(k_max=65) == _lib.DSA_ERR_UNSUPPORTED
+    assert tk(bs=48) == _lib.DSA_ERR_UNSUPPORTED
+    assert tk(queries=_queries(total_q=0)) == _lib.DSA_OK

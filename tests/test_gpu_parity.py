@@ -174,15 +174,18 @@ def _sample_queries(wl, n, rng):
 
 
 @pytest.mark.slow
+@pytest.mark.parametrize("fused", [False, True], ids=["score_topk", "fused_prefill"])
 @pytest.mark.parametrize("profile", PROFILES)
-def test_chunked_prefill_workload_sampled(profile, cuda_device):
+def test_chunked_prefill_workload_sampled(profile, fused, cuda_device):
+    """Separate scoring (tensor cores) + Top-K, or the fused prefill pipeline
+    (scoring and selection in one kernel, no score matrix, then attention)."""
     spec = profiled(wk.chunked_prefill(), profile)
     wl = wk.make_workload(spec, seed=1004, device=cuda_device)
     qs = _sample_queries(wl, 40, np.random.default_rng(0))
     ref = oracle_step(wl, queries=qs, want_scores=True)
-    bufs, err = gpu_step(wl, decode=False)
+    bufs, err = gpu_step(wl, decode=False, fused=fused)
     assert err == 0
-    compare(wl, ref, bufs)
+    compare(wl, ref, bufs, fused=fused)
     # properties of every query at full size
     cnt = bufs["cnt"].cpu().numpy()
     sel = bufs["sel"].cpu().numpy()
@@ -193,7 +196,7 @@ def test_chunked_prefill_workload_sampled(profile, cuda_device):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("decode,fused", [(True, False), (False, False), (True, True)])
+@pytest.mark.parametrize("decode,fused", [(True, False), (False, False), (True, True), (False, True)])
 @pytest.mark.parametrize("profile", PROFILES)
 def test_mixed_ragged_workload_sampled(profile, decode, fused, cuda_device):
     spec = profiled(wk.mixed_ragged(), profile)
@@ -449,6 +452,30 @@ def test_fused_decode_repeat_calls_and_equals_three_kernel_path(cuda_device):
             assert torch.equal(b[k], b_ref[k]), k
     ref = oracle_step(wl)
     compare(wl, ref, b, fused=True)
+
+
+def test_fused_decode_wait_runs_out_and_recovers(cuda_device):
+    """The single-launch step's wait for the appended tokens is bounded.  With a
+    token count that can never be reached -- the workspace's appended-token
+    counter (int32 word 2 of its 256-byte header) set far below zero before the
+    call -- every producer gives up after the in-kernel limit (2^32 SM cycles,
+    about 2 s), the call returns with DSA_DEV_ERR_WAIT, and the kernel leaves
+    the workspace ready again: the next call is exact."""
+    import time
+    wl = wk.make_workload(_small_spec("many_seqs_decode", "sharp"), seed=45, device=cuda_device)
+    ref = oracle_step(wl)
+    bufs, err = gpu_step(wl, fused_decode=True)
+    assert err == 0
+    compare(wl, ref, bufs, fused=True)
+    bufs["fused_ws"][:256].view(torch.int32)[2] = -(1 << 30)
+    t0 = time.time()
+    bufs, err = gpu_step(wl, bufs=bufs, fused_decode=True)   # appends the same tokens again: idempotent
+    assert err & dsa._lib.DEV_ERR_WAIT
+    assert time.time() - t0 < 120
+    assert int(bufs["fused_ws"][:256].view(torch.int32)[2]) == 0
+    bufs, err = gpu_step(wl, bufs=bufs, fused_decode=True)
+    assert err == 0
+    compare(wl, ref, bufs, fused=True)
 
 
 @pytest.mark.parametrize("what", ["page", "pos", "k"])

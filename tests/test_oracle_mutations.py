@@ -18,8 +18,30 @@ MUTATIONS = {
     "relu_is_abs": ("int64_t relu = dot > 0 ? dot : 0;", "int64_t relu = dot > 0 ? dot : -dot;"),
     "logical_not_physical_page": ("const int8_t *kc = kc_pool + (long)page * idx_dim;",
                                   "const int8_t *kc = kc_pool + (long)b * idx_dim;"),
-    "visibility_off_by_one": ("int n_vis = p / block_size + 1;\n        if (n_vis > max_blocks)",
-                              "int n_vis = p / block_size;\n        if (n_vis > max_blocks)"),
+    "visibility_off_by_one": ("int n_vis = p / block_size + 1;\n        if (n_vis > max_blocks) return ORC_BAD_POS;\n"
+                              "        for (int b = 0; b < max_blocks; ++b) scores[(long)t * max_blocks + b] = INT64_MIN;\n"
+                              "        for (int b = 0; b < n_vis; ++b) {\n"
+                              "            int page = block_table[(long)s * max_blocks + b];\n"
+                              "            if (page < 0 || page >= num_pages) return ORC_BAD_PAGE;\n"
+                              "            const int8_t *kc",
+                              "int n_vis = p / block_size;\n        if (n_vis > max_blocks) return ORC_BAD_POS;\n"
+                              "        for (int b = 0; b < max_blocks; ++b) scores[(long)t * max_blocks + b] = INT64_MIN;\n"
+                              "        for (int b = 0; b < n_vis; ++b) {\n"
+                              "            int page = block_table[(long)s * max_blocks + b];\n"
+                              "            if (page < 0 || page >= num_pages) return ORC_BAD_PAGE;\n"
+                              "            const int8_t *kc"),
+    "fp8_visibility_off_by_one": ("int n_vis = p / block_size + 1;\n        if (n_vis > max_blocks) return ORC_BAD_POS;\n"
+                                  "        for (int b = 0; b < max_blocks; ++b) scores[(long)t * max_blocks + b] = INT64_MIN;\n"
+                                  "        for (int b = 0; b < n_vis; ++b) {\n"
+                                  "            int page = block_table[(long)s * max_blocks + b];\n"
+                                  "            if (page < 0 || page >= num_pages) return ORC_BAD_PAGE;\n"
+                                  "            const uint8_t *kc",
+                                  "int n_vis = p / block_size;\n        if (n_vis > max_blocks) return ORC_BAD_POS;\n"
+                                  "        for (int b = 0; b < max_blocks; ++b) scores[(long)t * max_blocks + b] = INT64_MIN;\n"
+                                  "        for (int b = 0; b < n_vis; ++b) {\n"
+                                  "            int page = block_table[(long)s * max_blocks + b];\n"
+                                  "            if (page < 0 || page >= num_pages) return ORC_BAD_PAGE;\n"
+                                  "            const uint8_t *kc"),
     "weight_index_transposed": ("total += (int64_t)w[(long)t * num_idx_heads + h] * relu;",
                                 "total += (int64_t)w[(long)h * num_idx_heads + t % num_idx_heads] * relu;"),
     "tie_break_reversed": ("return (x->block > y->block) - (x->block < y->block);",
