@@ -185,7 +185,13 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
         } else if (gi == 0) {
             pdl_wait();
         }
-        warp_fold_topk(acc, v, kk);
+        if (gi == 0) {   // the first group: sorted, it is the warp's list (nothing to merge with)
+            warp_sort64_desc(v);
+            acc[0] = v[0];
+            acc[1] = v[1];
+        } else {
+            warp_fold_topk(acc, v, kk);
+        }
     }
     if (err_bits) set_err(a.dev_err, err_bits);
 
