@@ -31,10 +31,13 @@
 //         still reading that buffer have finished;
 //   1     MMA issuer (one thread): two K = 32 MMAs per item into one of two
 //         256-column accumulators;
-//   2-17  epilogue (four per SM sub-partition: a quarter of the rows and a
-//         quarter of the queries each): tcgen05.ld, after which the
-//         accumulator goes straight back to the MMA, then relu * w summed
-//         over heads and one coalesced 128-byte store per (query, warp).
+//   2-17  epilogue, two groups of eight warps taking alternate items (and the
+//         two accumulators), so that one group's tensor-memory loads overlap
+//         the other's arithmetic; in a group the two warps of each SM
+//         sub-partition take that sub-partition's 32 rows and half of the
+//         queries each, in two rounds of four queries: tcgen05.ld, after the
+//         second of which the accumulator goes back to the MMA, then relu * w
+//         summed over heads and one coalesced 128-byte store per (query, warp).
 // A query tile spanning several sequences runs once per sequence with the
 // other queries masked; items past every query's own block are skipped.  All
 // waits are bounded.
@@ -89,7 +92,8 @@ constexpr int kSmemBytes = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
 constexpr int kFullCountTma = 1;
 constexpr int kFullCountCpAsync = 33;
 constexpr int kAFullCount = 33;                      // the loader: 32 cp.async arrivals + one
-constexpr int kEmptyCount = 1 + kEpiWarps;           // MMA commit + the epilogue warps
+constexpr int kEpiGroup = kEpiWarps / 2;             // epilogue warps per item (two groups alternate items)
+constexpr int kEmptyCount = 1 + kEpiGroup;           // MMA commit + the item's epilogue warps
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 static_assert(kOffA % 1024 == 0, "A buffers keep the 64-byte swizzle's 512-byte alignment");
@@ -139,7 +143,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bars.tfull(b), 1);
-            mbar_init(bars.tempty(b), kEpiWarps);
+            mbar_init(bars.tempty(b), kEpiGroup);
             mbar_init(bars.afull(b), kAFullCount);
         }
         misc[1] = 0;
@@ -244,10 +248,16 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // cannot be confused with item j + 4's, which waits for this very
         // barrier before it is published (j < k - 4 is known finished already).
         int k_seen = -1;   // the latest item known to be finished
+        // Two epilogue groups take alternate items, each in order: items j and
+        // j - 1 finished mean every item before them is.  When item k is
+        // published, item k - 5 is known finished (the wait for item k - 1's
+        // stage), so neither wait below can meet a reused stage's later phase.
         auto wait_done = [&](int end) {
             const int j = end - 1;
             if (j <= k_seen) return true;
-            if (!mbar_wait(bars.empty(j & (kTcStages - 1)), (j / kTcStages) & 1, s_abort)) {
+            if (!mbar_wait(bars.empty(j & (kTcStages - 1)), (j / kTcStages) & 1, s_abort) ||
+                (j - 1 > k_seen && j >= 1 &&
+                 !mbar_wait(bars.empty((j - 1) & (kTcStages - 1)), ((j - 1) / kTcStages) & 1, s_abort))) {
                 *s_abort = 1;
                 return false;
             }
@@ -419,8 +429,8 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             fetch_batch(b0 + 2 * kBatch, pbuf);
             if (*s_abort) stop = true;
         }
-        // the end marker
-        if (!stop && !*s_abort) {
+        // two end markers: one for each epilogue group
+        for (int e = 0; e < 2 && !stop && !*s_abort; ++e) {
             const int st = k & (kTcStages - 1);
             if (k >= kTcStages && !mbar_wait(bars.empty(st), ((k / kTcStages) - 1) & 1, s_abort)) {
                 *s_abort = 1;
@@ -445,7 +455,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
         constexpr uint32_t idesc = tc::idesc_i8(kBT, kN);
-        int k = 0;
+        int k = 0, n_end = 0;
         while (true) {
             const int st = k % kTcStages, buf = k & 1;
             bool ok = mbar_wait(bars.full(st), (k / kTcStages) & 1, s_abort);
@@ -478,7 +488,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             __syncwarp();
             ++k;
-            if (end) break;
+            if (end && ++n_end == 2) break;
         }
         // the last MMAs have completed before the accumulator is released
         if (lane == 0 && k > 0) {
@@ -487,12 +497,18 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
     } else {
         // ============================================================ epilogue
+        // two groups of 8 warps take alternate items (group g: items g, g+2, ...,
+        // accumulator g), so one group's tensor-memory loads overlap the other's
+        // arithmetic.  In a group, the two warps of a sub-partition take the
+        // 32 rows that sub-partition can read and half of the 16 queries each,
+        // in two rounds of 4 queries (64 accumulator columns).
         const int ew = warp - kEpiWarp0;
+        const int grp = ew >> 3;                 // items of parity grp
         const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
-        const int qgrp = ew >> 2;                // queries 4*qgrp .. +3 (columns 64*qgrp ..)
+        const int half = (ew >> 2) & 1;          // queries 8*half .. +7
         const int row = quarter * 32 + lane;     // block row of the tile
         const int *s_own_e = reinterpret_cast<const int *>(g + kOffOwn);
-        int k = 0;
+        int k = grp;
         while (true) {
             const int st = k % kTcStages, buf = k & 1;
             bool ok = mbar_wait(bars.tfull(buf), (k >> 1) & 1, s_abort) &&
@@ -508,38 +524,43 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const int bt = i0w.x, y = i0w.y, mask = i0w.w;
             const int b = bt * kBT + row;
             const bool row_ok = (info->vbits[quarter] >> lane) & 1u;
-            const uint32_t taddr =
-                tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kN + qgrp * 64);
-            // own blocks of this warp's 4 queries (-1 outside this item's sequence) and their weights
-            const int4 o4 = *reinterpret_cast<const int4 *>(s_own_e + info->own_off + 4 * qgrp);
-            const int own4[4] = {(mask >> (4 * qgrp)) & 1 ? o4.x : -1, (mask >> (4 * qgrp + 1)) & 1 ? o4.y : -1,
-                                 (mask >> (4 * qgrp + 2)) & 1 ? o4.z : -1, (mask >> (4 * qgrp + 3)) & 1 ? o4.w : -1};
-            const int4 *w4 = reinterpret_cast<const int4 *>(g + st * kStageBytes + kOffW) + qgrp * kMaxIdxHeads;
             uint32_t v[2][32];
-            tc::ld_32x32b_x32(taddr, v[0]);
-            tc::ld_32x32b_x32(taddr + 32, v[1]);
-            tc::wait_ld();
-            // the accumulator is in registers: release it to the next MMA now
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bars.tempty(buf));
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {   // query 4*qgrp + u: columns 16u .. 16u+15 of this warp's 64
-                const uint32_t *x = v[u >> 1] + 16 * (u & 1);
-                int part[4];
-#pragma unroll
-                for (int h4 = 0; h4 < 4; ++h4) {   // four independent chains
-                    const int4 wv = w4[u * (kMaxIdxHeads / 4) + h4];
-                    part[h4] = wv.x * max((int)x[4 * h4 + 0], 0) + wv.y * max((int)x[4 * h4 + 1], 0) +
-                               wv.z * max((int)x[4 * h4 + 2], 0) + wv.w * max((int)x[4 * h4 + 3], 0);
+            for (int rnd = 0; rnd < 2; ++rnd) {
+                const int qgrp = 2 * half + rnd;   // queries 4*qgrp .. +3 (columns 64*qgrp ..)
+                const uint32_t taddr =
+                    tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kN + qgrp * 64);
+                tc::ld_32x32b_x32(taddr, v[0]);
+                tc::ld_32x32b_x32(taddr + 32, v[1]);
+                tc::wait_ld();
+                if (rnd == 1) {
+                    // the accumulator is all in registers: release it to the next MMA
+                    tc::fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bars.tempty(buf));
                 }
-                const int sum = (part[0] + part[1]) + (part[2] + part[3]);
-                if (row_ok && b <= own4[u])
-                    a.scores[(size_t)(kQT * y + 4 * qgrp + u) * a.max_blocks + b] = sum;
+                const int4 o4 = *reinterpret_cast<const int4 *>(s_own_e + info->own_off + 4 * qgrp);
+                const int own4[4] = {(mask >> (4 * qgrp)) & 1 ? o4.x : -1, (mask >> (4 * qgrp + 1)) & 1 ? o4.y : -1,
+                                     (mask >> (4 * qgrp + 2)) & 1 ? o4.z : -1, (mask >> (4 * qgrp + 3)) & 1 ? o4.w : -1};
+                const int4 *w4 = reinterpret_cast<const int4 *>(g + st * kStageBytes + kOffW) + qgrp * kMaxIdxHeads;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {   // query 4*qgrp + u: columns 16u .. 16u+15 of these 64
+                    const uint32_t *x = v[u >> 1] + 16 * (u & 1);
+                    int part[4];
+#pragma unroll
+                    for (int h4 = 0; h4 < 4; ++h4) {   // four independent chains
+                        const int4 wv = w4[u * (kMaxIdxHeads / 4) + h4];
+                        part[h4] = wv.x * max((int)x[4 * h4 + 0], 0) + wv.y * max((int)x[4 * h4 + 1], 0) +
+                                   wv.z * max((int)x[4 * h4 + 2], 0) + wv.w * max((int)x[4 * h4 + 3], 0);
+                    }
+                    const int sum = (part[0] + part[1]) + (part[2] + part[3]);
+                    if (row_ok && b <= own4[u])
+                        a.scores[(size_t)(kQT * y + 4 * qgrp + u) * a.max_blocks + b] = sum;
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.empty(st));   // the stage (info, weights, own blocks) is read
-            ++k;
+            k += 2;
         }
     }
 

@@ -443,6 +443,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             __syncwarp();
             const int blk = W[kWItemBlk + st];
             const uint32_t tk = sm.stage(st), tv = tk + 2 * kHalf;
+            // the last visible token of this tile (only the query's own tile is partial)
+            const int lim = (blk == pnv - 1) ? pp - blk * kBlockSize : kBlockSize - 1;
+            if (lim < kBlockSize - 1) {
+                // the slots past the query's position hold whatever the cache had
+                // there (nothing appended yet); a zero softmax weight times a NaN
+                // or infinite value is still NaN, so their value rows are cleared
+                // (both 128-byte halves, 16-byte chunks at their swizzled place)
+                for (int e = lane; e < (kBlockSize - 1 - lim) * 16; e += 32) {
+                    const int r = lim + 1 + (e >> 4), cc = e & 15;
+                    st_shared_zero16(tv + (cc >> 3) * kHalf + swz128(r, cc & 7));
+                }
+                __syncwarp();
+            }
             // ---- S^T = K Q^T: 4 m-tiles of 16 tokens x NT n-tiles of 8 heads
             float sc[4][NT][4];
 #pragma unroll
@@ -463,7 +476,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 }
             }
             // ---- causal mask (own block only), scale, online softmax per head column
-            const int lim = (blk == pnv - 1) ? pp - blk * kBlockSize : kBlockSize - 1;
             float alpha[NT][2];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
@@ -523,6 +535,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[dm][nt], va, pb[nt][0], pb[nt][1]);
                 }
             }
+            // generic-proxy stores (the cleared rows) before the TMA refills the stage
+            if (lim < kBlockSize - 1) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) mbar_arrive(sm.empty(st));
             ui += kConsumerWarps;

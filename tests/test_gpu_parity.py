@@ -290,6 +290,31 @@ def test_page_permutation_is_bit_identical(cuda_device):
         assert torch.equal(b1[k], b2[k]), k
 
 
+@pytest.mark.parametrize("block_size", [64, 256])
+@pytest.mark.parametrize("fused", [False, True], ids=["score_topk", "fused_select"])
+@pytest.mark.parametrize("decode", [True, False], ids=["decode_entry", "prefill_entry"])
+def test_unwritten_cache_slots_holding_nan(decode, fused, block_size, cuda_device):
+    """Slots of a sequence's last block past its length hold whatever the
+    cache had there (here NaN in K and V).  They are masked out, and a zero
+    softmax weight times NaN must not reach the output: results equal the
+    oracle's, which never reads those slots."""
+    kw = dict(num_q_heads=16, num_kv_heads=2, num_idx_heads=16, block_size=block_size)
+    kw.update(SMALL["ragged_prefill_tail"])
+    spec = wk.sharp(wk.WorkloadSpec(f"nan_tail_b{block_size}", **kw))
+    wl = wk.make_workload(spec, seed=46, device=cuda_device)
+    table = wl.block_table.cpu()
+    for s_, L in enumerate(spec.seq_lens):
+        if L % block_size:
+            page = int(table[s_, (L - 1) // block_size])
+            wl.k_pool[page, L % block_size:] = float("nan")
+            wl.v_pool[page, L % block_size:] = float("nan")
+    ref = oracle_step(wl)
+    bufs, err = gpu_step(wl, decode=decode, fused=fused)
+    assert err == 0
+    assert not torch.isnan(bufs["out"]).any() and not torch.isnan(bufs["lse"]).any()
+    compare(wl, ref, bufs, fused=fused)
+
+
 def test_v_all_ones_gives_ones(cuda_device):
     spec = _small_spec("ragged_prefill_tail", "sharp")
     wl = wk.make_workload(spec, seed=8, device=cuda_device)
