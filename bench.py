@@ -564,16 +564,20 @@ def end_to_end(cases, spec, path, decode, rotate, tm, world, device, stream, err
             self.bufs["out"] = view(self.dev_out_buf, out_offs["out"], c.bufs["out"])
             self.bufs["lse"] = view(self.dev_out_buf, out_offs["lse"], c.bufs["lse"])
             self.c = c
+            d = self.dev_in
+            # the step's calls with their arguments marshalled once (the public
+            # PreparedStep: a serving loop's way of issuing the same step again)
+            self.prep = dsa.PreparedStep(c.cache, c.seqs, c.queries, bufs=self.bufs, k_new=d["k_new"],
+                                         v_new=d["v_new"], kc_new=d["kc_new"], q=d["q"], q_idx=d["q_idx"], w=d["w"],
+                                         k_per_seq=c.wl.k_per_seq, k_max=spec.k_max, decode=decode,
+                                         fused_select=fused, overlap_append=fused and decode,
+                                         fused_decode=fused_decode, dev_err=err)
             self.in_ready = torch.cuda.Event()   # graph only: this batch's inputs landed
             self.consumed = torch.cuda.Event()   # its step ran
             self.out_done = torch.cuda.Event()   # its outputs read back
 
         def compute(self):
-            c, d = self.c, self.dev_in
-            dsa.step(c.cache, c.seqs, c.queries, k_new=d["k_new"], v_new=d["v_new"], kc_new=d["kc_new"], q=d["q"],
-                     q_idx=d["q_idx"], w=d["w"], k_per_seq=c.wl.k_per_seq, k_max=spec.k_max, decode=decode,
-                     fused_select=fused, overlap_append=fused and decode, fused_decode=fused_decode,
-                     bufs=self.bufs, dev_err=err)
+            self.prep()
 
         def step(self):
             """copy in, step, copy out, all on the current stream"""
@@ -651,7 +655,8 @@ def end_to_end(cases, spec, path, decode, rotate, tm, world, device, stream, err
         raise RuntimeError(f"device error bits {int(err.item())} in the end-to-end loop")
     del graph_e2e
     return {"value": e2e_eager, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "how": ("dsa.step called from Python every step, steps back to back over the independent batches; "
+            "how": ("the step issued from Python every step through dsa.PreparedStep (the step's library calls "
+                    "with their arguments marshalled once), steps back to back over the independent batches; "
                     "each step's inputs staged in one pinned buffer (one H2D copy) and out/lse read back from one "
                     "device buffer (one D2H copy), on the step's stream, inside the timed region"),
             "graph_value": e2e_graph,

@@ -37,8 +37,8 @@ __all__ = [
     "PagedKVCache", "SeqBatch", "QueryBatch", "DsaError", "load",
     "kv_append", "index_score", "topk_blocks", "select_blocks", "select_blocks_append", "sparse_attn_decode",
     "sparse_attn_prefill", "decode_fused", "decode_workspace_size", "select_workspace_size",
-    "decode_fused_workspace_size", "sparse_attn_decode_noalloc", "step", "index_score_i64", "index_score_fp8",
-    "topk_blocks_i64",
+    "decode_fused_workspace_size", "sparse_attn_decode_noalloc", "step", "PreparedStep", "index_score_i64",
+    "index_score_fp8", "topk_blocks_i64",
 ]
 
 BLOCK_SIZE = 64
@@ -390,6 +390,60 @@ def decode_fused(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, cu_ne
         q.shape[1], scale, _ptr(sel), _ptr(cnt), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
         _ptr(dev_err), _stream(stream)))
     return sel, cnt, out, lse
+
+
+class _Recorder:
+    """Stands in for the library while PreparedStep records a step: launches
+    are recorded with their marshalled arguments (and report success), size
+    and status queries go to the library."""
+
+    def __init__(self, lib):
+        self._real = lib
+        self.calls = []
+
+    def __getattr__(self, name):
+        real = getattr(self._real, name)
+        if name.endswith("_workspace_size") or name in ("dsa_status_string", "dsa_version"):
+            return real
+
+        def record(*args):
+            self.calls.append((name, real, args))
+            return _lib.DSA_OK
+        return record
+
+
+class PreparedStep:
+    """One pass of the hot path (the calls step() makes, same arguments) with
+    every argument marshalled once, for loops that run the same step on the
+    same buffers again and again (a serving loop, a benchmark).  Calling it
+    issues the library calls on ``stream`` (the stream given here, else the
+    current one) and returns the output buffers; the host cost per call is
+    the calls themselves.  The tensors passed here must stay allocated at the
+    same addresses while the object is used (it keeps references to them);
+    refill them in place between calls.  Not to be built while another thread
+    calls this module."""
+
+    def __init__(self, cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, *, bufs: Optional[dict] = None,
+                 stream=None, **step_kwargs):
+        global load
+        rec = _Recorder(_lib.load())
+        saved = load
+        load = lambda: rec   # noqa: E731 -- the binding's calls below go to the recorder
+        try:
+            self.bufs = step(cache, seqs, queries, bufs=bufs, **step_kwargs)
+        finally:
+            load = saved
+        self.calls = rec.calls
+        self._stream = None if stream is None else ctypes.c_void_p(stream.cuda_stream)
+        self._keep = (cache, seqs, queries, step_kwargs)
+
+    def __call__(self, stream=None):
+        s = _stream(stream) if (stream is not None or self._stream is None) else self._stream
+        for name, fn, args in self.calls:
+            rc = fn(*args[:-1], s)
+            if rc != _lib.DSA_OK:
+                _lib.check(name, rc)
+        return self.bufs
 
 
 def step(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, *, k_new, v_new, kc_new, q, q_idx, w,

@@ -36,6 +36,8 @@
 //     bytes on rank 0's inbox mbarrier (armed with the full count before the
 //     start-of-kernel cluster barrier); rank 0 combines and writes the output.
 // All waits are bounded (DSA_DEV_ERR_WAIT on timeout, no hang).
+#include <mutex>
+
 #include "dsa_kernels.h"
 #include "dsa_tma.cuh"
 #include "decode_fused.cuh"
@@ -836,7 +838,51 @@ struct AttnMaps {
     CUtensorMap k, v, q;
 };
 
+cudaError_t encode_maps(const AttnArgs &a, AttnMaps &m);
+
+// Encoded maps of the last few (pools, queries) a launch used: a decode loop
+// calls with the same buffers every step, and encoding three maps costs host
+// time on every call otherwise.  The key is everything the maps encode.
+struct MapKey {
+    int dev;
+    const void *k, *v, *q;
+    int num_pages, num_kv_heads, block_shift, total_q, num_q_heads;
+    bool operator==(const MapKey &o) const {
+        return dev == o.dev && k == o.k && v == o.v && q == o.q && num_pages == o.num_pages &&
+               num_kv_heads == o.num_kv_heads && block_shift == o.block_shift && total_q == o.total_q &&
+               num_q_heads == o.num_q_heads;
+    }
+};
+constexpr int kMapCache = 16;
+std::mutex g_map_mu;
+MapKey g_map_keys[kMapCache];
+AttnMaps g_map_vals[kMapCache];
+int g_map_n = 0, g_map_next = 0;
+
 cudaError_t make_maps(const AttnArgs &a, AttnMaps &m) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+    const MapKey key{dev, a.k_pool, a.v_pool, a.q, a.num_pages, a.num_kv_heads, a.block_shift, a.total_q,
+                     a.num_q_heads};
+    {
+        std::lock_guard<std::mutex> lock(g_map_mu);
+        for (int i = 0; i < g_map_n; ++i)
+            if (g_map_keys[i] == key) {
+                m = g_map_vals[i];
+                return cudaSuccess;
+            }
+    }
+    const cudaError_t e = encode_maps(a, m);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    g_map_keys[g_map_next] = key;
+    g_map_vals[g_map_next] = m;
+    g_map_next = (g_map_next + 1) % kMapCache;
+    if (g_map_n < kMapCache) ++g_map_n;
+    return cudaSuccess;
+}
+
+cudaError_t encode_maps(const AttnArgs &a, AttnMaps &m) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
     // K / V pool: dims (head_dim, kv_head, page*B+token), boxes of 64 dims x 1 head x 64 tokens (one tile)

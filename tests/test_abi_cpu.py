@@ -247,3 +247,51 @@ def test_wide_score_validation_codes():
     assert tk(k_max=65) == _lib.DSA_ERR_UNSUPPORTED
     assert tk(bs=48) == _lib.DSA_ERR_UNSUPPORTED
     assert tk(queries=_queries(total_q=0)) == _lib.DSA_OK
+
+
+def test_prepared_step_replays_the_calls_step_makes(monkeypatch):
+    """PreparedStep records the library calls of one step() with their
+    marshalled arguments and replays them; checked on the CPU with a fake
+    library that records calls (nothing is launched)."""
+    import torch
+
+    import dynamic_block_sparse_dsa_b200 as dsa
+    from dynamic_block_sparse_dsa_b200 import workloads as wk
+
+    class FakeLib:
+        def __init__(self):
+            self.log = []
+
+        def __getattr__(self, name):
+            if name.endswith("_workspace_size"):
+                return lambda *a: 256
+
+            def call(*args):
+                self.log.append((name, tuple(getattr(x, "value", x) if not hasattr(x, "_obj") else id(x._obj)
+                                             for x in args[:-1])))
+                return 0
+            return call
+
+    fake = FakeLib()
+    monkeypatch.setattr(dsa._lib, "load", lambda: fake)
+    monkeypatch.setattr(dsa, "load", lambda: fake)
+    monkeypatch.setattr(dsa, "_ptr", lambda t: None if t is None else ctypes.c_void_p(t.data_ptr()))
+    monkeypatch.setattr(dsa, "_stream", lambda s: ctypes.c_void_p(7))
+    spec = wk.WorkloadSpec("ps", seq_lens=(900, 300), n_new=(1, 1), k_per_seq=(4, 4), k_max=4, num_q_heads=8,
+                           num_kv_heads=1, num_idx_heads=4)
+    wl = wk.make_workload(spec, seed=3)
+    cache = dsa.PagedKVCache(wl.k_pool, wl.v_pool, wl.kc_pool)
+    seqs = dsa.SeqBatch(wl.block_table, wl.seq_lens)
+    queries = dsa.QueryBatch(wl.cu_q, wl.q_pos)
+    kw = dict(k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q, q_idx=wl.q_idx, w=wl.w,
+              k_per_seq=wl.k_per_seq, k_max=spec.k_max, fused_select=True, overlap_append=True)
+    bufs = dsa.step(cache, seqs, queries, **kw)
+    direct = [n for n, _ in fake.log]
+    fake.log.clear()
+    ps = dsa.PreparedStep(cache, seqs, queries, bufs=bufs, **kw)
+    assert fake.log == []                       # recording launches nothing
+    assert [c[0] for c in ps.calls] == direct == ["dsa_select_blocks_append", "dsa_sparse_attn_decode"]
+    for _ in range(2):
+        assert ps() is bufs
+    assert [n for n, _ in fake.log] == direct * 2
+    assert fake.log[0][1] == fake.log[2][1]     # same marshalled arguments every time

@@ -339,6 +339,30 @@ def test_repeat_calls_reuse_workspace(cuda_device):
     assert int(b["workspace"][:4 * spec.total_q * spec.num_kv_heads].view(torch.int32).abs().sum()) == 0
 
 
+@pytest.mark.parametrize("decode,fused,overlap", [(True, False, False), (True, True, True), (False, False, False),
+                                                   (False, True, False)])
+def test_prepared_step_matches_step(decode, fused, overlap, cuda_device):
+    # a step prepared once and issued again gives what step() gives, bit for bit
+    spec = _small_spec("ragged_prefill_tail", "sharp")
+    wl = wk.make_workload(spec, seed=12, device=cuda_device)
+    want, e = gpu_step(wl, decode=decode, fused=fused, overlap=overlap)
+    assert e == 0
+    want = {k: want[k].clone() for k in ("sel", "cnt", "out", "lse")}
+    cache, seqs, queries = _handles(wl)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    ps = dsa.PreparedStep(cache, seqs, queries, k_new=wl.k_new, v_new=wl.v_new, kc_new=wl.kc_new, q=wl.q,
+                          q_idx=wl.q_idx, w=wl.w, k_per_seq=wl.k_per_seq, k_max=spec.k_max, decode=decode,
+                          fused_select=fused or overlap, overlap_append=overlap, dev_err=err)
+    for _ in range(3):
+        for k in ("out", "lse"):
+            ps.bufs[k].fill_(float("nan"))
+        got = ps()
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        for k, v in want.items():
+            assert torch.equal(got[k], v), k
+
+
 # ----------------------------------------------------------------------------- device error flags
 @pytest.mark.parametrize("fused", [False, True])
 def test_bad_page_sets_flag_without_fault(fused, cuda_device):
