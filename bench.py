@@ -565,13 +565,17 @@ def end_to_end(cases, spec, path, decode, rotate, tm, world, device, stream, err
             self.bufs["lse"] = view(self.dev_out_buf, out_offs["lse"], c.bufs["lse"])
             self.c = c
             d = self.dev_in
+            kw = dict(bufs=self.bufs, k_new=d["k_new"], v_new=d["v_new"], kc_new=d["kc_new"], q=d["q"],
+                      q_idx=d["q_idx"], w=d["w"], k_per_seq=c.wl.k_per_seq, k_max=spec.k_max, decode=decode,
+                      fused_select=fused, overlap_append=fused and decode, fused_decode=fused_decode, dev_err=err)
             # the step's calls with their arguments marshalled once (the public
-            # PreparedStep: a serving loop's way of issuing the same step again)
-            self.prep = dsa.PreparedStep(c.cache, c.seqs, c.queries, bufs=self.bufs, k_new=d["k_new"],
-                                         v_new=d["v_new"], kc_new=d["kc_new"], q=d["q"], q_idx=d["q_idx"], w=d["w"],
-                                         k_per_seq=c.wl.k_per_seq, k_max=spec.k_max, decode=decode,
-                                         fused_select=fused, overlap_append=fused and decode,
-                                         fused_decode=fused_decode, dev_err=err)
+            # PreparedStep: a serving loop's way of issuing the same step
+            # again), once with the library's host staging of this batch's
+            # inputs and results (slot = the batch) and once bare, for capture
+            self.prep_staged = dsa.PreparedStep(c.cache, c.seqs, c.queries, stager=stager, slot=len(staged),
+                                                host_in=[(self.dev_in_buf, self.host_in)],
+                                                host_out=[(self.dev_out_buf, self.host_out)], **kw)
+            self.prep = dsa.PreparedStep(c.cache, c.seqs, c.queries, **kw)
             self.in_ready = torch.cuda.Event()   # graph only: this batch's inputs landed
             self.consumed = torch.cuda.Event()   # its step ran
             self.out_done = torch.cuda.Event()   # its outputs read back
@@ -580,16 +584,18 @@ def end_to_end(cases, spec, path, decode, rotate, tm, world, device, stream, err
             self.prep()
 
         def step(self):
-            """copy in, step, copy out, all on the current stream"""
-            self.dev_in_buf.copy_(self.host_in, non_blocking=True)
-            self.compute()
-            self.host_out.copy_(self.dev_out_buf, non_blocking=True)
+            """copy in, step, copy out: the copies on the stager's streams, the
+            step on `stream`"""
+            self.prep_staged()
 
-    staged = [Staged(c) for c in cases]
+    stager = dsa.Stager(n_case, stream)
+    staged = []
+    for c in cases:
+        staged.append(Staged(c))
     h2d, d2h = staged[0].in_bytes, staged[0].out_bytes
     for st in staged:   # first use outside any capture
-        with torch.cuda.stream(stream):
-            st.step()
+        st.step()
+    stager.join()
     torch.cuda.synchronize(device)
     # the graph: all of a rotation's input copies on one side stream, its steps
     # on the main stream, each step's read-back on another side stream as soon
@@ -624,9 +630,10 @@ def end_to_end(cases, spec, path, decode, rotate, tm, world, device, stream, err
             with torch.cuda.stream(stream):
                 e_s.record()
             if eager:
-                with torch.cuda.stream(stream):
-                    for i in range(n_e2e):
-                        staged[i % n_case].step()
+                e_s.synchronize()   # as below: the copy streams do not wait for `stream`
+                for i in range(n_e2e):
+                    staged[i % n_case].step()
+                stager.join()
             else:
                 with torch.cuda.stream(stream):
                     for i in range(n_e2e // n_case):
@@ -641,7 +648,14 @@ def end_to_end(cases, spec, path, decode, rotate, tm, world, device, stream, err
                 with torch.cuda.stream(stream):
                     tm.cold_l2()
                     e_s.record()
-                    staged[0].step() if eager else graph_e2e.replay()
+                    if eager:
+                        # the copy streams do not wait for `stream`: let the flush
+                        # and the start event pass before the input copy is issued
+                        e_s.synchronize()
+                        staged[0].step()
+                        stager.join()
+                    else:
+                        graph_e2e.replay()
                     e_e.record()
                 stream.synchronize()
                 total += e_s.elapsed_time(e_e) / 1e3
@@ -654,11 +668,14 @@ def end_to_end(cases, spec, path, decode, rotate, tm, world, device, stream, err
     if int(err.item()) != 0:
         raise RuntimeError(f"device error bits {int(err.item())} in the end-to-end loop")
     del graph_e2e
+    stager.close()
     return {"value": e2e_eager, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "how": ("the step issued from Python every step through dsa.PreparedStep (the step's library calls "
-                    "with their arguments marshalled once), steps back to back over the independent batches; "
-                    "each step's inputs staged in one pinned buffer (one H2D copy) and out/lse read back from one "
-                    "device buffer (one D2H copy), on the step's stream, inside the timed region"),
+                    "with their arguments marshalled once) with the library's host staging (dsa_stager): each "
+                    "step's inputs copied from one pinned buffer (one H2D copy) and out/lse read back into one "
+                    "(one D2H copy) on the library's two copy streams, so one batch's copies overlap the other "
+                    "batches' kernels; steps back to back over the independent batches, every copy inside the "
+                    "timed region"),
             "graph_value": e2e_graph,
             "graph_how": ("the same copies and calls captured once per rotation in a CUDA graph whose input copies "
                           "and read-backs run on side streams, overlapping the other batches' steps; replayed")}

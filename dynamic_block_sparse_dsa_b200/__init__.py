@@ -37,7 +37,7 @@ __all__ = [
     "PagedKVCache", "SeqBatch", "QueryBatch", "DsaError", "load",
     "kv_append", "index_score", "topk_blocks", "select_blocks", "select_blocks_append", "sparse_attn_decode",
     "sparse_attn_prefill", "decode_fused", "decode_workspace_size", "select_workspace_size",
-    "decode_fused_workspace_size", "sparse_attn_decode_noalloc", "step", "PreparedStep", "index_score_i64",
+    "decode_fused_workspace_size", "sparse_attn_decode_noalloc", "step", "PreparedStep", "Stager", "index_score_i64",
     "index_score_fp8", "topk_blocks_i64",
 ]
 
@@ -412,6 +412,62 @@ class _Recorder:
         return record
 
 
+def _host_ptr(t: torch.Tensor) -> int:
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("host staging buffers must be contiguous CPU tensors (pinned for asynchronous copies)")
+    return t.data_ptr()
+
+
+def _regions(pairs, host_first: bool):
+    """(dst array, src array, bytes array, n) of (device, host) tensor pairs."""
+    n = len(pairs)
+    dst, src, nb = (ctypes.c_void_p * max(n, 1))(), (ctypes.c_void_p * max(n, 1))(), (ctypes.c_size_t * max(n, 1))()
+    for i, (dev_t, host_t) in enumerate(pairs):
+        if dev_t.numel() * dev_t.element_size() != host_t.numel() * host_t.element_size():
+            raise ValueError("a staged device tensor and its host buffer differ in size")
+        d, h = _ptr(dev_t).value, _host_ptr(host_t)
+        dst[i], src[i] = (h, d) if host_first else (d, h)
+        nb[i] = dev_t.numel() * dev_t.element_size()
+    return dst, src, nb, n
+
+
+class Stager:
+    """Host staging of repeated steps (the library's dsa_stager): inputs copied
+    from pinned host memory and results copied back on two copy streams of the
+    library's own, so one batch's copies overlap the other batches' kernels.
+    ``num_slots`` batches, each with its own device buffers; ``stream`` is the
+    compute stream the steps run on (default: the current stream)."""
+
+    def __init__(self, num_slots: int, stream=None):
+        self._lib = load()
+        self.stream = torch.cuda.current_stream() if stream is None else stream
+        self._s = ctypes.c_void_p(self.stream.cuda_stream)
+        h = ctypes.c_void_p()
+        _lib.check("dsa_stager_create", self._lib.dsa_stager_create(num_slots, self._s, ctypes.byref(h)))
+        self._h = h
+        self.num_slots = num_slots
+
+    def wait(self, slot: int) -> None:
+        """Block until the slot's last read-back has landed."""
+        _lib.check("dsa_stager_wait", self._lib.dsa_stager_wait(self._h, slot))
+
+    def join(self) -> None:
+        """Make the compute stream wait for every copy issued so far."""
+        _lib.check("dsa_stager_join", self._lib.dsa_stager_join(self._h))
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            rc = self._lib.dsa_stager_destroy(self._h)
+            self._h = None
+            _lib.check("dsa_stager_destroy", rc)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
 class PreparedStep:
     """One pass of the hot path (the calls step() makes, same arguments) with
     every argument marshalled once, for loops that run the same step on the
@@ -421,10 +477,18 @@ class PreparedStep:
     the calls themselves.  The tensors passed here must stay allocated at the
     same addresses while the object is used (it keeps references to them);
     refill them in place between calls.  Not to be built while another thread
-    calls this module."""
+    calls this module.
+
+    With a ``stager`` (a Stager) the step also stages its own host data on it
+    as slot ``slot``: every call first copies ``host_in`` -- (device tensor,
+    pinned host tensor) pairs -- to the device and ends by copying
+    ``host_out`` -- (device tensor, pinned host tensor) pairs -- back, and the
+    step runs on the stager's stream.  ``stager.wait(slot)`` tells when the
+    host buffers may be read (results) and rewritten (inputs)."""
 
     def __init__(self, cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, *, bufs: Optional[dict] = None,
-                 stream=None, **step_kwargs):
+                 stream=None, stager: Optional[Stager] = None, slot: int = 0, host_in=(), host_out=(),
+                 **step_kwargs):
         global load
         rec = _Recorder(_lib.load())
         saved = load
@@ -434,16 +498,41 @@ class PreparedStep:
         finally:
             load = saved
         self.calls = rec.calls
+        if stager is not None:
+            if not 0 <= slot < stager.num_slots:
+                raise ValueError(f"slot {slot} outside the stager's {stager.num_slots} slots")
+            stream = stager.stream
+            lib = _lib.load()
+            self._begin = (lib.dsa_stager_begin, (stager._h, slot, *_rotate(_regions(host_in, False))))
+            self._end = (lib.dsa_stager_end, (stager._h, slot, *_rotate(_regions(host_out, True))))
+        elif host_in or host_out:
+            raise ValueError("host_in / host_out need a stager")
+        else:
+            self._begin = self._end = None
         self._stream = None if stream is None else ctypes.c_void_p(stream.cuda_stream)
-        self._keep = (cache, seqs, queries, step_kwargs)
+        self._keep = (cache, seqs, queries, step_kwargs, stager, tuple(host_in), tuple(host_out))
 
     def __call__(self, stream=None):
+        if self._begin is not None:
+            if stream is not None:
+                raise ValueError("a staged step runs on its stager's stream")
+            fn, args = self._begin
+            _lib.check("dsa_stager_begin", fn(*args))
         s = _stream(stream) if (stream is not None or self._stream is None) else self._stream
         for name, fn, args in self.calls:
             rc = fn(*args[:-1], s)
             if rc != _lib.DSA_OK:
                 _lib.check(name, rc)
+        if self._end is not None:
+            fn, args = self._end
+            _lib.check("dsa_stager_end", fn(*args))
         return self.bufs
+
+
+def _rotate(r):
+    """(dst, src, bytes, n) -> (n, dst, src, bytes): the C argument order."""
+    dst, src, nb, n = r
+    return n, dst, src, nb
 
 
 def step(cache: PagedKVCache, seqs: SeqBatch, queries: QueryBatch, *, k_new, v_new, kc_new, q, q_idx, w,

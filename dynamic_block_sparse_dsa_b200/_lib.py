@@ -63,6 +63,12 @@ SIGNATURES = {
     "dsa_decode_fused": ([P(KvCacheC), P(SeqsC), P(QueriesC), c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32,
                           c_i32, c_vp, c_i32, c_vp, c_i32, ctypes.c_float, c_vp, c_vp, c_vp, c_vp, c_vp,
                           ctypes.c_size_t, c_vp, c_vp], c_i32),
+    "dsa_stager_create": ([c_i32, c_vp, P(c_vp)], c_i32),
+    "dsa_stager_destroy": ([c_vp], c_i32),
+    "dsa_stager_begin": ([c_vp, c_i32, c_i32, c_vp, c_vp, c_vp], c_i32),
+    "dsa_stager_end": ([c_vp, c_i32, c_i32, c_vp, c_vp, c_vp], c_i32),
+    "dsa_stager_wait": ([c_vp, c_i32], c_i32),
+    "dsa_stager_join": ([c_vp], c_i32),
     "dsa_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "dsa_version": ([], ctypes.c_int),
 }

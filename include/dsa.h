@@ -344,6 +344,57 @@ int dsa_sparse_attn_decode_noalloc(const dsa_kv_cache *cache, const dsa_seqs *se
                                    float sm_scale, void *out, float *lse, int32_t *dev_err,
                                    dsa_stream_t stream);
 
+/*
+ * Host staging of repeated steps.  The pages have no counterpart to this
+ * part: it is runtime plumbing for a loop that issues one step per batch from
+ * the host, each step's inputs in pinned host memory and its results wanted
+ * back on the host.  A stager owns two copy streams (created at
+ * dsa_stager_create, on the device current then) and one set of events per
+ * slot; a slot is one batch whose device buffers are reused step after step.
+ * The copies of one slot overlap the kernels of the other slots' steps while
+ * each step still sees its own inputs and leaves its own results:
+ *
+ *   dsa_stager_begin(st, slot, ...)   inputs host -> device
+ *   <the step's library calls on the stager's stream>
+ *   dsa_stager_end(st, slot, ...)     results device -> host
+ *
+ *  - dsa_stager_create: num_slots in 1..4096; `stream` is the compute stream
+ *    the steps are issued on (the stager does not own it).  *out receives the
+ *    handle.  DSA_ERR_CUDA if a stream or event cannot be created.
+ *  - dsa_stager_begin: n regions (0..64), region i copies bytes[i] bytes from
+ *    host_src[i] to dev_dst[i] (cudaMemcpyAsync; asynchronous only if the
+ *    host memory is pinned).  The copies wait until the slot's previous step
+ *    (the calls between its previous begin and end) has run, since that step
+ *    reads those device buffers; then the compute stream waits for them and
+ *    for the slot's previous read-back.  Any other reader or writer of those
+ *    buffers must be ordered by the caller.  The host must not rewrite
+ *    host_src before the copies have landed (dsa_stager_wait on the slot
+ *    covers it).
+ *  - dsa_stager_end: after the step's calls; region i copies bytes[i] bytes
+ *    from dev_src[i] to host_dst[i] once the step has run.
+ *  - dsa_stager_wait: blocks the host until the slot's last read-back has
+ *    landed.  dsa_stager_join: makes the compute stream wait for every copy
+ *    issued so far (before an event or a synchronisation on that stream).
+ *  - dsa_stager_destroy: waits for the copy streams, then frees everything
+ *    (NULL is a no-op).
+ *  - Errors: DSA_ERR_INVALID_ARG for a NULL handle, a slot outside
+ *    [0, num_slots), n outside 0..64 or a NULL pointer of a non-empty
+ *    region (nothing is issued); DSA_ERR_CUDA when a CUDA call fails.
+ *  - Call with the device of create current; not under stream capture (a
+ *    graph captures the plain calls and torch-side copies instead); one
+ *    thread at a time per stager.
+ */
+typedef struct dsa_stager dsa_stager;
+
+int dsa_stager_create(int32_t num_slots, dsa_stream_t stream, dsa_stager **out);
+int dsa_stager_destroy(dsa_stager *st);
+int dsa_stager_begin(dsa_stager *st, int32_t slot, int32_t n, void *const *dev_dst, const void *const *host_src,
+                     const size_t *bytes);
+int dsa_stager_end(dsa_stager *st, int32_t slot, int32_t n, void *const *host_dst, const void *const *dev_src,
+                   const size_t *bytes);
+int dsa_stager_wait(dsa_stager *st, int32_t slot);
+int dsa_stager_join(dsa_stager *st);
+
 /* human-readable name of a status code (static string) */
 const char *dsa_status_string(int status);
 

@@ -295,3 +295,27 @@ def test_prepared_step_replays_the_calls_step_makes(monkeypatch):
         assert ps() is bufs
     assert [n for n, _ in fake.log] == direct * 2
     assert fake.log[0][1] == fake.log[2][1]     # same marshalled arguments every time
+
+
+def test_stager_validates_on_the_host():
+    lib = _lib.load()
+    h = ctypes.c_void_p()
+    assert lib.dsa_stager_create(0, None, ctypes.byref(h)) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_stager_create(4097, None, ctypes.byref(h)) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_stager_create(2, None, None) == _lib.DSA_ERR_INVALID_ARG
+    arr = (ctypes.c_void_p * 1)(FAKE)
+    nb = (ctypes.c_size_t * 1)(16)
+    for fn in (lib.dsa_stager_begin, lib.dsa_stager_end):
+        assert fn(None, 0, 1, arr, arr, nb) == _lib.DSA_ERR_INVALID_ARG
+        assert fn(None, 0, 0, None, None, None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_stager_wait(None, 0) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_stager_join(None) == _lib.DSA_ERR_INVALID_ARG
+    assert lib.dsa_stager_destroy(None) == _lib.DSA_OK
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except Exception:
+        has_gpu = False
+    if not has_gpu:   # without a device the streams cannot be made: a CUDA error, no handle
+        assert lib.dsa_stager_create(2, None, ctypes.byref(h)) == _lib.DSA_ERR_CUDA
+        assert not h.value

@@ -343,7 +343,8 @@ def test_repeat_calls_reuse_workspace(cuda_device):
                                                    (False, True, False)])
 def test_prepared_step_matches_step(decode, fused, overlap, cuda_device):
     # a step prepared once and issued again gives what step() gives, bit for bit
-    spec = _small_spec("ragged_prefill_tail", "sharp")
+    # (the appending selection takes decode batches only: one query per sequence)
+    spec = _small_spec("many_seqs_decode" if overlap else "ragged_prefill_tail", "sharp")
     wl = wk.make_workload(spec, seed=12, device=cuda_device)
     want, e = gpu_step(wl, decode=decode, fused=fused, overlap=overlap)
     assert e == 0
