@@ -102,6 +102,7 @@ void attn_schedule(AttnArgs &a, bool allow_split, bool allow_cluster = false) {
     long long C = sm_count();
     if (C > kAttnMaxCtas) C = kAttnMaxCtas;
     a.cluster2 = 0;
+    a.interleave = 0;
     // between a quarter and a half as many pairs as SMs: one 2-CTA cluster per
     // pair keeps at least half of the SMs streaming and merges on chip
     if (allow_cluster && allow_split && (a.k_max << a.tile_shift) >= 2 && 4 * pairs >= C && 2 * pairs <= C) {
@@ -118,6 +119,11 @@ void attn_schedule(AttnArgs &a, bool allow_split, bool allow_cluster = false) {
     // a pair may be split over at most ~60 CTAs (the kernel merges <= 63 partials)
     if (C > pairs * 60) C = pairs * 60;
     a.num_ctas = (int)C;
+    // whole pairs: KV-head-major and interleaved over the CTAs (a query's
+    // selected blocks are scattered over the pool, so the queries running at
+    // one time share blocks only through L2, and one KV head's slice of the
+    // pool fits there where the whole pool often does not)
+    a.interleave = (a.pair_aligned && a.num_kv_heads > 1) ? 1 : 0;
 }
 
 int attn_common(const dsa_kv_cache *cache, const dsa_seqs *seqs, const dsa_queries *queries,

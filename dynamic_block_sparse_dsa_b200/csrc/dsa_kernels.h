@@ -141,6 +141,10 @@ struct AttnArgs {
     long long total_units;   // U
     int num_ctas;            // C (= gridDim.x)
     int pair_aligned;
+    // with pair_aligned: CTA c runs instead the pairs r = c, c + C, c + 2C, ...
+    // of the KV-head-major order r = kvh * T + t, so that all CTAs work on
+    // the same KV head at a time and its blocks are re-read from L2
+    int interleave;
     // 1: pair p is run by the 2-CTA cluster (2p, 2p+1), each CTA taking half
     // of its units; the halves merge through distributed shared memory and
     // no workspace is touched

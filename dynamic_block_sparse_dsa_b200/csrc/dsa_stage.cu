@@ -17,7 +17,7 @@
 
 #include <new>
 
-#include "../../include/dsa.h"
+#include "dsa.h"
 
 struct dsa_stager {
     int device;

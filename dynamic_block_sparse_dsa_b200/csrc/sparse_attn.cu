@@ -166,6 +166,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         const unit_t h0 = (K + 1) / 2;
         u0 = p0 + ((c & 1) ? h0 : 0);
         u1 = p0 + ((c & 1) ? K : h0);
+    } else if (!kFused && a.interleave) {
+        // pairs c, c + C, c + 2C, ... of the KV-head-major order: local pair i
+        // of this CTA is r = i * C + c (r = kvh * T + t)
+        const unit_t P = (unit_t)a.total_q * (unit_t)a.num_kv_heads, C = (unit_t)a.num_ctas;
+        u0 = 0;
+        u1 = ((unit_t)c < P ? (P - 1 - (unit_t)c) / C + 1 : 0) * K;
     } else {
         u0 = range_begin(a, c);
         u1 = range_begin(a, c + 1);
@@ -256,8 +262,14 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 const unit_t pair = uu / K;
                 const int ju = (int)(uu - pair * K);
                 const int j = ju >> a.tile_shift, sub = ju & ((1 << a.tile_shift) - 1);
-                t = (int)(pair / Hkv);
-                kvh = (int)(pair - (unit_t)t * Hkv);
+                if (!kFused && a.interleave) {
+                    const unit_t r = pair * (unit_t)a.num_ctas + (unit_t)c;
+                    kvh = (int)(r / (unit_t)a.total_q);
+                    t = (int)(r - (unit_t)kvh * (unit_t)a.total_q);
+                } else {
+                    t = (int)(pair / Hkv);
+                    kvh = (int)(pair - (unit_t)t * Hkv);
+                }
                 s = seq_of(a, s_cuq, t);
                 p = __ldg(a.q_pos + t);
                 const int len = __ldg(a.seq_lens + s);
