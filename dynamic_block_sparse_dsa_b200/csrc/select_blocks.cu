@@ -10,19 +10,20 @@
 //
 // Grid: (query, chunk of 512*G candidate blocks).  Each CTA scores its chunk
 // with the int8 indexer on the tensor cores (mma.m16n8k32 s8, coarse keys as
-// the M operand loaded straight into fragments, 64 blocks per warp step; a
-// CUDA-core dp4a version measured ALU-bound at the 1M-token decode shape),
-// keeps the chunk's local Top-(K-1)
-// (warp-level bitonic Top-64 on unique 64-bit keys, then a merge tree over
-// the warps) and writes it to the workspace.  The last CTA of the query --
-// elected with an atomic counter, nothing waits -- merges the chunks' sorted
-// lists the same way, appends the query's own block and writes the ascending
-// selection.  Result is identical to dsa_index_score followed by
+// the M operand loaded straight into fragments, 64 blocks per warp step, the
+// warps' groups interleaved; a CUDA-core dp4a version measured ALU-bound at
+// the 1M-token decode shape), keeps every candidate as a unique 64-bit key in
+// registers and finds the chunk's Top-(K-1) with a CTA-wide radix select
+// (radix_select.cuh), which it writes to the workspace.  The last CTA of the
+// query -- elected with an atomic counter, nothing waits -- selects again
+// over the chunks' lists, appends the query's own block and writes the
+// ascending selection.  Result is identical to dsa_index_score followed by
 // dsa_topk_blocks.
 #include "dsa_kernels.h"
 #include "dsa_tma.cuh"
 #include "indexer_core.cuh"
 #include "kv_append.cuh"
+#include "radix_select.cuh"
 #include "warp_topk.cuh"
 
 namespace dsa {
@@ -35,12 +36,13 @@ constexpr long long kSelBusyCtas = 8 * 148;   // a grid this large keeps every S
 }  // namespace
 
 template <int G>   // 64-block groups per warp: a chunk is kSelWarps * 64 * G blocks
-__global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(kSelThreads, 2) select_blocks_kernel(SelectArgs a) {
     __shared__ int4 s_q[kMaxIdxHeads][kIdxDim / 16];
     __shared__ int s_w[kMaxIdxHeads];
     __shared__ int s_cuq[kCuqCache + 1];
-    __shared__ key64 s_lists[kSelWarps * 64];
-    __shared__ int s_last;
+    __shared__ RadixScratch s_rx;
+    __shared__ uint32_t s_ids[kSelMaxK];
+    __shared__ int s_last, s_nsel[2];
     constexpr int CH = kSelWarps * 64 * G;
     const int t = blockIdx.x, c = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, cq = lane & 3;
@@ -69,7 +71,7 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
         // page ids of this warp's first group, before the facts are checked
         // (rows end at max_blocks; ids past the own block are never used)
         const int32_t *row = a.block_table + (size_t)sq * a.max_blocks;
-        const int base = c * CH + (warp * G) * 64;
+        const int base = c * CH + warp * 64;
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
@@ -86,6 +88,7 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
         s_q[e >> 2][e & 3] = (e >> 2) < H
             ? __ldg(reinterpret_cast<const int4 *>(a.q_idx + (size_t)t * H * kIdxDim) + e) : make_int4(0, 0, 0, 0);
     if (tid < kMaxIdxHeads) s_w[tid] = tid < H ? __ldg(a.w + (size_t)t * H + tid) : 0;
+    if (tid < 2) s_nsel[tid] = 0;
     __syncthreads();
     int s;
     if (cached) {
@@ -149,11 +152,12 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
             wl[nt][1] = s_w[8 * nt + 2 * cq + 1];
         }
     }
-    key64 acc[2] = {0ull, 0ull};
+    // this thread's candidates: per group, blocks 16cq+g and 16cq+g+8 of it
+    key64 keys[2 * G];
     uint32_t err_bits = 0;
-#pragma unroll 1
+#pragma unroll
     for (int gi = 0; gi < G; ++gi) {
-        const int base = c * CH + (warp * G + gi) * 64;
+        const int base = c * CH + (gi * kSelWarps + warp) * 64;
         key64 v[2] = {0ull, 0ull};
         if (base < own) {
             // all of the group's page ids, then all of its coarse-key fragments,
@@ -185,29 +189,26 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
         } else if (gi == 0) {
             pdl_wait();
         }
-        if (gi == 0) {   // the first group: sorted, it is the warp's list (nothing to merge with)
-            warp_sort64_desc(v);
-            acc[0] = v[0];
-            acc[1] = v[1];
-        } else {
-            warp_fold_topk(acc, v, kk);
-        }
+        keys[2 * gi] = v[0];
+        keys[2 * gi + 1] = v[1];
     }
     if (err_bits) set_err(a.dev_err, err_bits);
 
-    // ---- chunk Top-64 over the warps (the query's Top-64 when it has one chunk)
-    cta_merge_top64<kSelWarps>(acc, s_lists);
+    // ---- the chunk's Top-(K-1) (the query's, when it has one chunk)
+    key64 prefix, mask;
+    const int n_real = cta_radix_threshold<kSelThreads, 2 * G>(keys, (uint32_t)kk, s_rx, prefix, mask);
     if (n_chunks > 1) {
-        // kept sorted in the workspace
+        // to the workspace, in any order; slots past the chunk's winners are zeroed
         key64 *cand = a.cand + ((size_t)t * kSelMaxChunks + c) * (kSelMaxK - 1);
-        if (warp == 0) {
-            if (lane < kk) cand[lane] = acc[0];
-            if (32 + lane < kk) cand[32 + lane] = acc[1];
-        }
-        // ---- the last chunk CTA of this query merges the chunks' lists: the
-        // barrier orders warp 0's list stores before tid 0's release-add, and
-        // the last adder's acquire (then the barrier) orders every list before
-        // the loads below
+        const int n_win = min(n_real, kk);
+#pragma unroll
+        for (int i = 0; i < 2 * G; ++i)
+            if (keys[i] != 0ull && (keys[i] & mask) >= prefix) cand[atomicAdd(&s_nsel[0], 1)] = keys[i];
+        for (int i = n_win + tid; i < kk; i += kSelThreads) cand[i] = 0ull;
+        // ---- the last chunk CTA of this query selects over the chunks'
+        // lists: the barrier orders every list store before tid 0's
+        // release-add, and the last adder's acquire (then the barrier) orders
+        // every list before the loads below
         __syncthreads();
         if (tid == 0) {
             const int old = atomic_add_acq_rel_gpu(a.counters + t, 1);
@@ -215,31 +216,34 @@ __global__ void __launch_bounds__(kSelThreads) select_blocks_kernel(SelectArgs a
         }
         __syncthreads();
         if (!s_last) return;
-        constexpr int kPer = (kSelMaxChunks + kSelWarps - 1) / kSelWarps;   // lists per warp
-        key64 lists[kPer][2];
+        constexpr int kLoad = (kSelMaxChunks * (kSelMaxK - 1) + kSelThreads - 1) / kSelThreads;
+        key64 lk[kLoad];
+        const int n_slots = n_chunks * kk;
 #pragma unroll
-        for (int k = 0; k < kPer; ++k) {   // every load in flight before the first merge
-            const int ci = warp + k * kSelWarps;
-            const key64 *src = a.cand + ((size_t)t * kSelMaxChunks + ci) * (kSelMaxK - 1);
-            const bool in = ci < n_chunks;
-            lists[k][0] = in && lane < kk ? __ldcg(src + lane) : 0ull;
-            lists[k][1] = in && 32 + lane < kk ? __ldcg(src + 32 + lane) : 0ull;
+        for (int j = 0; j < kLoad; ++j) {   // every load in flight before the selection
+            const int e = tid + j * kSelThreads;
+            const int ci = e / kk, ei = e - ci * kk;
+            lk[j] = e < n_slots ? __ldcg(a.cand + ((size_t)t * kSelMaxChunks + ci) * (kSelMaxK - 1) + ei) : 0ull;
         }
-        acc[0] = lists[0][0];
-        acc[1] = lists[0][1];
+        cta_radix_threshold<kSelThreads, kLoad>(lk, (uint32_t)kk, s_rx, prefix, mask);
 #pragma unroll
-        for (int k = 1; k < kPer; ++k)
-            if (warp + k * kSelWarps < n_chunks) warp_merge64_desc(acc, lists[k]);
-        cta_merge_top64<kSelWarps>(acc, s_lists);
+        for (int j = 0; j < kLoad; ++j)
+            if (lk[j] != 0ull && (lk[j] & mask) >= prefix) s_ids[atomicAdd(&s_nsel[1], 1)] = key64_id(lk[j]);
+        __syncthreads();
+    } else {
+#pragma unroll
+        for (int i = 0; i < 2 * G; ++i)
+            if (keys[i] != 0ull && (keys[i] & mask) >= prefix) s_ids[atomicAdd(&s_nsel[1], 1)] = key64_id(keys[i]);
+        __syncthreads();
     }
     if (warp == 0) {
-        // the winners (non-zero keys among the first kk) in ascending block order
-        const bool v0 = lane < kk && acc[0] != 0ull, v1 = 32 + lane < kk && acc[1] != 0ull;
-        const int km = __popc(__ballot_sync(0xffffffffu, v0)) + __popc(__ballot_sync(0xffffffffu, v1));
-        uint32_t ids[2] = {v0 ? key64_id(acc[0]) : 0xffffffffu, v1 ? key64_id(acc[1]) : 0xffffffffu};
+        // the winners in ascending block order
+        const int km = s_nsel[1];   // min(kk, candidates with a valid page)
+        uint32_t ids[2] = {lane < km ? s_ids[lane] : 0xffffffffu, 32 + lane < km ? s_ids[32 + lane] : 0xffffffffu};
         warp_sort64_asc_u32(ids);
-        if (lane < km) out[lane] = (int32_t)ids[0];
-        if (32 + lane < km) out[32 + lane] = (int32_t)ids[1];
+        const bool v0 = lane < km, v1 = 32 + lane < km;
+        if (v0) out[lane] = (int32_t)ids[0];
+        if (v1) out[32 + lane] = (int32_t)ids[1];
         if (lane == 0) {
             out[km] = own;              // the own block: the largest visible id, last in order
             a.cnt[t] = km + 1;
