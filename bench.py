@@ -108,7 +108,7 @@ class ClockSampler:
     }
 
     def __init__(self, device_index: int, period_s: float = 0.0002):
-        self.samples, self.reasons = [], set()
+        self.samples, self.reasons, self.stamps = [], set(), []
         self.max_mhz = None
         self._stop = threading.Event()
         self._thr = None
@@ -127,6 +127,7 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.stamps.append(time.monotonic())
                 r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
                 for bit, name in self.REASONS.items():
                     if r & bit:
@@ -152,6 +153,9 @@ class ClockSampler:
         if self._thr is not None:
             self._thr.join()
             sys.setswitchinterval(self._switch)
+
+    def count_between(self, t0: float, t1: float) -> int:
+        return sum(1 for t in list(self.stamps) if t0 <= t <= t1)
 
     def summary(self):
         if not self.samples:
@@ -432,12 +436,14 @@ def run_ours(args, world, rank, device):
     barrier(world)
     torch.cuda.synchronize(device)
     with ClockSampler(device.index if device.index is not None else 0) as clk:
+        time.sleep(0.002)   # the sampler's first samples, before the timed region
+        t_begin = time.monotonic()
         if rotate:
             total_s = tm.rotated(rot_graph, steps_g, args.steps)
         else:
             total_s = sum(tm.isolated(case0.graph, case0.ev, args.steps)) / 1e3
         torch.cuda.synchronize(device)
-        n_timed_samples = len(clk.samples)
+        n_timed_samples = clk.count_between(t_begin, time.monotonic())
         # the same steps again, untimed, so that the clock record has more than
         # a handful of samples of the load the timed region ran under
         if rotate:

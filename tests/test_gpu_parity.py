@@ -23,7 +23,7 @@ import torch
 
 import dynamic_block_sparse_dsa_b200 as dsa
 from dynamic_block_sparse_dsa_b200 import workloads as wk
-from oracle.harness import oracle_step
+from oracle.harness import oracle_select, oracle_step
 
 pytestmark = pytest.mark.gpu
 
@@ -652,3 +652,37 @@ def test_select_append_1m_workload(profile, cuda_device):
     bufs, err = gpu_step(wl, overlap=True)
     assert err == 0
     compare(wl, ref, bufs, fused=True)
+
+
+# ----------------------------------------------------------------------------- many-query selection, every query
+@pytest.mark.parametrize("variant", ["plain", "ties", "signed"])
+@pytest.mark.parametrize("prefix", [58_000, 128_000], ids=["two_groups_per_warp", "four_groups_per_warp"])
+def test_fused_selection_many_queries_every_query(prefix, variant, cuda_device):
+    # 1200 queries of two sequences with about 900 (or 2000) visible blocks:
+    # the fused selection runs one CTA per query with two (four) 64-block
+    # groups per warp, the radix-select path; the separate score + Top-K calls
+    # run the radix Top-K.  Every query's selection against the oracle, bit for
+    # bit, on the pool as generated (no append).  "ties": the pool holds only
+    # four distinct coarse keys (page p gets key p % 4), so every query's
+    # threshold falls inside a group of hundreds of equal scores and the
+    # lowest ids must win, and every third query has all-zero weights (every
+    # score 0).  "signed": weights drawn from [-16, 16].
+    spec = wk.WorkloadSpec("many_query_select", seq_lens=(prefix + 600, prefix - 1000), n_new=(600, 600),
+                           k_per_seq=(16, 9), k_max=16, num_q_heads=8, num_kv_heads=1, num_idx_heads=16,
+                           w_min=-16 if variant == "signed" else 0)
+    wl = wk.make_workload(spec, seed=91, device=cuda_device)
+    if variant == "ties":
+        keys4 = wl.kc_pool[:4].clone()
+        wl.kc_pool.copy_(keys4[torch.arange(wl.kc_pool.shape[0], device=cuda_device) % 4])
+        wl.w[::3] = 0
+    cache, seqs, queries = _handles(wl)
+    ref = oracle_select(wl)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    sel, cnt = dsa.select_blocks(cache, seqs, queries, wl.q_idx, wl.w, wl.k_per_seq, spec.k_max, dev_err=err)
+    scores = dsa.index_score(cache, seqs, queries, wl.q_idx, wl.w, dev_err=err)
+    sel2, cnt2 = dsa.topk_blocks(seqs, queries, scores, wl.k_per_seq, spec.k_max, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for s_, c_ in ((sel, cnt), (sel2, cnt2)):
+        assert np.array_equal(c_.cpu().numpy(), ref["cnt"])
+        assert np.array_equal(s_.cpu().numpy(), ref["sel"])
