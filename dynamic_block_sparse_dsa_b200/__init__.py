@@ -503,11 +503,13 @@ class PreparedStep:
                 raise ValueError(f"slot {slot} outside the stager's {stager.num_slots} slots")
             stream = stager.stream
             lib = _lib.load()
+            self._stager = stager
             self._begin = (lib.dsa_stager_begin, (stager._h, slot, *_rotate(_regions(host_in, False))))
             self._end = (lib.dsa_stager_end, (stager._h, slot, *_rotate(_regions(host_out, True))))
         elif host_in or host_out:
             raise ValueError("host_in / host_out need a stager")
         else:
+            self._stager = None
             self._begin = self._end = None
         self._stream = None if stream is None else ctypes.c_void_p(stream.cuda_stream)
         self._keep = (cache, seqs, queries, step_kwargs, stager, tuple(host_in), tuple(host_out))
@@ -516,6 +518,8 @@ class PreparedStep:
         if self._begin is not None:
             if stream is not None:
                 raise ValueError("a staged step runs on its stager's stream")
+            if not self._stager._h:
+                raise ValueError("the step's stager has been closed")
             fn, args = self._begin
             _lib.check("dsa_stager_begin", fn(*args))
         s = _stream(stream) if (stream is not None or self._stream is None) else self._stream

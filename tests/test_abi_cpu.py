@@ -319,3 +319,42 @@ def test_stager_validates_on_the_host():
     if not has_gpu:   # without a device the streams cannot be made: a CUDA error, no handle
         assert lib.dsa_stager_create(2, None, ctypes.byref(h)) == _lib.DSA_ERR_CUDA
         assert not h.value
+
+
+def test_prepared_step_refuses_a_closed_stager(monkeypatch):
+    """A staged PreparedStep whose Stager was closed raises instead of handing
+    the library a freed handle (checked with a fake library; nothing runs)."""
+    import torch
+
+    import dynamic_block_sparse_dsa_b200 as dsa
+
+    class FakeLib:
+        def __getattr__(self, name):
+            if name.endswith("_workspace_size"):
+                return lambda *a: 256
+            if name == "dsa_stager_create":
+                def create(n, s, out):
+                    out._obj.value = 0x1234
+                    return 0
+                return create
+            return lambda *a: 0
+
+    fake = FakeLib()
+    monkeypatch.setattr(dsa._lib, "load", lambda: fake)
+    monkeypatch.setattr(dsa, "load", lambda: fake)
+    monkeypatch.setattr(dsa, "_ptr", lambda t: None if t is None else ctypes.c_void_p(t.data_ptr() or 16))
+    monkeypatch.setattr(dsa, "_host_ptr", lambda t: t.data_ptr())
+
+    class FakeStream:
+        cuda_stream = 7
+
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda: FakeStream())
+    st = dsa.Stager(1, FakeStream())
+    ps = dsa.PreparedStep.__new__(dsa.PreparedStep)
+    ps.calls, ps.bufs, ps._stream = [], {}, ctypes.c_void_p(7)
+    ps._stager = st
+    ps._begin = ps._end = (lambda *a: 0, ())
+    assert ps() == {}
+    st.close()
+    with pytest.raises(ValueError):
+        ps()
