@@ -969,12 +969,12 @@ def main(argv=None):
     init_dist(world, "nccl")
     res, cases = run_ours(args, world, rank, device)
     wl = cases[0].wl
-    if rank == 0 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline:   # the CPU baseline and the extra records: one GPU only
         res["cpu_baseline"] = cpu_baseline(wl)
     del cases, wl
     torch.cuda.synchronize(device)
     torch.cuda.empty_cache()
-    if rank == 0 and not args.no_prefill:
+    if world == 1 and not args.no_prefill:
         res["prefill_indexer"] = prefill_indexer(device)
     if world == 1 and not args.no_configs:
         # the other workloads, one GPU: step time and each launch against its roofline
