@@ -48,8 +48,12 @@ constexpr int kRadixMinGroups = 2;
 constexpr bool kFinalRadix = false;
 }  // namespace
 
-template <int G>   // 64-block groups per warp: a chunk is kSelWarps * 64 * G blocks
-__global__ void __launch_bounds__(kSelThreads, 2) select_blocks_kernel(SelectArgs a) {
+// 64-block groups per warp: a chunk is kSelWarps * 64 * G blocks.  Chunks of
+// G >= 2 (many-query batches) run three CTAs per SM: measured faster than two
+// despite a few spilled registers (chunked prefill 189 -> 169 us), and than
+// keeping the keys in shared memory instead (198 us).
+template <int G>
+__global__ void __launch_bounds__(kSelThreads, G >= 2 ? 3 : 2) select_blocks_kernel(SelectArgs a) {
     __shared__ int4 s_q[kMaxIdxHeads][kIdxDim / 16];
     __shared__ int s_w[kMaxIdxHeads];
     __shared__ int s_cuq[kCuqCache + 1];
