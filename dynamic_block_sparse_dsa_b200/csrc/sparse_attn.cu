@@ -12,7 +12,12 @@
 // units u = (query t, KV head, selection slot j) -- one 64-token page slice of
 // K and of V (16 KiB each) -- and CTA c takes the contiguous range
 // [c*U/C, (c+1)*U/C), so every SM streams the same number of bytes whatever
-// the batch looks like.  Inside the CTA:
+// the batch looks like.  When every CTA takes whole (query, KV head) pairs
+// (prefill, and decode batches with many pairs) the pairs instead run
+// KV-head-major and interleaved over the CTAs -- CTA c takes pairs c, c + C,
+// ... of the order kvh * T + t -- so all CTAs read one KV head's slice of the
+// pool at a time and the queries that select the same block find it in L2.
+// Inside the CTA:
 //   * a producer warp walks the range and, for each selected block, issues four
 //     boxes of a 3-D TMA tensor map over the pool (K and V, two 128-byte halves
 //     each, SWIZZLE_128B, no multicast) into a 6-stage (5 for 16-head groups)
