@@ -358,3 +358,51 @@ def test_prepared_step_refuses_a_closed_stager(monkeypatch):
     st.close()
     with pytest.raises(ValueError):
         ps()
+
+
+def test_prepared_step_argument_checks(monkeypatch):
+    """Host buffers need a stager, slots must exist, staged pairs must match in
+    size (fake library; nothing runs)."""
+    import torch
+
+    import dynamic_block_sparse_dsa_b200 as dsa
+
+    class FakeLib:
+        def __getattr__(self, name):
+            if name.endswith("_workspace_size"):
+                return lambda *a: 256
+            if name == "dsa_stager_create":
+                def create(n, s, out):
+                    out._obj.value = 0x1234
+                    return 0
+                return create
+            return lambda *a: 0
+
+    fake = FakeLib()
+    monkeypatch.setattr(dsa._lib, "load", lambda: fake)
+    monkeypatch.setattr(dsa, "load", lambda: fake)
+
+    class FakeStream:
+        cuda_stream = 7
+
+    dev = torch.zeros(64, dtype=torch.uint8)
+    host = torch.zeros(64, dtype=torch.uint8)
+    host_short = torch.zeros(32, dtype=torch.uint8)
+    # the staged pairs are checked for size before any pointer is taken
+    monkeypatch.setattr(dsa, "_ptr", lambda t: ctypes.c_void_p(16))
+    with pytest.raises(ValueError):
+        dsa._regions([(dev, host_short)], False)
+    dst, src, nb, n = dsa._regions([(dev, host)], False)
+    assert n == 1 and nb[0] == 64
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda: FakeStream())
+    st = dsa.Stager(2, FakeStream())
+    monkeypatch.setattr(dsa, "step", lambda *a, **k: {})
+    with pytest.raises(ValueError):
+        dsa.PreparedStep(None, None, None, host_in=[(dev, host)])          # no stager
+    with pytest.raises(ValueError):
+        dsa.PreparedStep(None, None, None, stager=st, slot=2)               # no such slot
+    ps = dsa.PreparedStep(None, None, None, stager=st, slot=1, host_in=[(dev, host)], host_out=[(dev, host)])
+    with pytest.raises(ValueError):
+        ps(stream=FakeStream())                                             # staged steps run on the stager's stream
+    assert ps() == {}
+    st.close()
