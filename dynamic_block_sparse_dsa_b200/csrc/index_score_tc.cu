@@ -21,23 +21,25 @@
 // 128 coarse keys (the MMA's A operand, gathered through the block table) for
 // many query tiles.  Per item only asynchronous copies remain: one 3-D TMA box
 // of the 16 queries' rows (heads past H zero-filled) and one 2-D box of their
-// head weights.  Warps:
-//   0     loader.  It works through its items 32 at a time: the batch's query
+// head weights.  The CTA runs two independent pipelines, each on half of its
+// items with its own ring, A buffers and one 256-column accumulator, because
+// one loader warp's per-item chain (decide, wait for a stage, publish, issue
+// the copies) paced a single pipeline.  Warps of pipeline p:
+//   2p    loader.  It works through its items 32 at a time: the batch's query
 //         positions arrive in shared memory a batch ahead (cp.async), every
 //         lane then decides one item (its sequences, whether any of its blocks
 //         is visible), and a short loop publishes the visible items into a
 //         4-stage ring.  When the (sequence, block tile) changes it gathers the
 //         new tile (64-byte swizzle) into one of two A buffers, once the items
 //         still reading that buffer have finished;
-//   1     MMA issuer (one thread): two K = 32 MMAs per item into one of two
-//         256-column accumulators;
-//   2-17  epilogue, two groups of eight warps taking alternate items (and the
-//         two accumulators), so that one group's tensor-memory loads overlap
-//         the other's arithmetic; in a group the two warps of each SM
-//         sub-partition take that sub-partition's 32 rows and half of the
-//         queries each, in two rounds of four queries: tcgen05.ld, after the
-//         second of which the accumulator goes back to the MMA, then relu * w
-//         summed over heads and one coalesced 128-byte store per (query, warp).
+//   2p+1  MMA issuer (one thread): two K = 32 MMAs per item into the
+//         pipeline's 256-column accumulator;
+//   4+8p .. 11+8p  epilogue: the two warps of each SM sub-partition take that
+//         sub-partition's 32 rows and half of the queries each, in two rounds
+//         of four queries: tcgen05.ld, after the second of which the
+//         accumulator goes back to the MMA, then relu * w summed over heads and
+//         one coalesced 128-byte store per (query, warp).  The other
+//         pipeline's MMA and loads overlap this arithmetic.
 // A query tile spanning several sequences runs once per sequence with the
 // other queries masked; items past every query's own block are skipped.  All
 // waits are bounded.
@@ -50,11 +52,11 @@
 namespace dsa {
 
 namespace {
-constexpr int kEpiWarps = 16;                      // four per SM sub-partition
-constexpr int kLoadWarp = 0;
-constexpr int kMmaWarp = 1;
-constexpr int kEpiWarp0 = 2;
-constexpr int kTcThreads = 32 * (2 + kEpiWarps);   // loader, MMA, epilogue
+constexpr int kPipes = 2;                          // independent pipelines per CTA
+constexpr int kEpiWarps = 16;                      // four per SM sub-partition, eight per pipeline
+constexpr int kPipeEpi = kEpiWarps / kPipes;
+constexpr int kEpiWarp0 = 2 * kPipes;              // warps 2p and 2p + 1: pipeline p's loader and MMA
+constexpr int kTcThreads = 32 * (2 * kPipes + kEpiWarps);
 constexpr int kTcStages = 4;
 constexpr int kBT = 128;                 // blocks per tile (MMA M)
 constexpr int kQT = 16;                  // queries per tile (MMA N = 16 x 16 heads)
@@ -85,16 +87,18 @@ constexpr int kOffOwn = kOffPos + 2 * kBatch * kQT * 4;   // [2][kBatch][kQT] in
 constexpr int kWBytes = kQT * kMaxIdxHeads * 4;      // one tile's head weights
 // + alignment slack; at least 116 KiB so that two CTAs never share an SM (each
 // holds all 512 tensor-memory columns)
-constexpr int kSmemUsed = kOffOwn + 2 * kBatch * kQT * 4 + 1024;
+// one such layout per pipeline, kPipeBytes apart (the shared words of kOffMisc
+// are pipeline 0's)
+constexpr int kPipeBytes = (kOffOwn + 2 * kBatch * kQT * 4 + 1023) / 1024 * 1024;
+constexpr int kSmemUsed = kPipes * kPipeBytes + 1024;
 constexpr int kSmemBytes = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
 // full barrier: the loader's arrival with the TMA bytes, plus 32 cp.async
 // arrivals when the weights are copied by cp.async (H not a multiple of 4)
 constexpr int kFullCountTma = 1;
 constexpr int kFullCountCpAsync = 33;
 constexpr int kAFullCount = 33;                      // the loader: 32 cp.async arrivals + one
-constexpr int kEpiGroup = kEpiWarps / 2;             // epilogue warps per item (two groups alternate items)
-constexpr int kEmptyCount = 1 + kEpiGroup;           // MMA commit + the item's epilogue warps
-constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
+constexpr int kEmptyCount = 1 + kPipeEpi;            // MMA commit + the pipeline's epilogue warps
+constexpr uint32_t kTmemCols = 512;                  // one 256-column accumulator per pipeline
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 static_assert(kOffA % 1024 == 0, "A buffers keep the 64-byte swizzle's 512-byte alignment");
 static_assert(kOffPos % 16 == 0 && kOffOwn % 16 == 0, "positions and own blocks move in 16-byte pieces");
@@ -129,28 +133,28 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *g = smem_raw + (base - raw);
-    Bars bars{base};
-    // [0] tmem base, [1] abort, [2] never set
+    // [0] tmem base, [1] abort, [2] never set (shared by both pipelines)
     volatile int *misc = reinterpret_cast<volatile int *>(g + kOffMisc);
     volatile int *s_abort = misc + 1;
     const volatile int *s_never = misc + 2;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
-        for (int s = 0; s < kTcStages; ++s) {
-            mbar_init(bars.full(s), w_tma ? kFullCountTma : kFullCountCpAsync);
-            mbar_init(bars.empty(s), kEmptyCount);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(bars.tfull(b), 1);
-            mbar_init(bars.tempty(b), kEpiGroup);
-            mbar_init(bars.afull(b), kAFullCount);
+        for (int p = 0; p < kPipes; ++p) {
+            const Bars bp{base + (uint32_t)(p * kPipeBytes)};
+            for (int s = 0; s < kTcStages; ++s) {
+                mbar_init(bp.full(s), w_tma ? kFullCountTma : kFullCountCpAsync);
+                mbar_init(bp.empty(s), kEmptyCount);
+            }
+            mbar_init(bp.tfull(0), 1);
+            mbar_init(bp.tempty(0), kPipeEpi);
+            for (int b = 0; b < 2; ++b) mbar_init(bp.afull(b), kAFullCount);
         }
         misc[1] = 0;
         misc[2] = 0;
         fence_barrier_init();
     }
-    if (warp == kMmaWarp) {
+    if (warp == 1) {   // pipeline 0's MMA warp holds tensor memory for both
         tc::tmem_alloc(smem_u32(g + kOffMisc), kTmemCols);
         tc::tmem_relinquish();
     }
@@ -162,17 +166,24 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
     // item indices fit 32 bits (the host checks); only this split uses 64-bit products
     const unsigned n_items = (unsigned)n_bt * (unsigned)n_qt;
-    const unsigned i0 = (unsigned)((unsigned long long)n_items * blockIdx.x / gridDim.x);
-    const unsigned i1 = (unsigned)((unsigned long long)n_items * (blockIdx.x + 1) / gridDim.x);
+    const unsigned c0 = (unsigned)((unsigned long long)n_items * blockIdx.x / gridDim.x);
+    const unsigned c1 = (unsigned)((unsigned long long)n_items * (blockIdx.x + 1) / gridDim.x);
     const int H = a.num_idx_heads;
+    // the pipeline of this warp: the first or the second half of the CTA's items
+    const int pipe = warp < kEpiWarp0 ? (warp >> 1) : (warp - kEpiWarp0) / kPipeEpi;
+    const unsigned cmid = c0 + (c1 - c0 + 1) / 2;
+    const unsigned i0 = pipe == 0 ? c0 : cmid, i1 = pipe == 0 ? cmid : c1;
+    const uint32_t pbase = base + (uint32_t)(pipe * kPipeBytes);
+    uint8_t *gp = g + pipe * kPipeBytes;
+    const Bars bars{pbase};
 
-    if (warp == kLoadWarp) {
+    if (warp < kEpiWarp0 && !(warp & 1)) {
         // ============================================================ loader
         if (lane == 0) {
             prefetch_tensormap(&tm_q);
             if (w_tma) prefetch_tensormap(&tm_w);
         }
-        int *s_cuq = reinterpret_cast<int *>(g + kOffCuq);
+        int *s_cuq = reinterpret_cast<int *>(gp + kOffCuq);
         int *s_len = s_cuq + kSeqCache;
         const bool cached = a.num_seqs + 1 <= kSeqCache;
         if (cached) {
@@ -193,7 +204,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         auto seq_len = [&](int s) { return cached ? s_len[s] : __ldg(a.seq_lens + s); };
         // the query positions of items b0 .. b0+31 into buffer `buf` (16 bytes
         // per copy, zero past the last query); one commit group per batch
-        int *s_posb = reinterpret_cast<int *>(g + kOffPos);
+        int *s_posb = reinterpret_cast<int *>(gp + kOffPos);
         const uint32_t s_posb_u32 = smem_u32(s_posb);
         auto fetch_batch = [&](unsigned b0, int buf) {
 #pragma unroll
@@ -232,7 +243,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         pdl_wait();   // coarse keys may come from the preceding append
         fetch_batch(i0, 0);
         fetch_batch(i0 + kBatch, 1);
-        int *s_own = reinterpret_cast<int *>(g + kOffOwn);
+        int *s_own = reinterpret_cast<int *>(gp + kOffOwn);
         int k = 0;          // items published
         int a_s = -1, a_bt = -1, ab = 1;
         int agen0 = 0, agen1 = 0, alast0 = -1, alast1 = -1;   // per A buffer: fill number, last item
@@ -248,10 +259,11 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // cannot be confused with item j + 4's, which waits for this very
         // barrier before it is published (j < k - 4 is known finished already).
         int k_seen = -1;   // the latest item known to be finished
-        // Two epilogue groups take alternate items, each in order: items j and
-        // j - 1 finished mean every item before them is.  When item k is
-        // published, item k - 5 is known finished (the wait for item k - 1's
-        // stage), so neither wait below can meet a reused stage's later phase.
+        // The pipeline's epilogue warps take its items in order, so item j
+        // finished means every item before it is (the wait on j - 1 as well
+        // costs nothing then).  When item k is published, item k - 5 is known
+        // finished (the wait for item k - 1's stage), so neither wait below can
+        // meet a reused stage's later phase.
         auto wait_done = [&](int end) {
             const int j = end - 1;
             if (j <= k_seen) return true;
@@ -367,7 +379,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                             const int b = bt * kBT + 32 * j + lane;
                             page[j] = b < n_blocks && b < a.max_blocks ? __ldg(row + b) : -1;
                         }
-                        const uint32_t sa = base + kOffA + ab * kABytes;
+                        const uint32_t sa = pbase + kOffA + ab * kABytes;
 #pragma unroll
                         for (int j = 0; j < kBT / 32; ++j) {
                             const int b = bt * kBT + 32 * j + lane;
@@ -396,7 +408,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         stop = true;
                         break;
                     }
-                    const uint32_t sb = base + st * kStageBytes;
+                    const uint32_t sb = pbase + st * kStageBytes;
                     if (!w_tma) {
                         // the tile's head weights (16 queries x 16 heads, zero past H and the last query)
 #pragma unroll
@@ -409,7 +421,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     }
                     __syncwarp();   // the own blocks written above, before the release arrival
                     if (lane == 0) {
-                        int4 *info = reinterpret_cast<int4 *>(g + st * kStageBytes + kOffInfo);
+                        int4 *info = reinterpret_cast<int4 *>(gp + st * kStageBytes + kOffInfo);
                         info[0] = make_int4(bt, y, ab | ((ab ? agen1 : agen0) << 1), mask);
                         info[1] = ab ? make_int4((int)vb1[0], (int)vb1[1], (int)vb1[2], (int)vb1[3])
                                      : make_int4((int)vb0[0], (int)vb0[1], (int)vb0[2], (int)vb0[3]);
@@ -429,13 +441,13 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             fetch_batch(b0 + 2 * kBatch, pbuf);
             if (*s_abort) stop = true;
         }
-        // two end markers: one for each epilogue group
-        for (int e = 0; e < 2 && !stop && !*s_abort; ++e) {
+        // the end marker (the pipeline's epilogue warps all read every item)
+        for (int e = 0; e < 1 && !stop && !*s_abort; ++e) {
             const int st = k & (kTcStages - 1);
             if (k >= kTcStages && !mbar_wait(bars.empty(st), ((k / kTcStages) - 1) & 1, s_abort)) {
                 *s_abort = 1;
             } else {
-                StageInfo *info = reinterpret_cast<StageInfo *>(g + st * kStageBytes + kOffInfo);
+                StageInfo *info = reinterpret_cast<StageInfo *>(gp + st * kStageBytes + kOffInfo);
                 if (lane == 0) info->bt = -1;
                 if (!w_tma) tc::cp_async_arrive_noinc(bars.full(st));
                 __syncwarp();
@@ -452,73 +464,71 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             for (int j = max(0, k - kTcStages); j < k; ++j)
                 mbar_wait(bars.full(j % kTcStages), (j / kTcStages) & 1, s_never);
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp < kEpiWarp0) {
         // ============================================================ MMA issuer
         constexpr uint32_t idesc = tc::idesc_i8(kBT, kN);
-        int k = 0, n_end = 0;
+        int k = 0;
         while (true) {
-            const int st = k % kTcStages, buf = k & 1;
+            const int st = k % kTcStages;
             bool ok = mbar_wait(bars.full(st), (k / kTcStages) & 1, s_abort);
-            const StageInfo *info = reinterpret_cast<const StageInfo *>(g + st * kStageBytes + kOffInfo);
+            const StageInfo *info = reinterpret_cast<const StageInfo *>(gp + st * kStageBytes + kOffInfo);
             const bool end = ok && info->bt < 0;
             const int abw = ok ? info->abw : 0;
             if (ok && !end) ok = mbar_wait(bars.afull(abw & 1), ((abw >> 1) - 1) & 1, s_abort);
             // the accumulator's previous item has been read (the end marker's
             // arrival on tfull must not run two phases ahead of the epilogue)
-            if (ok && k >= 2) ok = mbar_wait(bars.tempty(buf), ((k >> 1) - 1) & 1, s_abort);
+            if (ok && k >= 1) ok = mbar_wait(bars.tempty(0), (k - 1) & 1, s_abort);
             if (!ok) {
                 if (lane == 0) *s_abort = 1;
                 break;
             }
             if (lane == 0) {
                 if (end) {
-                    mbar_arrive(bars.tfull(buf));   // wake the epilogue to see the end marker
+                    mbar_arrive(bars.tfull(0));   // wake the epilogue to see the end marker
                 } else {
                     tc::fence_proxy_async_smem();   // the cp.async-written keys, for the tensor core
                     tc::fence_after_sync();
-                    const uint32_t sa = base + kOffA + (abw & 1) * kABytes;
-                    const uint32_t sb = base + st * kStageBytes;
-                    const uint32_t d = tmem + (uint32_t)(buf * kN);
+                    const uint32_t sa = pbase + kOffA + (abw & 1) * kABytes;
+                    const uint32_t sb = pbase + st * kStageBytes;
+                    const uint32_t d = tmem + (uint32_t)(pipe * kN);
                     const uint64_t da = tc::smem_desc_k64_sw64(sa), db = tc::smem_desc_k64_sw64(sb);
                     tc::mma_i8(d, da, db, idesc, false);
                     tc::mma_i8(d, da + (32 >> 4), db + (32 >> 4), idesc, true);   // K bytes 32..63
                     tc::commit(bars.empty(st));
-                    tc::commit(bars.tfull(buf));
+                    tc::commit(bars.tfull(0));
                 }
             }
             __syncwarp();
             ++k;
-            if (end && ++n_end == 2) break;
+            if (end) break;
         }
         // the last MMAs have completed before the accumulator is released
         if (lane == 0 && k > 0) {
             const int j = k - 1;
-            mbar_wait(bars.tfull(j & 1), (j >> 1) & 1, s_never);
+            mbar_wait(bars.tfull(0), j & 1, s_never);
         }
     } else {
         // ============================================================ epilogue
-        // two groups of 8 warps take alternate items (group g: items g, g+2, ...,
-        // accumulator g), so one group's tensor-memory loads overlap the other's
-        // arithmetic.  In a group, the two warps of a sub-partition take the
-        // 32 rows that sub-partition can read and half of the 16 queries each,
-        // in two rounds of 4 queries (64 accumulator columns).
+        // the pipeline's 8 warps take each of its items; the two warps of a
+        // sub-partition take the 32 rows that sub-partition can read and half
+        // of the 16 queries each, in two rounds of 4 queries (64 accumulator
+        // columns of the pipeline's accumulator)
         const int ew = warp - kEpiWarp0;
-        const int grp = ew >> 3;                 // items of parity grp
         const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
         const int half = (ew >> 2) & 1;          // queries 8*half .. +7
         const int row = quarter * 32 + lane;     // block row of the tile
-        const int *s_own_e = reinterpret_cast<const int *>(g + kOffOwn);
-        int k = grp;
+        const int *s_own_e = reinterpret_cast<const int *>(gp + kOffOwn);
+        int k = 0;
         while (true) {
-            const int st = k % kTcStages, buf = k & 1;
-            bool ok = mbar_wait(bars.tfull(buf), (k >> 1) & 1, s_abort) &&
+            const int st = k % kTcStages;
+            bool ok = mbar_wait(bars.tfull(0), k & 1, s_abort) &&
                       mbar_wait(bars.full(st), (k / kTcStages) & 1, s_abort);   // acquire the info words
             if (!ok) {
                 if (lane == 0) *s_abort = 1;
                 break;
             }
             tc::fence_after_sync();
-            const StageInfo *info = reinterpret_cast<const StageInfo *>(g + st * kStageBytes + kOffInfo);
+            const StageInfo *info = reinterpret_cast<const StageInfo *>(gp + st * kStageBytes + kOffInfo);
             const int4 i0w = *reinterpret_cast<const int4 *>(info);
             if (i0w.x < 0) break;   // the end marker
             const int bt = i0w.x, y = i0w.y, mask = i0w.w;
@@ -529,7 +539,7 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             for (int rnd = 0; rnd < 2; ++rnd) {
                 const int qgrp = 2 * half + rnd;   // queries 4*qgrp .. +3 (columns 64*qgrp ..)
                 const uint32_t taddr =
-                    tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kN + qgrp * 64);
+                    tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(pipe * kN + qgrp * 64);
                 tc::ld_32x32b_x32(taddr, v[0]);
                 tc::ld_32x32b_x32(taddr + 32, v[1]);
                 tc::wait_ld();
@@ -537,12 +547,12 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     // the accumulator is all in registers: release it to the next MMA
                     tc::fence_before_sync();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bars.tempty(buf));
+                    if (lane == 0) mbar_arrive(bars.tempty(0));
                 }
                 const int4 o4 = *reinterpret_cast<const int4 *>(s_own_e + info->own_off + 4 * qgrp);
                 const int own4[4] = {(mask >> (4 * qgrp)) & 1 ? o4.x : -1, (mask >> (4 * qgrp + 1)) & 1 ? o4.y : -1,
                                      (mask >> (4 * qgrp + 2)) & 1 ? o4.z : -1, (mask >> (4 * qgrp + 3)) & 1 ? o4.w : -1};
-                const int4 *w4 = reinterpret_cast<const int4 *>(g + st * kStageBytes + kOffW) + qgrp * kMaxIdxHeads;
+                const int4 *w4 = reinterpret_cast<const int4 *>(gp + st * kStageBytes + kOffW) + qgrp * kMaxIdxHeads;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {   // query 4*qgrp + u: columns 16u .. 16u+15 of these 64
                     const uint32_t *x = v[u >> 1] + 16 * (u & 1);
@@ -560,13 +570,13 @@ index_score_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bars.empty(st));   // the stage (info, weights, own blocks) is read
-            k += 2;
+            ++k;
         }
     }
 
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (warp == 1) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
     }
