@@ -42,6 +42,11 @@
  *    k_per_seq, q_idx, w, q): these must not be outputs of the library call
  *    issued just before it on the same stream.  Work from other kernels is
  *    waited for in full, as usual.
+ *  - Calls on different streams may run at the same time (independent
+ *    batches in flight, one stream each) as long as no call writes what
+ *    another reads or writes: each needs its own outputs and workspaces.  The
+ *    library keeps no device state between calls apart from the fixed
+ *    scratch of dsa_sparse_attn_decode_noalloc.
  *
  * KV cache layout [P5 "KV Cache Layout"; P1 4(2) two storage types]:
  *   k_pool, v_pool : bf16  [num_pages][block_size][num_kv_heads][head_dim]
