@@ -43,3 +43,17 @@ def test_chunked_prefill_indexer_ops():
     ab = bench.algorithmic_bytes(_W(spec))
     # every query selects 64 blocks of its ~2080 visible ones
     assert ab["kv"] == spec.n_new[0] * 64 * 8 * (64 * 128 * 2) * 2
+
+
+def test_overlapped_record_arithmetic(monkeypatch):
+    """The overlapped-batches record turns its measured seconds per step into
+    tokens/s and a fraction of the peak over the step's algorithmic bytes."""
+    spec = wk.decode_1m()
+    ab = bench.algorithmic_bytes(_W(spec))
+    monkeypatch.setattr(bench, "time_overlapped", lambda cases, stream, device, steps: (20e-6, 240))
+    rec = bench.overlapped_record([None] * 3, spec, ab, None, None, 200, 6450.3)
+    assert rec["batches_in_flight"] == 3 and rec["steps_timed"] == 240
+    assert rec["ms_per_step"] == 0.02
+    assert rec["tokens_per_s"] == 400_000.0   # 8 queries per step
+    assert rec["step_gbs"] == round(75_497_472 / 20e-6 / 1e9, 1) == 3774.9
+    assert rec["step_frac_of_measured"] == round(3774.8736 / 6450.3, 4)
