@@ -11,7 +11,9 @@ step traffic together exceeds the L2 by half, so no step finds its data in L2;
 the K steps are timed with one pair of CUDA events on the launching stream.
 Workloads too small for that are timed one step at a time after a cold-L2
 flush (512 MiB written, then 256 MiB read so no dirty lines remain), which is
-also reported for the first batch as the isolated step time.
+also reported for the first batch as the isolated step time.  Decode lines
+also carry an `overlapped` record: the same batches all in flight at once,
+each on a stream of its own (a serving schedule; not part of `value`).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun every rank runs its own batch (weak scaling, no collective on
